@@ -1,0 +1,140 @@
+"""Seeded synthetic inputs for the Gated DeltaNet-2 operator.
+
+This module is shared by the tests, the benchmark and the smoke check, and by
+both sides of every parity comparison (the CUDA library and the fp64 oracle).
+It holds only the input recipe -- random draws and the pre-processing a layer
+applies before the operator (L2-normalised q/k, SiLU values, sigmoid gates,
+negative log-decay) -- and none of the operator's own arithmetic.
+
+Recipe (all draws on a CPU ``torch.Generator`` seeded per case, in the order
+q, k, v, b, w, log_alpha, S0):
+  * q, k ~ N(0, 1) in fp32, L2-normalised over the head dimension per
+    (batch, token, head), then cast to the input dtype;
+  * v = SiLU(N(0, 1));
+  * b (dk channels) and w (dv channels) = sigmoid(N(0, sigma_gate));
+  * log_alpha = -exp(U(lo, hi)), fp32, one value per token and key channel;
+  * S0 = 0, or N(0, sigma_s0) in fp32.
+The shapes follow the layer described on the pages: 16 heads with a 128 x 128
+state per head and a 4K training context ("Gated DeltaNet-2" on iplexlaw.co.kr,
+section "Condiciones de comparación"), stand-ins for the FineWeb-Edu
+activations of a trained 1.3B model, which are not available here.
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass
+
+import torch
+
+
+@dataclass(frozen=True)
+class FwdCase:
+    name: str
+    B: int
+    T: int
+    H: int
+    dk: int
+    dv: int
+    dtype: torch.dtype
+    seed: int
+    log_alpha_range: tuple = (-5.0, -1.0)
+    gate_sigma: float = 1.0
+    s0_sigma: float = 0.0  # 0 => zero initial state
+
+
+@dataclass(frozen=True)
+class DecodeCase:
+    name: str
+    B: int
+    H: int
+    dk: int
+    dv: int
+    steps: int
+    dtype: torch.dtype = torch.float32
+    seed: int = 4
+    state_sigma: float = 0.05
+    step_seed_base: int = 4_000_000
+
+
+# The five workloads of the operator (sizes, distributions and seeds).
+ORACLE_FP32 = FwdCase("oracle_fp32_B1_H2_T256_d64", 1, 256, 2, 64, 64, torch.float32, seed=0)
+LAYER_BF16 = FwdCase("layer_bf16_B1_H16_T4096_d128", 1, 4096, 16, 128, 128, torch.bfloat16, seed=1)
+TRAIN_BF16 = FwdCase("train_bf16_B8_H16_T4096_d128", 8, 4096, 16, 128, 128, torch.bfloat16, seed=2,
+                     s0_sigma=0.02)
+LONG_BF16 = FwdCase("long_bf16_B1_H16_T65536_d128", 1, 65536, 16, 128, 128, torch.bfloat16, seed=3,
+                    log_alpha_range=(-9.0, 0.0), gate_sigma=2.0)
+DECODE_F32 = DecodeCase("decode_f32_B256_H16_d128_1000steps", 256, 16, 128, 128, steps=1000)
+
+FWD_CASES = {c.name: c for c in (ORACLE_FP32, LAYER_BF16, TRAIN_BF16, LONG_BF16)}
+
+
+def _l2norm(x: torch.Tensor) -> torch.Tensor:
+    return x / x.norm(dim=-1, keepdim=True).clamp_min(1e-12)
+
+
+def draw_fwd(B, T, H, dk, dv, *, seed, dtype=torch.float32, log_alpha_range=(-5.0, -1.0),
+             gate_sigma=1.0, s0_sigma=0.0, with_s0=None):
+    """Draw one forward batch.  Returns a dict of CPU tensors.
+
+    q, k, v, b, w are in ``dtype``; log_alpha and S0 are fp32.  ``S0`` is None
+    when ``s0_sigma == 0`` unless ``with_s0`` forces a zero tensor.
+    """
+    g = torch.Generator(device="cpu").manual_seed(int(seed))
+    q = _l2norm(torch.randn(B, T, H, dk, generator=g))
+    k = _l2norm(torch.randn(B, T, H, dk, generator=g))
+    v = torch.nn.functional.silu(torch.randn(B, T, H, dv, generator=g))
+    b = torch.sigmoid(gate_sigma * torch.randn(B, T, H, dk, generator=g))
+    w = torch.sigmoid(gate_sigma * torch.randn(B, T, H, dv, generator=g))
+    lo, hi = log_alpha_range
+    u = torch.rand(B, T, H, dk, generator=g) * (hi - lo) + lo
+    log_alpha = -torch.exp(u)
+    if s0_sigma > 0:
+        S0 = s0_sigma * torch.randn(B, H, dk, dv, generator=g)
+    elif with_s0:
+        S0 = torch.zeros(B, H, dk, dv)
+    else:
+        S0 = None
+    out = dict(q=q, k=k, v=v, b=b, w=w)
+    out = {n: t.to(dtype).contiguous() for n, t in out.items()}
+    out["log_alpha"] = log_alpha.contiguous()
+    out["S0"] = S0
+    return out
+
+
+def draw_case(case: FwdCase, *, T=None, B=None, seed=None):
+    """Draw a workload's inputs, optionally at a different T/B/seed."""
+    return draw_fwd(B or case.B, T or case.T, case.H, case.dk, case.dv,
+                    seed=case.seed if seed is None else seed, dtype=case.dtype,
+                    log_alpha_range=case.log_alpha_range, gate_sigma=case.gate_sigma,
+                    s0_sigma=case.s0_sigma)
+
+
+def draw_decode_state(case: DecodeCase, B=None):
+    g = torch.Generator(device="cpu").manual_seed(int(case.seed))
+    return case.state_sigma * torch.randn(B or case.B, case.H, case.dk, case.dv, generator=g)
+
+
+def draw_decode_token(case: DecodeCase, step: int, B=None):
+    """Per-token decode inputs for one step ([B,H,d]); drawn like the fp32 forward case."""
+    d = draw_fwd(B or case.B, 1, case.H, case.dk, case.dv, seed=case.step_seed_base + step,
+                 dtype=case.dtype)
+    return {n: (t[:, 0].contiguous() if t is not None else None) for n, t in d.items()
+            if n != "S0"}
+
+
+def draw_fwd_device(B, T, H, dk, dv, *, seed, device, dtype=torch.bfloat16,
+                    log_alpha_range=(-5.0, -1.0), gate_sigma=1.0):
+    """Same recipe drawn with a device generator (for timing-only buffers)."""
+    g = torch.Generator(device=device).manual_seed(int(seed))
+
+    def rn(*s):
+        return torch.randn(*s, generator=g, device=device)
+    q = _l2norm(rn(B, T, H, dk))
+    k = _l2norm(rn(B, T, H, dk))
+    v = torch.nn.functional.silu(rn(B, T, H, dv))
+    b = torch.sigmoid(gate_sigma * rn(B, T, H, dk))
+    w = torch.sigmoid(gate_sigma * rn(B, T, H, dv))
+    lo, hi = log_alpha_range
+    u = torch.rand(B, T, H, dk, generator=g, device=device) * (hi - lo) + lo
+    out = {n: t.to(dtype).contiguous() for n, t in dict(q=q, k=k, v=v, b=b, w=w).items()}
+    out["log_alpha"] = (-torch.exp(u)).contiguous()
+    return out

@@ -1,0 +1,28 @@
+"""The chunkwise WY algebra used by the kernels equals the token recurrence."""
+import numpy as np
+import pytest
+
+import oracle
+from oracle_pins import _inputs
+from wy_model import wy_forward
+
+
+@pytest.mark.parametrize("C", [1, 2, 4, 16, 64])
+def test_wy_model_matches_oracle(C):
+    q, k, v, b, w, la, s0 = _inputs(150, 8, 6, seed=200 + C, B=1, H=2)
+    o_ref, s_ref = oracle.fwd(q, k, v, b, w, la, S0=s0)
+    o, s = wy_forward(q, k, v, b, w, la, S0=s0, C=C)
+    scale = np.abs(o_ref).max()
+    assert np.abs(o - o_ref).max() <= 1e-12 * scale
+    assert np.abs(s - s_ref).max() <= 1e-12 * np.abs(s_ref).max()
+
+
+def test_wy_model_strong_decay_and_wide_erase():
+    """Long-context decay range (log alpha down to -1) and erase gates in [0, 2]."""
+    r = np.random.default_rng(7)
+    q, k, v, b, w, _, s0 = _inputs(200, 16, 8, seed=8)
+    la = -np.exp(r.uniform(-9.0, 0.0, q.shape))
+    o_ref, s_ref = oracle.fwd(q, k, v, 2 * b, w, la, S0=s0)
+    o, s = wy_forward(q, k, v, 2 * b, w, la, S0=s0, C=64)
+    assert np.abs(o - o_ref).max() <= 1e-11 * np.abs(o_ref).max()
+    assert np.abs(s - s_ref).max() <= 1e-11 * np.abs(s_ref).max()
