@@ -1,0 +1,349 @@
+#!/usr/bin/env python
+"""Benchmark of the Gated DeltaNet-2 operator on B200.
+
+One step = one gdn2_fwd_chunked call over the 1.3B-layer workload (B=1, H=16,
+T=4096, dk=dv=128, bf16 inputs, fp32 decay and state, chunk 64).  The same
+run also times gdn2_decode_step on the decode workload (B=256, H=16, d=128,
+fp32 state of 268 MB updated in place) and reports its HBM bandwidth.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+N > 1 runs N independent replicas (the operator is independent per
+(batch, head); there is no exchange step), one process per GPU, launched by
+torch.distributed.run.  Rank 0 prints one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+from pathlib import Path
+
+import torch
+
+ROOT = Path(__file__).resolve().parent
+sys.path.insert(0, str(ROOT))
+
+import synth  # noqa: E402
+
+FALLBACK_HBM_GBS = 6650.0
+METRIC = "tokens/s of GDN-2 fwd (H=16,dk=dv=128) + % roofline; decode HBM GB/s"
+CASE = synth.LAYER_BF16
+DEC = synth.DECODE_F32
+N_INPUT_SETS = 4  # rotating input sets: 4 x 136 MB > 126 MB of L2
+
+# dram__bytes_read.sum + dram__bytes_write.sum per launch from an ncu capture of
+# the current kernels (None once a kernel has changed since the capture).
+NCU_TRAFFIC_BYTES = {"fwd": None, "decode": None}
+
+
+def peaks():
+    p = ROOT / "MEASURED_PEAKS.json"
+    if p.exists():
+        d = json.loads(p.read_text())
+        return float(d["hbm_gbs"]), "measured"
+    return FALLBACK_HBM_GBS, "fallback"
+
+
+def fwd_algorithmic_bytes(B, T, H, dk, dv, s_in, s_out, has_s0, has_st):
+    per_head_token = (3 * dk + 2 * dv) * s_in + 4 * dk + dv * s_out
+    state = B * H * dk * dv * 4
+    return B * T * H * per_head_token + state * (int(has_s0) + int(has_st))
+
+
+def decode_algorithmic_bytes(B, H, dk, dv, s_in=4, s_out=4):
+    # state read + written once, q,k,b (dk) and v,w (dv) in the input dtype,
+    # log_alpha fp32, o in the input dtype
+    return B * H * (2 * dk * dv * 4 + (3 * dk + 2 * dv) * s_in + 4 * dk + dv * s_out)
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.t0 = self.t1 = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (FileNotFoundError, OSError):
+            self.proc = None
+
+    def mark(self, which):
+        setattr(self, which, time.time())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        out, _ = self.proc.communicate(timeout=10)
+        rows = [r.split(", ") for r in out.strip().splitlines() if r.count(",") >= 8]
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].strip() == "Active"})
+        load = sorted(sm)[len(sm) // 2:] if sm else []
+        return {"sm_mhz": statistics.median(load) if load else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons, "samples": len(rows)}
+
+
+def dist_setup(args):
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if ws > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    return ws, rank, local
+
+
+def barrier(ws):
+    if ws > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, ws: int) -> float:
+    if ws == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], device="cuda", dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def cpu_oracle_tokens_per_s(sample_T: int, heads: int):
+    """Oracle (fp64, OpenMP over heads) on a bounded sample of the workload."""
+    import oracle
+    d = synth.draw_fwd(1, sample_T, heads, CASE.dk, CASE.dv, seed=CASE.seed, dtype=CASE.dtype,
+                       log_alpha_range=CASE.log_alpha_range, gate_sigma=CASE.gate_sigma)
+    args = [d[n] for n in ("q", "k", "v", "b", "w", "log_alpha")]
+    orc = oracle.load()
+    cores = orc.max_threads()
+    t = time.perf_counter()
+    orc.fwd(*args, S0=None)
+    dt = time.perf_counter() - t
+    return sample_T * heads / dt, cores, dt
+
+
+def run_reference(args, ws, rank):
+    """The oracle timed as it stands; each step a bounded sample of the workload."""
+    if rank != 0:
+        return
+    heads = CASE.H
+    rate, cores, _ = cpu_oracle_tokens_per_s(256, heads)          # calibration
+    per_step_s = 120.0 / (args.steps + args.warmup)                # whole run ~2 min
+    T = int(max(64, min(CASE.T, per_step_s * rate / heads)))
+    vals = []
+    for i in range(args.warmup + args.steps):
+        v, cores, dt = cpu_oracle_tokens_per_s(T, heads)
+        if i >= args.warmup:
+            vals.append(v)
+    value = statistics.median(vals)
+    sample = (f"per step B=1 H={heads} T={T} d=128 of the B=1 H=16 T=4096 workload, fp64, "
+              f"OpenMP over heads")
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+            "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": CASE.B * CASE.T * CASE.H / value * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": CASE.name, "B": 1, "T": CASE.T, "H": heads, "dk": 128,
+                       "dv": 128, "chunk": 64},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=400)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--decode-steps", type=int, default=1000)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    if args.impl == "reference":
+        ws = int(os.environ.get("WORLD_SIZE", "1"))
+        rank = int(os.environ.get("RANK", "0"))
+        run_reference(args, ws, rank)
+        return
+
+    import gated_delta_rule_118_b200 as g
+    ws, rank, local = dist_setup(args)
+    dev = torch.device("cuda", torch.cuda.current_device())
+    stream = torch.cuda.current_stream()
+    hbm_peak, peak_kind = peaks()
+
+    # ---------------- chunked forward: device-resident inputs ----------------
+    c = CASE
+    sets = [synth.draw_fwd_device(c.B, c.T, c.H, c.dk, c.dv, seed=100 * rank + i, device=dev,
+                                  dtype=c.dtype, log_alpha_range=c.log_alpha_range,
+                                  gate_sigma=c.gate_sigma) for i in range(N_INPUT_SETS)]
+    o = torch.empty(c.B, c.T, c.H, c.dv, dtype=c.dtype, device=dev)
+    S_T = torch.empty(c.B, c.H, c.dk, c.dv, dtype=torch.float32, device=dev)
+    names = ("q", "k", "v", "b", "w", "log_alpha")
+
+    def step(i):
+        d = sets[i % N_INPUT_SETS]
+        g.gdn2_fwd_chunked(*(d[n] for n in names), S0=None, o=o, S_T=S_T, check=False)
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    if g.gdn2_check_device_error() != g.GDN2_OK:
+        raise RuntimeError("device error during warm-up")
+
+    clocks = ClockSampler(local)
+    clocks.start()
+    # soak so the clock sampler sees the GPU under load before the timed region
+    soak_end = time.time() + 1.0
+    i = 0
+    while time.time() < soak_end:
+        step(i); i += 1
+        if i % 50 == 0:
+            torch.cuda.synchronize()
+    torch.cuda.synchronize()
+
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    barrier(ws)
+    torch.cuda.synchronize()
+    t_all0 = torch.cuda.Event(enable_timing=True)
+    t_all1 = torch.cuda.Event(enable_timing=True)
+    t_all0.record(stream)
+    for i in range(args.steps):
+        ev[i][0].record(stream)
+        step(i)
+        ev[i][1].record(stream)
+    t_all1.record(stream)
+    torch.cuda.synchronize()
+    barrier(ws)
+    clk = clocks.stop()
+    total_ms = max_over_ranks(t_all0.elapsed_time(t_all1), ws)
+    launch_ms = [a.elapsed_time(b) for a, b in ev]
+    mean_launch_ms = sum(launch_ms) / len(launch_ms)
+    if g.gdn2_check_device_error() != g.GDN2_OK:
+        raise RuntimeError("device error during the timed region")
+
+    tokens_per_step = c.B * c.T * c.H
+    value = tokens_per_step * args.steps * ws / (total_ms / 1e3)
+    alg_bytes = fwd_algorithmic_bytes(c.B, c.T, c.H, c.dk, c.dv, 2, 2, False, True)
+    achieved = alg_bytes / (mean_launch_ms / 1e3) / 1e9
+
+    # ---------------- end to end through the C ABI with host buffers ----------------
+    host = {n: sets[0][n].cpu().pin_memory() for n in names}
+    dev_in = {n: torch.empty_like(sets[0][n]) for n in names}
+    o_host = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = o_host.numel() * o_host.element_size()
+    e2e_steps = max(3, min(args.steps, 20))
+
+    def e2e_step():
+        for n in names:
+            dev_in[n].copy_(host[n], non_blocking=True)
+        g.gdn2_fwd_chunked(*(dev_in[n] for n in names), S0=None, o=o, S_T=S_T, check=False)
+        o_host.copy_(o, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize()
+    barrier(ws)
+    e0 = torch.cuda.Event(enable_timing=True); e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), ws)
+    e2e_value = tokens_per_step * e2e_steps * ws / (e2e_ms / 1e3)
+    del sets, host, dev_in
+
+    # ---------------- decode: fp32 state resident in HBM, in place ----------------
+    dc = DEC
+    S = 0.05 * torch.randn(dc.B, dc.H, dc.dk, dc.dv, device=dev)
+    tok_sets = []
+    for i in range(8):
+        dd = synth.draw_fwd_device(dc.B, 1, dc.H, dc.dk, dc.dv, seed=7000 + i, device=dev,
+                                   dtype=torch.float32)
+        tok_sets.append({n: dd[n][:, 0].contiguous() for n in names})
+    od = torch.empty(dc.B, dc.H, dc.dv, device=dev)
+    for i in range(5):
+        x = tok_sets[i % 8]
+        g.gdn2_decode_step(*(x[n] for n in names), S, o=od, check=False)
+    torch.cuda.synchronize()
+    barrier(ws)
+    d0 = torch.cuda.Event(enable_timing=True); d1 = torch.cuda.Event(enable_timing=True)
+    d0.record(stream)
+    for i in range(args.decode_steps):
+        x = tok_sets[i % 8]
+        g.gdn2_decode_step(*(x[n] for n in names), S, o=od, check=False)
+    d1.record(stream)
+    torch.cuda.synchronize()
+    dec_ms = max_over_ranks(d0.elapsed_time(d1), ws) / args.decode_steps
+    dec_bytes = decode_algorithmic_bytes(dc.B, dc.H, dc.dk, dc.dv)
+    dec_gbs = dec_bytes / (dec_ms / 1e3) / 1e9
+    if g.gdn2_check_device_error() != g.GDN2_OK:
+        raise RuntimeError("device error during decode timing")
+
+    # ---------------- CPU baseline (oracle) on rank 0, N = 1 ----------------
+    cpu = None
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        v, cores, dt = cpu_oracle_tokens_per_s(c.T, c.H)
+        cpu = {"value": v, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+               "sample": f"the whole workload (B=1 H=16 T=4096 d=128, 65,536 head-tokens), fp64, "
+                         f"{dt:.1f} s"}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": ws,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_ms / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic",
+            "config": {"workload": c.name, "B": c.B, "T": c.T, "H": c.H, "dk": c.dk, "dv": c.dv,
+                       "chunk": 64, "inputs": "bf16 q,k,v,b,w; fp32 log_alpha; fp32 state",
+                       "l2": f"rotating {N_INPUT_SETS} device input sets "
+                             f"({N_INPUT_SETS * alg_bytes / 1e6:.0f} MB > 126 MB L2)",
+                       "replicas": ws},
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
+                         "frac": achieved / hbm_peak, "traffic": NCU_TRAFFIC_BYTES["fwd"],
+                         "peak_kind": peak_kind, "algorithmic_bytes_per_launch": alg_bytes,
+                         "mean_launch_us": mean_launch_ms * 1e3, "kernel": "gdn2_fwd_chunked"},
+            "decode": {"workload": dc.name, "us_per_step": dec_ms * 1e3, "hbm_gbs": dec_gbs,
+                       "frac": dec_gbs / hbm_peak, "peak": hbm_peak,
+                       "algorithmic_bytes_per_step": dec_bytes, "steps": args.decode_steps,
+                       "traffic": NCU_TRAFFIC_BYTES["decode"],
+                       "l2": "state 268 MB > 126 MB L2, streamed every step"},
+            "cpu_baseline": cpu,
+            "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h, "steps": e2e_steps},
+            "gpu_launches": args.steps,
+            "clocks": clk,
+        }
+        print(json.dumps(line), flush=True)
+    if ws > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

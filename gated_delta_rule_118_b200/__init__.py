@@ -1,0 +1,132 @@
+"""Gated DeltaNet-2 operator on B200: Python binding of libgdn2.so.
+
+The binding only marshals torch tensors (device memory) and the current CUDA
+stream into the C ABI declared in ``include/gdn2.h``; every step of the
+operator runs in the library's CUDA kernels.  There is no CPU fallback: if the
+native library is missing or cannot be loaded, every call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+from pathlib import Path
+
+import torch
+
+_PKG = Path(__file__).resolve().parent
+LIBRARY_PATH = _PKG / "libgdn2.so"
+
+GDN2_OK = 0
+GDN2_ERR_NULL = 1
+GDN2_ERR_SHAPE = 2
+GDN2_ERR_DTYPE = 3
+GDN2_ERR_ALIGN = 4
+GDN2_ERR_UNSUPPORTED = 5
+GDN2_ERR_CUDA = 6
+GDN2_ERR_DEVICE_TIMEOUT = 7
+GDN2_ERR_RANGE = 8
+
+GDN2_F32 = 0
+GDN2_BF16 = 1
+
+# Every symbol include/gdn2.h declares.
+EXPORTED = ("gdn2_fwd_chunked", "gdn2_decode_step", "gdn2_check_device_error",
+            "gdn2_status_string")
+
+_lib = None
+
+
+class Gdn2Error(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {status_string(status)}")
+
+
+def lib() -> ctypes.CDLL:
+    """Load libgdn2.so (built in-tree by ``gated_delta_rule_118_b200.build``)."""
+    global _lib
+    if _lib is None:
+        if not LIBRARY_PATH.exists():
+            raise RuntimeError(f"native library {LIBRARY_PATH} is missing; run "
+                               "`python -m gated_delta_rule_118_b200.build` (there is no fallback)")
+        L = ctypes.CDLL(str(LIBRARY_PATH))
+        vp, fp, ci = ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int
+        L.gdn2_fwd_chunked.argtypes = [vp] * 5 + [fp, fp, vp, fp] + [ci] * 6 + [vp]
+        L.gdn2_fwd_chunked.restype = ci
+        L.gdn2_decode_step.argtypes = [vp] * 5 + [fp, fp, vp] + [ci] * 5 + [vp]
+        L.gdn2_decode_step.restype = ci
+        L.gdn2_check_device_error.argtypes = [vp]
+        L.gdn2_check_device_error.restype = ci
+        L.gdn2_status_string.argtypes = [ci]
+        L.gdn2_status_string.restype = ctypes.c_char_p
+        _lib = L
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return lib().gdn2_status_string(int(status)).decode()
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return GDN2_F32
+    if t.dtype == torch.bfloat16:
+        return GDN2_BF16
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def gdn2_fwd_chunked(q, k, v, b, w, log_alpha, S0=None, o=None, S_T=None, *,
+                     stream=None, want_state=True, check=True):
+    """Chunked forward.  Tensors are CUDA, contiguous, [B,T,H,d]; returns (o, S_T).
+
+    ``o`` and ``S_T`` are allocated with torch when not given (S_T only when
+    ``want_state``).  Raises Gdn2Error on a non-OK status.
+    """
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    if o is None:
+        o = torch.empty((B, T, H, dv), dtype=q.dtype, device=q.device)
+    if S_T is None and want_state:
+        S_T = torch.empty((B, H, dk, dv), dtype=torch.float32, device=q.device)
+    for name, t in (("q", q), ("k", k), ("v", v), ("b", b), ("w", w), ("log_alpha", log_alpha),
+                    ("o", o), ("S0", S0), ("S_T", S_T)):
+        if t is not None and not (t.is_cuda and t.is_contiguous()):
+            raise ValueError(f"{name} must be a contiguous CUDA tensor")
+    if log_alpha.dtype != torch.float32 or (S0 is not None and S0.dtype != torch.float32):
+        raise TypeError("log_alpha and S0 must be float32")
+    st = lib().gdn2_fwd_chunked(_ptr(q), _ptr(k), _ptr(v), _ptr(b), _ptr(w), _ptr(log_alpha),
+                                _ptr(S0), _ptr(o), _ptr(S_T), B, T, H, dk, dv, _dtype_code(q),
+                                _stream(stream))
+    if check and st != GDN2_OK:
+        raise Gdn2Error(st, "gdn2_fwd_chunked")
+    return o, S_T
+
+
+def gdn2_decode_step(q, k, v, b, w, log_alpha, S, o=None, *, stream=None, check=True):
+    """One recurrent token: [B,H,d] inputs, S [B,H,dk,dv] fp32 updated in place; returns o."""
+    B, H, dk = q.shape
+    dv = v.shape[-1]
+    if o is None:
+        o = torch.empty((B, H, dv), dtype=q.dtype, device=q.device)
+    st = lib().gdn2_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(b), _ptr(w), _ptr(log_alpha),
+                                _ptr(S), _ptr(o), B, H, dk, dv, _dtype_code(q), _stream(stream))
+    if check and st != GDN2_OK:
+        raise Gdn2Error(st, "gdn2_decode_step")
+    return o
+
+
+def gdn2_check_device_error(stream=None) -> int:
+    """Synchronise ``stream`` and return (and clear) the device error status."""
+    return int(lib().gdn2_check_device_error(_stream(stream)))
+
+
+def gdn2_status_string(status: int) -> str:
+    return status_string(status)

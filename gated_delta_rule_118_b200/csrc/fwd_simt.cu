@@ -1,0 +1,216 @@
+// fwd_simt.cu -- chunkwise forward on the fp32 FMA pipes.
+//
+// This is the fp32-input path of gdn2_fwd_chunked: every product runs in fp32
+// on CUDA cores, so it meets the fp32 tolerance that tensor-core operands in
+// bf16 cannot.  It follows the chunkwise (WY) form with chunks of 64 tokens
+// ("Gated DeltaNet-2", iplexlaw.co.kr, section "Procesamiento del token y
+// entrenamiento paralelo"; gist.science, section 3 "Efficient chunkwise
+// parallel training"), with Gamma the chunk-local cumulative log-decay in fp32
+// and r the chunk midpoint:
+//   Ehat = e^{Gamma-Gamma_r} b k,  Qhat = e^{Gamma-Gamma_r} q,
+//   Khat = e^{Gamma_r-Gamma} k,    Ktil = e^{Gamma_C-Gamma} k,
+//   A = strict_lower(Ehat Khat^T), P = lower(Qhat Khat^T), Sref = e^{Gamma_r} S,
+//   (I + A) U = Z - Ehat Sref,     O = Qhat Sref + P U,
+//   S <- e^{Gamma_C} S + Ktil^T U.
+// One CTA owns one (batch, head, 32-column value tile); value columns of the
+// state are independent because the erase and the decay act on key rows.
+#include "common.cuh"
+#include "launch.h"
+
+namespace gdn2 {
+namespace {
+
+constexpr int kSimtThreads = 256;
+constexpr int kSimtDvTile = 32;
+
+template <int DK, int DVT>
+struct SimtSmem {
+    static constexpr int LDK = DK + 1;     // padded rows: conflict-free column walks
+    static constexpr int LDC = kChunk + 1;
+    static constexpr int kFloats = 4 * kChunk * LDK   // Qhat, Khat, Ehat, Ktil
+                                   + 2 * kChunk * LDC // A, P
+                                   + 2 * DK * DVT     // S, Sref
+                                   + kChunk * DVT     // Z -> U
+                                   + 2 * DK;          // Gamma_r, Gamma_C
+    static constexpr size_t kBytes = sizeof(float) * kFloats;
+};
+
+template <typename T, int DK, int DVT>
+__global__ void __launch_bounds__(kSimtThreads)
+fwd_simt_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__ v,
+                const T *__restrict__ b, const T *__restrict__ w,
+                const float *__restrict__ log_alpha, const float *S0, T *__restrict__ o,
+                float *S_T, int Tlen, int H, int DV, unsigned int *err)
+{
+    using L = SimtSmem<DK, DVT>;
+    constexpr int C = kChunk, LDK = L::LDK, LDC = L::LDC;
+    extern __shared__ float smem[];
+    float *sQ = smem;                 // q  -> Qhat        [C][LDK]
+    float *sK = sQ + C * LDK;         // k  -> Khat
+    float *sE = sK + C * LDK;         // b  -> Ehat
+    float *sG = sE + C * LDK;         // log_alpha -> Gamma -> Ktil
+    float *sA = sG + C * LDK;         // A  [C][LDC]
+    float *sP = sA + C * LDC;         // P
+    float *sS = sP + C * LDC;         // S  [DK][DVT]
+    float *sR = sS + DK * DVT;        // Sref
+    float *sU = sR + DK * DVT;        // Z -> U  [C][DVT]
+    float *sGr = sU + C * DVT;        // Gamma_r [DK]
+    float *sGc = sGr + DK;            // Gamma_C [DK]
+
+    const int tid = threadIdx.x;
+    const int j0 = blockIdx.x * DVT;  // first value column of this tile
+    const int h = blockIdx.y;
+    const long bi = blockIdx.z;
+    const long pair = bi * H + h;
+
+    for (int idx = tid; idx < DK * DVT; idx += kSimtThreads) {
+        const int i = idx / DVT, j = idx % DVT;
+        sS[idx] = S0 ? S0[(pair * DK + i) * DV + j0 + j] : 0.f;
+    }
+
+    const int nchunks = (Tlen + C - 1) / C;
+    for (int c = 0; c < nchunks; ++c) {
+        const int t0 = c * C;
+        const int Lc = min(C, Tlen - t0);
+        __syncthreads();  // previous chunk done with every buffer
+
+        // ---- load the chunk (rows past the sequence end are zero) ----
+        for (int idx = tid; idx < C * DK; idx += kSimtThreads) {
+            const int t = idx / DK, i = idx % DK;
+            float qv = 0.f, kv = 0.f, bv = 0.f, la = 0.f;
+            if (t < Lc) {
+                const long off = ((bi * Tlen + t0 + t) * H + h) * (long)DK + i;
+                qv = to_f32(q[off]); kv = to_f32(k[off]); bv = to_f32(b[off]); la = log_alpha[off];
+            }
+            sQ[t * LDK + i] = qv; sK[t * LDK + i] = kv; sE[t * LDK + i] = bv; sG[t * LDK + i] = la;
+        }
+        for (int idx = tid; idx < C * DVT; idx += kSimtThreads) {
+            const int t = idx / DVT, j = idx % DVT;
+            float z = 0.f;
+            if (t < Lc) {
+                const long off = ((bi * Tlen + t0 + t) * H + h) * (long)DV + j0 + j;
+                z = to_f32(w[off]) * to_f32(v[off]);
+            }
+            sU[idx] = z;
+        }
+        __syncthreads();
+
+        // ---- Gamma: inclusive cumulative log-decay per key channel, fp32 ----
+        const int rmid = min(C / 2, Lc);  // reference token count (midpoint)
+        for (int i = tid; i < DK; i += kSimtThreads) {
+            float g = 0.f, gr = 0.f;
+            for (int t = 0; t < C; ++t) {
+                g += sG[t * LDK + i];
+                sG[t * LDK + i] = g;
+                if (t == rmid - 1) gr = g;
+            }
+            sGr[i] = gr;
+            sGc[i] = g;
+        }
+        __syncthreads();
+
+        // ---- decay-absorbed factors; Sref = e^{Gamma_r} S ----
+        unsigned int bad = 0;
+        for (int idx = tid; idx < C * DK; idx += kSimtThreads) {
+            const int t = idx / DK, i = idx % DK;
+            const float g = sG[t * LDK + i];
+            const float x = g - sGr[i];
+            bad |= (fabsf(x) > kMaxHalfChunkLogDecay);
+            const float up = expf(x), dn = expf(-x), tl = expf(sGc[i] - g);
+            const float kv = sK[t * LDK + i];
+            sQ[t * LDK + i] *= up;
+            sE[t * LDK + i] *= up * kv;
+            sK[t * LDK + i] = dn * kv;
+            sG[t * LDK + i] = tl * kv;
+        }
+        if (bad) atomicOr(err, kErrRange);
+        for (int idx = tid; idx < DK * DVT; idx += kSimtThreads)
+            sR[idx] = expf(sGr[idx / DVT]) * sS[idx];
+        __syncthreads();
+
+        // ---- A = strict_lower(Ehat Khat^T), P = lower(Qhat Khat^T) ----
+        for (int idx = tid; idx < C * C; idx += kSimtThreads) {
+            const int t = idx / C, s = idx % C;
+            float a = 0.f, p = 0.f;
+            if (s <= t) {
+                const float *e = sE + t * LDK, *qq = sQ + t * LDK, *kk = sK + s * LDK;
+#pragma unroll 8
+                for (int i = 0; i < DK; ++i) {
+                    a += e[i] * kk[i];
+                    p += qq[i] * kk[i];
+                }
+            }
+            sA[t * LDC + s] = (s < t) ? a : 0.f;
+            sP[t * LDC + s] = p;
+        }
+        // ---- right-hand side Z - Ehat Sref (in place in sU) ----
+        for (int idx = tid; idx < C * DVT; idx += kSimtThreads) {
+            const int t = idx / DVT, j = idx % DVT;
+            const float *e = sE + t * LDK;
+            float acc = 0.f;
+#pragma unroll 8
+            for (int i = 0; i < DK; ++i) acc += e[i] * sR[i * DVT + j];
+            sU[idx] -= acc;
+        }
+        __syncthreads();
+
+        // ---- forward substitution (I + A) U = RHS, column-oriented ----
+        for (int s = 0; s < Lc - 1; ++s) {
+            for (int idx = tid; idx < (C - 1 - s) * DVT; idx += kSimtThreads) {
+                const int t = s + 1 + idx / DVT, j = idx % DVT;
+                sU[t * DVT + j] -= sA[t * LDC + s] * sU[s * DVT + j];
+            }
+            __syncthreads();
+        }
+
+        // ---- O = Qhat Sref + P U ----
+        for (int idx = tid; idx < Lc * DVT; idx += kSimtThreads) {
+            const int t = idx / DVT, j = idx % DVT;
+            const float *qq = sQ + t * LDK, *pp = sP + t * LDC;
+            float acc = 0.f;
+#pragma unroll 8
+            for (int i = 0; i < DK; ++i) acc += qq[i] * sR[i * DVT + j];
+            for (int s = 0; s <= t; ++s) acc += pp[s] * sU[s * DVT + j];
+            o[((bi * Tlen + t0 + t) * H + h) * (long)DV + j0 + j] = from_f32<T>(acc);
+        }
+        // ---- S <- e^{Gamma_C} S + Ktil^T U ----
+        for (int idx = tid; idx < DK * DVT; idx += kSimtThreads) {
+            const int i = idx / DVT, j = idx % DVT;
+            float acc = expf(sGc[i]) * sS[idx];
+            for (int s = 0; s < Lc; ++s) acc += sG[s * LDK + i] * sU[s * DVT + j];
+            sS[idx] = acc;
+        }
+    }
+    __syncthreads();
+    if (S_T) {
+        for (int idx = tid; idx < DK * DVT; idx += kSimtThreads) {
+            const int i = idx / DVT, j = idx % DVT;
+            S_T[(pair * DK + i) * DV + j0 + j] = sS[idx];
+        }
+    }
+}
+
+template <typename T, int DK>
+cudaError_t launch(const FwdArgs &a)
+{
+    constexpr int DVT = kSimtDvTile;
+    const size_t smem = SimtSmem<DK, DVT>::kBytes;
+    auto kern = fwd_simt_kernel<T, DK, DVT>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    dim3 grid(a.dv / DVT, a.H, a.B);
+    kern<<<grid, kSimtThreads, smem, a.stream>>>(
+        (const T *)a.q, (const T *)a.k, (const T *)a.v, (const T *)a.b, (const T *)a.w,
+        a.log_alpha, a.S0, (T *)a.o, a.S_T, a.T, a.H, a.dv, a.err);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_fwd_simt(const FwdArgs &a)
+{
+    if (a.bf16) return a.dk == 128 ? launch<__nv_bfloat16, 128>(a) : launch<__nv_bfloat16, 64>(a);
+    return a.dk == 128 ? launch<float, 128>(a) : launch<float, 64>(a);
+}
+
+}  // namespace gdn2

@@ -1,0 +1,153 @@
+// gdn2_api.cu -- the C ABI of libgdn2.so: argument checks, the device error
+// word, and the launch of the forward and decode kernels on the caller's stream.
+#include <cuda_runtime.h>
+
+#include <mutex>
+#include <stdint.h>
+
+#include "gdn2.h"
+#include "common.cuh"
+#include "launch.h"
+
+namespace gdn2 {
+
+// Device-side error word: kernels OR bits into it (kErrTimeout, kErrRange);
+// gdn2_check_device_error() reads and clears it.  One per device (module global).
+__device__ unsigned int g_device_error = 0;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+std::mutex g_init_mutex;
+unsigned int *g_err_ptr[kMaxDevices] = {};
+int g_num_sms[kMaxDevices] = {};
+
+// Address of the error word and the SM count on the current device.
+gdn2_status device_context(unsigned int **err, int *num_sms)
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return GDN2_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(g_init_mutex);
+    if (!g_err_ptr[dev]) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_device_error) != cudaSuccess) return GDN2_ERR_CUDA;
+        int sms = 0;
+        if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+            return GDN2_ERR_CUDA;
+        g_err_ptr[dev] = static_cast<unsigned int *>(p);
+        g_num_sms[dev] = sms;
+    }
+    *err = g_err_ptr[dev];
+    *num_sms = g_num_sms[dev];
+    return GDN2_OK;
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool head_dim_ok(int d) { return d == 64 || d == 128; }
+
+gdn2_status check_dims(int dk, int dv)
+{
+    if (dk <= 0 || dv <= 0) return GDN2_ERR_SHAPE;
+    if (!head_dim_ok(dk) || !head_dim_ok(dv)) return GDN2_ERR_UNSUPPORTED;
+    return GDN2_OK;
+}
+
+}  // namespace
+}  // namespace gdn2
+
+using namespace gdn2;
+
+extern "C" gdn2_status gdn2_fwd_chunked(const void *q, const void *k, const void *v,
+                                        const void *b, const void *w, const float *log_alpha,
+                                        const float *S0, void *o, float *S_T,
+                                        int B, int T, int H, int dk, int dv,
+                                        gdn2_dtype dtype, gdn2_stream_t stream)
+{
+    if (dtype != GDN2_F32 && dtype != GDN2_BF16) return GDN2_ERR_DTYPE;
+    if (B <= 0 || H <= 0 || T < 0) return GDN2_ERR_SHAPE;
+    gdn2_status st = check_dims(dk, dv);
+    if (st != GDN2_OK) return st;
+    if (B > 65535 || H > 65535) return GDN2_ERR_UNSUPPORTED;  // grid y/z limits
+    const void *ins[] = {q, k, v, b, w, log_alpha, o};
+    if (T > 0)
+        for (const void *p : ins)
+            if (!p) return GDN2_ERR_NULL;
+    const void *all[] = {q, k, v, b, w, log_alpha, o, S0, S_T};
+    for (const void *p : all)
+        if (p && !aligned16(p)) return GDN2_ERR_ALIGN;
+
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (T == 0) {  // nothing to run: S_T = S0 (or zeros)
+        if (!S_T) return GDN2_OK;
+        const size_t bytes = sizeof(float) * (size_t)B * H * dk * dv;
+        cudaError_t e = S0 ? (S0 == S_T ? cudaSuccess
+                                        : cudaMemcpyAsync(S_T, S0, bytes, cudaMemcpyDeviceToDevice, s))
+                           : cudaMemsetAsync(S_T, 0, bytes, s);
+        return e == cudaSuccess ? GDN2_OK : GDN2_ERR_CUDA;
+    }
+
+    FwdArgs a{};
+    a.q = q; a.k = k; a.v = v; a.b = b; a.w = w; a.log_alpha = log_alpha;
+    a.S0 = S0; a.o = o; a.S_T = S_T;
+    a.B = B; a.T = T; a.H = H; a.dk = dk; a.dv = dv;
+    a.bf16 = (dtype == GDN2_BF16);
+    a.stream = s;
+    st = device_context(&a.err, &a.num_sms);
+    if (st != GDN2_OK) return st;
+    return launch_fwd_simt(a) == cudaSuccess ? GDN2_OK : GDN2_ERR_CUDA;
+}
+
+extern "C" gdn2_status gdn2_decode_step(const void *q, const void *k, const void *v,
+                                        const void *b, const void *w, const float *log_alpha,
+                                        float *S, void *o, int B, int H, int dk, int dv,
+                                        gdn2_dtype dtype, gdn2_stream_t stream)
+{
+    if (dtype != GDN2_F32 && dtype != GDN2_BF16) return GDN2_ERR_DTYPE;
+    if (B <= 0 || H <= 0) return GDN2_ERR_SHAPE;
+    gdn2_status st = check_dims(dk, dv);
+    if (st != GDN2_OK) return st;
+    if ((long long)B * H > 0x7fffffffLL) return GDN2_ERR_UNSUPPORTED;  // grid x limit
+    const void *all[] = {q, k, v, b, w, log_alpha, S, o};
+    for (const void *p : all) {
+        if (!p) return GDN2_ERR_NULL;
+        if (!aligned16(p)) return GDN2_ERR_ALIGN;
+    }
+    DecodeArgs a{};
+    a.q = q; a.k = k; a.v = v; a.b = b; a.w = w; a.log_alpha = log_alpha;
+    a.S = S; a.o = o; a.B = B; a.H = H; a.dk = dk; a.dv = dv;
+    a.bf16 = (dtype == GDN2_BF16);
+    a.stream = reinterpret_cast<cudaStream_t>(stream);
+    return launch_decode(a) == cudaSuccess ? GDN2_OK : GDN2_ERR_CUDA;
+}
+
+extern "C" gdn2_status gdn2_check_device_error(gdn2_stream_t stream)
+{
+    unsigned int *err = nullptr;
+    int sms = 0;
+    if (device_context(&err, &sms) != GDN2_OK) return GDN2_ERR_CUDA;
+    if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+        return GDN2_ERR_CUDA;
+    unsigned int word = 0;
+    if (cudaMemcpy(&word, err, sizeof(word), cudaMemcpyDeviceToHost) != cudaSuccess)
+        return GDN2_ERR_CUDA;
+    if (word && cudaMemset(err, 0, sizeof(word)) != cudaSuccess) return GDN2_ERR_CUDA;
+    if (word & kErrTimeout) return GDN2_ERR_DEVICE_TIMEOUT;
+    if (word & kErrRange) return GDN2_ERR_RANGE;
+    return GDN2_OK;
+}
+
+extern "C" const char *gdn2_status_string(gdn2_status status)
+{
+    switch (status) {
+    case GDN2_OK: return "GDN2_OK";
+    case GDN2_ERR_NULL: return "GDN2_ERR_NULL: a required pointer is NULL";
+    case GDN2_ERR_SHAPE: return "GDN2_ERR_SHAPE: a size is out of range";
+    case GDN2_ERR_DTYPE: return "GDN2_ERR_DTYPE: unknown dtype code";
+    case GDN2_ERR_ALIGN: return "GDN2_ERR_ALIGN: a pointer is not 16-byte aligned";
+    case GDN2_ERR_UNSUPPORTED: return "GDN2_ERR_UNSUPPORTED: request outside the implemented set";
+    case GDN2_ERR_CUDA: return "GDN2_ERR_CUDA: a CUDA runtime call or launch failed";
+    case GDN2_ERR_DEVICE_TIMEOUT: return "GDN2_ERR_DEVICE_TIMEOUT: a device-side bounded wait gave up";
+    case GDN2_ERR_RANGE: return "GDN2_ERR_RANGE: a chunk's cumulative decay left the factored range";
+    }
+    return "GDN2 unknown status";
+}

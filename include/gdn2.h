@@ -1,0 +1,132 @@
+/*
+ * gdn2.h -- C ABI of the Gated DeltaNet-2 operator library (libgdn2.so).
+ *
+ * The operator is the gated delta rule with decoupled erase and write gates
+ * ("Gated DeltaNet-2: Decoupling Erase and Write in Linear Attention").  Per
+ * (batch, head) it keeps a dk x dv state S and, for each token t,
+ *
+ *     Sbar = Diag(alpha_t) S_{t-1}          alpha_t = exp(log_alpha_t), per key channel
+ *     e_t  = b_t (*) k_t                    erase gate b_t on the key axis
+ *     z_t  = w_t (*) v_t                    write gate w_t on the value axis
+ *     r_t  = Sbar^T e_t
+ *     S_t  = Sbar + k_t (z_t - r_t)^T
+ *     o_t  = S_t^T q_t                      the query reads the updated state
+ *
+ * as stated on the iplexlaw.co.kr page, section "Decisiones independientes en
+ * dos ejes", and in product form S_t = (I - k_t (b_t (*) k_t)^T) D_t S_{t-1}
+ * + k_t (w_t (*) v_t)^T in the zubnet.ai news item and the gist.science
+ * summary (section 1, "Gated Delta Rule-2").  No scale is applied to q.
+ *
+ * Conventions shared by every entry point:
+ *   - All tensor arguments are DEVICE pointers owned by the caller.  The
+ *     library allocates no memory, keeps no per-call state and never
+ *     synchronises the stream; work is queued on `stream` (NULL = the legacy
+ *     default stream) and the call returns once it is queued.
+ *   - Layouts are dense row-major: q, k, b, log_alpha are [B][T][H][dk];
+ *     v, w, o are [B][T][H][dv]; states are [B][H][dk][dv].  (The decode entry
+ *     point drops the T axis.)
+ *   - `dtype` is the element type of q, k, v, b, w and o.  log_alpha and
+ *     every state are always fp32.  bf16 outputs are rounded to nearest even.
+ *   - Every pointer must be 16-byte aligned.
+ *   - Supported head sizes: dk and dv each 64 or 128.
+ *   - The returned status covers argument checks and launch errors only.
+ *     Conditions found while the kernels run (a bounded wait that gave up, a
+ *     decay outside the supported range) are recorded in a device-side error
+ *     word and reported by gdn2_check_device_error().
+ *   - Gates are used as given: values outside [0, 1] (the pages' ablation
+ *     widens the erase range to [0, 2]) are not clamped.
+ */
+#ifndef GDN2_H
+#define GDN2_H
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum gdn2_status {
+    GDN2_OK = 0,
+    GDN2_ERR_NULL = 1,           /* a required pointer is NULL                        */
+    GDN2_ERR_SHAPE = 2,          /* a size is out of range (negative, zero, too big)  */
+    GDN2_ERR_DTYPE = 3,          /* unknown gdn2_dtype code                           */
+    GDN2_ERR_ALIGN = 4,          /* a pointer is not 16-byte aligned                  */
+    GDN2_ERR_UNSUPPORTED = 5,    /* valid request outside the implemented set         */
+    GDN2_ERR_CUDA = 6,           /* a CUDA runtime call or launch failed              */
+    GDN2_ERR_DEVICE_TIMEOUT = 7, /* a device-side bounded wait gave up                */
+    GDN2_ERR_RANGE = 8           /* a chunk's cumulative decay left the factored range */
+} gdn2_status;
+
+typedef enum gdn2_dtype {
+    GDN2_F32 = 0,
+    GDN2_BF16 = 1
+} gdn2_dtype;
+
+/* Same type as cudaStream_t; declared here so this header needs no CUDA header. */
+typedef struct CUstream_st *gdn2_stream_t;
+
+/*
+ * gdn2_fwd_chunked -- prefill / training forward over a whole sequence.
+ *
+ * Computes o_t for t = 0..T-1 and the final state S_T of the recurrence above,
+ * chunkwise with chunks of 64 tokens: the per-channel decay is cumulated in
+ * fp32 inside each chunk and folded into asymmetric decayed erase/key factors,
+ * the strictly lower triangular 64 x 64 system is solved per chunk, and the
+ * state is passed from chunk to chunk (iplexlaw.co.kr, section "Procesamiento
+ * del token y entrenamiento paralelo"; gist.science, section 3 "Efficient
+ * chunkwise parallel training").  The result equals the token recurrence up
+ * to rounding.
+ *
+ *   q, k, b     [B][T][H][dk]  dtype   query, key, erase gate
+ *   v, w        [B][T][H][dv]  dtype   value, write gate
+ *   log_alpha   [B][T][H][dk]  fp32    log of the per-key-channel decay (<= 0)
+ *   S0          [B][H][dk][dv] fp32    initial state; NULL means zero
+ *   o           [B][T][H][dv]  dtype   output, written (never read)
+ *   S_T         [B][H][dk][dv] fp32    final state; NULL means not written.
+ *                                      May alias S0 (in-place advance).
+ *   B, H >= 1; T >= 0 (T = 0 only copies S0, or zeros, into S_T).
+ *
+ * Range: inside each 64-token chunk the cumulative log-decay of every key
+ * channel is split at the chunk midpoint and each half must stay above -80
+ * (any log_alpha >= -2.5 satisfies this).  A chunk outside this range sets
+ * GDN2_ERR_RANGE in the device error word and its results are not valid.
+ */
+gdn2_status gdn2_fwd_chunked(const void *q, const void *k, const void *v,
+                             const void *b, const void *w, const float *log_alpha,
+                             const float *S0, void *o, float *S_T,
+                             int B, int T, int H, int dk, int dv,
+                             gdn2_dtype dtype, gdn2_stream_t stream);
+
+/*
+ * gdn2_decode_step -- one token of the recurrence with the state resident in
+ * device memory (recurrent decoding with a fixed-size state instead of a
+ * growing cache: gist.science, "Problem Statement"; iplexlaw.co.kr, "De una
+ * caché creciente a un estado fijo").
+ *
+ *   q, k, b     [B][H][dk]      dtype
+ *   v, w        [B][H][dv]      dtype
+ *   log_alpha   [B][H][dk]      fp32
+ *   S           [B][H][dk][dv]  fp32   read and updated in place
+ *   o           [B][H][dv]      dtype  written
+ *   B, H >= 1.
+ *
+ * Each state is streamed through the GPU once: read once, written once.
+ */
+gdn2_status gdn2_decode_step(const void *q, const void *k, const void *v,
+                             const void *b, const void *w, const float *log_alpha,
+                             float *S, void *o, int B, int H, int dk, int dv,
+                             gdn2_dtype dtype, gdn2_stream_t stream);
+
+/*
+ * gdn2_check_device_error -- wait for `stream`, then read and clear the
+ * device error word of the current device.  Returns GDN2_OK,
+ * GDN2_ERR_DEVICE_TIMEOUT, GDN2_ERR_RANGE or GDN2_ERR_CUDA.
+ */
+gdn2_status gdn2_check_device_error(gdn2_stream_t stream);
+
+/* Human-readable name of a status code (static storage, never NULL). */
+const char *gdn2_status_string(gdn2_status status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GDN2_H */

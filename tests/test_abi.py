@@ -1,0 +1,85 @@
+"""The C-ABI library builds, loads, exports every declared symbol and rejects
+bad arguments on the host before touching a GPU (CPU-only tests)."""
+import ctypes
+import re
+from pathlib import Path
+
+import pytest
+
+import gated_delta_rule_118_b200 as g
+from gated_delta_rule_118_b200 import build
+
+HEADER = Path(__file__).resolve().parent.parent / "include" / "gdn2.h"
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build_library()
+    return g.lib()
+
+
+def declared_functions():
+    text = re.sub(r"/\*.*?\*/", "", HEADER.read_text(), flags=re.S)
+    return sorted(set(re.findall(r"\b(gdn2_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = declared_functions()
+    assert set(names) == set(g.EXPORTED), names
+    for n in names:
+        assert hasattr(lib, n), f"{n} not exported by {g.LIBRARY_PATH}"
+
+
+def test_library_is_built_for_sm100a(lib):
+    # the build passes only compute_100a/sm_100a to nvcc
+    assert build.ARCH == ["-gencode", "arch=compute_100a,code=sm_100a"]
+
+
+def test_status_strings(lib):
+    for code in range(9):
+        s = g.status_string(code)
+        assert s.startswith("GDN2_")
+    assert "unknown" in g.status_string(99)
+
+
+# Host-side validation.  Fake (never dereferenced) device addresses: every
+# call below must be rejected before any CUDA call is made.
+P = ctypes.c_void_p(0x10000)       # 16-byte aligned
+MIS = ctypes.c_void_p(0x10008)     # misaligned
+
+
+def fwd(lib, *, q=P, o=P, S0=None, B=1, T=8, H=2, dk=64, dv=64, dtype=1):
+    return lib.gdn2_fwd_chunked(q, P, P, P, P, P, S0, o, None, B, T, H, dk, dv, dtype, None)
+
+
+def dec(lib, *, S=P, B=1, H=2, dk=64, dv=64, dtype=0, q=P):
+    return lib.gdn2_decode_step(q, P, P, P, P, P, S, P, B, H, dk, dv, dtype, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(dtype=5), g.GDN2_ERR_DTYPE),
+    (dict(B=0), g.GDN2_ERR_SHAPE),
+    (dict(H=-1), g.GDN2_ERR_SHAPE),
+    (dict(T=-3), g.GDN2_ERR_SHAPE),
+    (dict(dk=0), g.GDN2_ERR_SHAPE),
+    (dict(dk=96), g.GDN2_ERR_UNSUPPORTED),
+    (dict(dv=256), g.GDN2_ERR_UNSUPPORTED),
+    (dict(B=70000), g.GDN2_ERR_UNSUPPORTED),
+    (dict(q=None), g.GDN2_ERR_NULL),
+    (dict(o=None), g.GDN2_ERR_NULL),
+    (dict(q=MIS), g.GDN2_ERR_ALIGN),
+    (dict(S0=MIS), g.GDN2_ERR_ALIGN),
+])
+def test_fwd_rejects_bad_arguments(lib, kw, code):
+    assert fwd(lib, **kw) == code
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(dtype=2), g.GDN2_ERR_DTYPE),
+    (dict(B=0), g.GDN2_ERR_SHAPE),
+    (dict(dk=32), g.GDN2_ERR_UNSUPPORTED),
+    (dict(S=None), g.GDN2_ERR_NULL),
+    (dict(q=MIS), g.GDN2_ERR_ALIGN),
+])
+def test_decode_rejects_bad_arguments(lib, kw, code):
+    assert dec(lib, **kw) == code
