@@ -94,7 +94,10 @@ extern "C" gdn2_status gdn2_fwd_chunked(const void *q, const void *k, const void
     a.stream = s;
     st = device_context(&a.err, &a.num_sms);
     if (st != GDN2_OK) return st;
-    return launch_fwd_simt(a) == cudaSuccess ? GDN2_OK : GDN2_ERR_CUDA;
+    // bf16 inputs with dk = 128 run on the tensor cores; fp32 inputs (and dk = 64)
+    // run on the fp32 pipes, which meet the fp32 tolerance.
+    const cudaError_t e = (a.bf16 && dk == 128) ? launch_fwd_tc(a) : launch_fwd_simt(a);
+    return e == cudaSuccess ? GDN2_OK : GDN2_ERR_CUDA;
 }
 
 extern "C" gdn2_status gdn2_decode_step(const void *q, const void *k, const void *v,

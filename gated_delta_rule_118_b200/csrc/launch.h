@@ -31,5 +31,7 @@ struct FwdArgs {
 
 cudaError_t launch_decode(const DecodeArgs &a);
 cudaError_t launch_fwd_simt(const FwdArgs &a);
+cudaError_t launch_fwd_tc(const FwdArgs &a);
+int fwd_tc_tile(int B, int H, int dv, int num_sms);
 
 }  // namespace gdn2
