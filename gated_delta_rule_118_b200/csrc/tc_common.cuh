@@ -1,0 +1,91 @@
+// tc_common.cuh -- helpers shared by the tensor-core forward kernels: bf16
+// packing, the shared-memory plan of one prep record, and the record layout in
+// the workspace that carries a chunk's state-independent quantities from the
+// prep kernel to the chain kernel.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "common.cuh"
+#include "sm100.cuh"
+
+namespace gdn2 {
+
+using bf16 = __nv_bfloat16;
+
+constexpr float kLog2e = 1.4426950408889634f;
+
+__host__ __device__ constexpr int align_up(int x, int a) { return (x + a - 1) / a * a; }
+
+// One prep record per (batch, head, chunk), consumed by the chain and output kernels.
+//   GC  [128 rows = key channel][128 K = key channel] bf16, K-major, 128-byte
+//       swizzle, two 64-column blocks of 16 KB: G = Ktil^T T Ehat (the part of
+//       the chunk transition that the erase projection removes)
+//   QP  [64 rows = token][128 K] bf16, K-major, swizzled, blocks of 8 KB:
+//       Q' = Qhat - P T Ehat
+//   PU  [dv/64 blocks][64 tokens][64] bf16, rows swizzled: P T Z (the output's
+//       state-independent part)
+//   NC  [dv/64 blocks][128 key channels][64] bf16, rows swizzled: Ktil^T T Z
+//   DEC [2][128] fp32: e^{Gamma_C}, e^{Gamma_r} per key channel
+template <int DV>
+struct Record {
+    static constexpr int GC = 0;
+    static constexpr int QP = GC + 32768;
+    static constexpr int PU = QP + 16384;
+    static constexpr int NC = PU + 64 * DV * 2;
+    static constexpr int DEC = NC + 128 * DV * 2;
+    static constexpr int BYTES = DEC + 1024;
+};
+
+// The chain kernel exports Sref = e^{Gamma_r} S of every chunk for the output
+// kernel: [128 key channels][DV] bf16 as dv/64 blocks of [128 rows][128 B],
+// 128-byte swizzle, i.e. the MN-major operand layout of the output UMMA.
+template <int DV>
+struct SrefSlot {
+    static constexpr int BYTES = 128 * DV * 2;
+};
+
+__device__ __forceinline__ uint4 pack8(const float *f)
+{
+    uint4 r;
+    __nv_bfloat162 h;
+    h = __floats2bfloat162_rn(f[0], f[1]); r.x = *reinterpret_cast<uint32_t *>(&h);
+    h = __floats2bfloat162_rn(f[2], f[3]); r.y = *reinterpret_cast<uint32_t *>(&h);
+    h = __floats2bfloat162_rn(f[4], f[5]); r.z = *reinterpret_cast<uint32_t *>(&h);
+    h = __floats2bfloat162_rn(f[6], f[7]); r.w = *reinterpret_cast<uint32_t *>(&h);
+    return r;
+}
+
+__device__ __forceinline__ void unpack8(uint4 v, float *f)
+{
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const float2 p = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&w[i]));
+        f[2 * i] = p.x;
+        f[2 * i + 1] = p.y;
+    }
+}
+
+__device__ __forceinline__ float2 ld_bf16x2(const uint8_t *p)
+{
+    return __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(p));
+}
+__device__ __forceinline__ void st_bf16x2(uint8_t *p, float a, float b)
+{
+    *reinterpret_cast<__nv_bfloat162 *>(p) = __floats2bfloat162_rn(a, b);
+}
+
+__device__ __forceinline__ float ex2_approx(float x)
+{
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+// fp32 64x64 matrix in shared memory with 16-byte chunks XOR-swizzled by row,
+// so that row-per-thread float4 stores and column walks avoid bank conflicts.
+__device__ __forceinline__ int af_off(int t, int s) { return t * 64 + ((((s >> 2) ^ (t & 15)) << 2) | (s & 3)); }
+
+}  // namespace gdn2
