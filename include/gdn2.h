@@ -19,9 +19,12 @@
  *
  * Conventions shared by every entry point:
  *   - All tensor arguments are DEVICE pointers owned by the caller.  The
- *     library allocates no memory, keeps no per-call state and never
- *     synchronises the stream; work is queued on `stream` (NULL = the legacy
- *     default stream) and the call returns once it is queued.
+ *     library keeps no per-call state and never synchronises the stream; work
+ *     is queued on `stream` (NULL = the legacy default stream) and the call
+ *     returns once it is queued.  The bf16 path of gdn2_fwd_chunked needs a
+ *     workspace, which it takes from a stream-ordered pool owned by the
+ *     library (allocated and released on `stream`; the pool keeps freed
+ *     blocks for reuse).  Nothing else allocates.
  *   - Layouts are dense row-major: q, k, b, log_alpha are [B][T][H][dk];
  *     v, w, o are [B][T][H][dv]; states are [B][H][dk][dv].  (The decode entry
  *     point drops the T axis.)
