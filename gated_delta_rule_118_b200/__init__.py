@@ -24,13 +24,14 @@ GDN2_ERR_UNSUPPORTED = 5
 GDN2_ERR_CUDA = 6
 GDN2_ERR_DEVICE_TIMEOUT = 7
 GDN2_ERR_RANGE = 8
+GDN2_ERR_SCRATCH_LIMIT = 9
 
 GDN2_F32 = 0
 GDN2_BF16 = 1
 
 # Every symbol include/gdn2.h declares.
-EXPORTED = ("gdn2_fwd_chunked", "gdn2_decode_step", "gdn2_check_device_error",
-            "gdn2_status_string")
+EXPORTED = ("gdn2_fwd_chunked", "gdn2_fwd_chunked_noalloc", "gdn2_decode_step",
+            "gdn2_check_device_error", "gdn2_status_string")
 
 _lib = None
 
@@ -52,6 +53,8 @@ def lib() -> ctypes.CDLL:
         vp, fp, ci = ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int
         L.gdn2_fwd_chunked.argtypes = [vp] * 5 + [fp, fp, vp, fp] + [ci] * 6 + [vp]
         L.gdn2_fwd_chunked.restype = ci
+        L.gdn2_fwd_chunked_noalloc.argtypes = [vp] * 5 + [fp, fp, vp, fp] + [ci] * 6 + [vp]
+        L.gdn2_fwd_chunked_noalloc.restype = ci
         L.gdn2_decode_step.argtypes = [vp] * 5 + [fp, fp, vp] + [ci] * 5 + [vp]
         L.gdn2_decode_step.restype = ci
         L.gdn2_check_device_error.argtypes = [vp]
@@ -107,6 +110,29 @@ def gdn2_fwd_chunked(q, k, v, b, w, log_alpha, S0=None, o=None, S_T=None, *,
                                 _stream(stream))
     if check and st != GDN2_OK:
         raise Gdn2Error(st, "gdn2_fwd_chunked")
+    return o, S_T
+
+
+def gdn2_fwd_chunked_noalloc(q, k, v, b, w, log_alpha, S0=None, o=None, S_T=None, *, stream=None,
+                             check=True):
+    """The chunked forward through the entry point that allocates no device memory.
+
+    Pass ``o`` (and ``S_T`` when the final state is wanted) preallocated; the
+    native call itself uses only its fixed scratch buffer.  Returns (o, S_T).
+    """
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    if o is None:
+        raise ValueError("gdn2_fwd_chunked_noalloc needs a preallocated output o")
+    for name, t in (("q", q), ("k", k), ("v", v), ("b", b), ("w", w), ("log_alpha", log_alpha),
+                    ("o", o), ("S0", S0), ("S_T", S_T)):
+        if t is not None and not (t.is_cuda and t.is_contiguous()):
+            raise ValueError(f"{name} must be a contiguous CUDA tensor")
+    st = lib().gdn2_fwd_chunked_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(b), _ptr(w),
+                                        _ptr(log_alpha), _ptr(S0), _ptr(o), _ptr(S_T),
+                                        B, T, H, dk, dv, _dtype_code(q), _stream(stream))
+    if check and st != GDN2_OK:
+        raise Gdn2Error(st, "gdn2_fwd_chunked_noalloc")
     return o, S_T
 
 

@@ -53,6 +53,14 @@ gdn2_status check_dims(int dk, int dv)
 }
 
 }  // namespace
+
+// Device address of the error word on the current device (for other entry points).
+bool device_error_word(unsigned int **err)
+{
+    int sms = 0;
+    return device_context(err, &sms) == GDN2_OK;
+}
+
 }  // namespace gdn2
 
 using namespace gdn2;
@@ -151,6 +159,7 @@ extern "C" const char *gdn2_status_string(gdn2_status status)
     case GDN2_ERR_CUDA: return "GDN2_ERR_CUDA: a CUDA runtime call or launch failed";
     case GDN2_ERR_DEVICE_TIMEOUT: return "GDN2_ERR_DEVICE_TIMEOUT: a device-side bounded wait gave up";
     case GDN2_ERR_RANGE: return "GDN2_ERR_RANGE: a chunk's cumulative decay left the factored range";
+    case GDN2_ERR_SCRATCH_LIMIT: return "GDN2_ERR_SCRATCH_LIMIT: the problem needs more than the fixed scratch buffer";
     }
     return "GDN2 unknown status";
 }

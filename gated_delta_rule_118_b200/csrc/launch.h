@@ -32,6 +32,7 @@ struct FwdArgs {
     int num_sms;
 };
 
+bool device_error_word(unsigned int **err);
 cudaError_t launch_decode(const DecodeArgs &a);
 cudaError_t launch_fwd_simt(const FwdArgs &a);
 

@@ -55,7 +55,8 @@ typedef enum gdn2_status {
     GDN2_ERR_UNSUPPORTED = 5,    /* valid request outside the implemented set         */
     GDN2_ERR_CUDA = 6,           /* a CUDA runtime call or launch failed              */
     GDN2_ERR_DEVICE_TIMEOUT = 7, /* a device-side bounded wait gave up                */
-    GDN2_ERR_RANGE = 8           /* a chunk's cumulative decay left the factored range */
+    GDN2_ERR_RANGE = 8,          /* a chunk's cumulative decay left the factored range */
+    GDN2_ERR_SCRATCH_LIMIT = 9   /* needs more than gdn2_fwd_chunked_noalloc's fixed buffer */
 } gdn2_status;
 
 typedef enum gdn2_dtype {
@@ -97,6 +98,37 @@ gdn2_status gdn2_fwd_chunked(const void *q, const void *k, const void *v,
                              const float *S0, void *o, float *S_T,
                              int B, int T, int H, int dk, int dv,
                              gdn2_dtype dtype, gdn2_stream_t stream);
+
+/*
+ * gdn2_fwd_chunked_noalloc -- gdn2_fwd_chunked without any device allocation.
+ *
+ * The pages have no counterpart to this entry point; it serves callers that
+ * cannot let a library allocate device memory: a runtime that hands out all
+ * device memory itself, a hot loop that must never enter the driver's
+ * allocator (an allocation can block, or fail on a fragmented heap), or a
+ * process that must know its whole device footprint before it starts.
+ *
+ * Same arguments, layouts, dtypes and results as gdn2_fwd_chunked.  Instead of
+ * drawing its workspace from a memory pool, it uses one fixed 32 MiB buffer in
+ * the library's device image (held on every GPU that loads the library, until
+ * the process exits) and processes the sequence in as many windows as needed
+ * to fit it.  A problem whose single chunk of records does not fit (about
+ * 193 KiB per (batch, head) pair for dv = 128, so B*H up to 169) returns
+ * GDN2_ERR_SCRATCH_LIMIT and launches nothing.
+ *
+ * The first call on a device looks the buffer's device address up
+ * (cudaGetSymbolAddress) with that device current; make that first call
+ * before any stream capture.  All calls share the one buffer: calls whose
+ * work overlaps on the GPU (different streams, or devices sharing nothing but
+ * this buffer's name) race and corrupt each other's results; serialize them.
+ * Every byte of the buffer that a call reads, that call writes first, so its
+ * leftover contents from earlier calls do not matter.
+ */
+gdn2_status gdn2_fwd_chunked_noalloc(const void *q, const void *k, const void *v,
+                                     const void *b, const void *w, const float *log_alpha,
+                                     const float *S0, void *o, float *S_T,
+                                     int B, int T, int H, int dk, int dv,
+                                     gdn2_dtype dtype, gdn2_stream_t stream);
 
 /*
  * gdn2_decode_step -- one token of the recurrence with the state resident in

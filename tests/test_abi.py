@@ -36,7 +36,7 @@ def test_library_is_built_for_sm100a(lib):
 
 
 def test_status_strings(lib):
-    for code in range(9):
+    for code in range(10):
         s = g.status_string(code)
         assert s.startswith("GDN2_")
     assert "unknown" in g.status_string(99)
