@@ -171,6 +171,30 @@ def run_reference(args, ws, rank):
     print(json.dumps(line), flush=True)
 
 
+def run_profile_case(args):
+    """A few launches of one operator on the bench workload, for ncu (-s/-c pick one)."""
+    import gated_delta_rule_118_b200 as g
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    names = ("q", "k", "v", "b", "w", "log_alpha")
+    if args.profile == "fwd":
+        c = CASE
+        d = synth.draw_fwd_device(c.B, c.T, c.H, c.dk, c.dv, seed=0, device=dev, dtype=c.dtype,
+                                  log_alpha_range=c.log_alpha_range, gate_sigma=c.gate_sigma)
+        for _ in range(args.warmup + args.steps):
+            g.gdn2_fwd_chunked(*(d[n] for n in names), S0=None)
+    else:
+        dc = DEC
+        S = 0.05 * torch.randn(dc.B, dc.H, dc.dk, dc.dv, device=dev)
+        dd = synth.draw_fwd_device(dc.B, 1, dc.H, dc.dk, dc.dv, seed=7000, device=dev, dtype=torch.float32)
+        x = {n: dd[n][:, 0].contiguous() for n in names}
+        for _ in range(args.warmup + args.steps):
+            g.gdn2_decode_step(*(x[n] for n in names), S)
+    torch.cuda.synchronize()
+    if g.gdn2_check_device_error() != g.GDN2_OK:
+        raise RuntimeError("device error")
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -179,6 +203,9 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--decode-steps", type=int, default=1000)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--profile", choices=["fwd", "decode"], default=None,
+                    help="run a few launches of one operator on the bench workload for an ncu "
+                         "capture (no timing, no JSON line)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -189,6 +216,9 @@ def main():
         return
 
     import gated_delta_rule_118_b200 as g
+    if args.profile:
+        run_profile_case(args)
+        return
     ws, rank, local = dist_setup(args)
     dev = torch.device("cuda", torch.cuda.current_device())
     stream = torch.cuda.current_stream()

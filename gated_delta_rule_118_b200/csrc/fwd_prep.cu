@@ -21,9 +21,9 @@
 // hides the other's load and UMMA latencies.  q, k, b and log_alpha arrive by
 // TMA straight into the operand buffers and the factors are formed in place;
 // v and w are read with plain vector loads.  Products are tcgen05 UMMAs with
-// fp32 accumulators in tensor memory; the solve is fp32 on CUDA cores (16x16
-// diagonal blocks by substitution, then two levels of register-blocked block
-// merging).  Record pieces leave through bulk copies from freed buffers.
+// fp32 accumulators in tensor memory; the solve is fp32 (16x16 diagonal blocks
+// by substitution on CUDA cores, then two levels of block merging whose small
+// products run as warp-level tf32 MMAs).  Record pieces leave through bulk copies from freed buffers.
 #include <cuda.h>
 
 #include "launch.h"
@@ -131,25 +131,30 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     const uint32_t tmem = *slot;
     const uint32_t lane_base = (uint32_t)(wq * 32) << 16;
 
+    // One thread polls each barrier; the others park on the CTA barrier, which
+    // leaves the issue slots to the co-resident CTA.  tcgen05.fence::after
+    // orders the tensor-memory reads after that barrier.
     auto mma_done = [&]() {
-        const bool mine = mbar_wait(bar_mma, mma_phase, err);
+        const bool mine = (tid == 0) ? mbar_wait(bar_mma, mma_phase, err) : true;
         mma_phase ^= 1;
+        const bool all = __syncthreads_and(mine) != 0;
         tc_fence_after();
-        return __syncthreads_and(mine) != 0;
+        return all;
     };
-    bool ok = __syncthreads_and(mbar_wait(bar_tma, 0, err)) != 0;
+    bool ok = __syncthreads_and((tid == 0) ? mbar_wait(bar_tma, 0, err) : true) != 0;
 
     if (ok) {
         // ---------------------------------------------------------- Gamma and factors (in place)
         const int p = tid & 63, qr = tid >> 6;           // channel pair, token quarter
         const int kb = p >> 5, cb = (p & 31) * 4;
+        float2 lv[16];
+#pragma unroll
+        for (int u = 0; u < 16; ++u) lv[u] = *reinterpret_cast<const float2 *>(la + (qr * 16 + u) * kDK + 2 * p);
         float g0 = 0.f, g1 = 0.f;
 #pragma unroll
         for (int u = 0; u < 16; ++u) {
-            float2 *e = reinterpret_cast<float2 *>(la + (qr * 16 + u) * kDK + 2 * p);
-            const float2 v2 = *e;
-            g0 += v2.x; g1 += v2.y;
-            *e = make_float2(g0, g1);
+            g0 += lv[u].x; g1 += lv[u].y;
+            lv[u] = make_float2(g0, g1);
         }
         tot[qr * kDK + 2 * p] = g0;
         tot[qr * kDK + 2 * p + 1] = g1;
@@ -172,11 +177,11 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         const float ecr0 = ex2_approx((gc0 - gr0) * kLog2e), ecr1 = ex2_approx((gc1 - gr1) * kLog2e);
         uint8_t *eq = sm + L::EQ + kb * 16384, *kh = sm + L::KH + kb * 8192, *kt = sm + L::KT + kb * 8192;
         unsigned int bad = 0;
-#pragma unroll 4
+        const float sh0 = pre0 - gr0, sh1 = pre1 - gr1;
+#pragma unroll
         for (int u = 0; u < 16; ++u) {
             const int t = qr * 16 + u;
-            const float2 gg = *reinterpret_cast<const float2 *>(la + t * kDK + 2 * p);
-            const float x0 = gg.x + pre0 - gr0, x1 = gg.y + pre1 - gr1;
+            const float x0 = lv[u].x + sh0, x1 = lv[u].y + sh1;
             bad |= (fabsf(x0) > kMaxHalfChunkLogDecay) | (fabsf(x1) > kMaxHalfChunkLogDecay);
             const float up0 = ex2_approx(x0 * kLog2e), up1 = ex2_approx(x1 * kLog2e);
             const float dn0 = ex2_approx(-x0 * kLog2e), dn1 = ex2_approx(-x1 * kLog2e);
@@ -279,57 +284,80 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
             }
         }
         __syncthreads();
-        // (b) T_{b+1,b} = -D_{b+1} (A_{b+1,b} D_b) for the pairs (0,1), (2,3);
-        //     thread: pair, row r, four columns
-        if (tid < 128) {
-            const int which = tid >> 6, r = (tid >> 2) & 15, c4 = (tid & 3) * 4;
+        // (b), (c): the merges are small products inside a dependency chain; they
+        // run as warp-level tf32 MMAs (m16n8k8) on the fp32 blocks.  g, c: fragment
+        // coordinates of this lane.
+        const int fg = lane >> 2, fc = lane & 3;
+        // (b) T_{b+1,b} = -D_{b+1} (A_{b+1,b} D_b) for the pairs (0,1), (2,3).
+        //     Warp w < 4: pair w >> 1, 8-column tile w & 1 of the 16x16 block.
+        if (warp < 4) {
+            const int which = warp >> 1, n0 = (warp & 1) * 8;
             const int R0 = 16 + 32 * which, C0 = 32 * which;
-            float x0 = 0.f, x1 = 0.f, x2 = 0.f, x3 = 0.f;
+            float d[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-            for (int k = 0; k < 16; ++k) {
-                const float a = Af[af_off(R0 + r, C0 + k)];
-                const float4 d = *reinterpret_cast<const float4 *>(Tf + af_off(C0 + k, C0 + c4));
-                x0 += a * d.x; x1 += a * d.y; x2 += a * d.z; x3 += a * d.w;
+            for (int k0 = 0; k0 < 16; k0 += 8) {
+                mma_tf32(d, to_tf32(Af[af_off(R0 + fg, C0 + k0 + fc)]), to_tf32(Af[af_off(R0 + fg + 8, C0 + k0 + fc)]),
+                         to_tf32(Af[af_off(R0 + fg, C0 + k0 + fc + 4)]), to_tf32(Af[af_off(R0 + fg + 8, C0 + k0 + fc + 4)]),
+                         to_tf32(Tf[af_off(C0 + k0 + fc, C0 + n0 + fg)]), to_tf32(Tf[af_off(C0 + k0 + fc + 4, C0 + n0 + fg)]));
             }
-            *reinterpret_cast<float4 *>(Xs + which * 256 + r * 16 + c4) = make_float4(x0, x1, x2, x3);
+            float *x = Xs + which * 256;  // X[16][16]
+            x[fg * 16 + n0 + 2 * fc] = d[0];
+            x[fg * 16 + n0 + 2 * fc + 1] = d[1];
+            x[(fg + 8) * 16 + n0 + 2 * fc] = d[2];
+            x[(fg + 8) * 16 + n0 + 2 * fc + 1] = d[3];
         }
         __syncthreads();
-        if (tid < 128) {
-            const int which = tid >> 6, r = (tid >> 2) & 15, c4 = (tid & 3) * 4;
+        if (warp < 4) {
+            const int which = warp >> 1, n0 = (warp & 1) * 8;
             const int R0 = 16 + 32 * which, C0 = 32 * which;
-            float y0 = 0.f, y1 = 0.f, y2 = 0.f, y3 = 0.f;
+            const float *x = Xs + which * 256;
+            float d[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-            for (int k = 0; k < 16; ++k) {
-                const float d = Tf[af_off(R0 + r, R0 + k)];
-                const float4 x = *reinterpret_cast<const float4 *>(Xs + which * 256 + k * 16 + c4);
-                y0 += d * x.x; y1 += d * x.y; y2 += d * x.z; y3 += d * x.w;
+            for (int k0 = 0; k0 < 16; k0 += 8) {
+                mma_tf32(d, to_tf32(Tf[af_off(R0 + fg, R0 + k0 + fc)]), to_tf32(Tf[af_off(R0 + fg + 8, R0 + k0 + fc)]),
+                         to_tf32(Tf[af_off(R0 + fg, R0 + k0 + fc + 4)]), to_tf32(Tf[af_off(R0 + fg + 8, R0 + k0 + fc + 4)]),
+                         to_tf32(x[(k0 + fc) * 16 + n0 + fg]), to_tf32(x[(k0 + fc + 4) * 16 + n0 + fg]));
             }
-            *reinterpret_cast<float4 *>(Tf + af_off(R0 + r, C0 + c4)) = make_float4(-y0, -y1, -y2, -y3);
+            Tf[af_off(R0 + fg, C0 + n0 + 2 * fc)] = -d[0];
+            Tf[af_off(R0 + fg, C0 + n0 + 2 * fc + 1)] = -d[1];
+            Tf[af_off(R0 + fg + 8, C0 + n0 + 2 * fc)] = -d[2];
+            Tf[af_off(R0 + fg + 8, C0 + n0 + 2 * fc + 1)] = -d[3];
         }
         __syncthreads();
-        // (c) T[32:64, 0:32] = -T_BB (A[32:64, 0:32] T_AA); thread: row r, four columns
+        // (c) T[32:64, 0:32] = -T_BB (A[32:64, 0:32] T_AA).  Warp w: 16-row tile w >> 2,
+        //     8-column tile w & 3 of the 32x32 block; T_AA and T_BB are lower triangular.
         {
-            const int r = tid >> 3, c4 = (tid & 7) * 4;
-            float x0 = 0.f, x1 = 0.f, x2 = 0.f, x3 = 0.f;
+            const int m0 = (warp >> 2) * 16, n0 = (warp & 3) * 8;
+            float d[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-            for (int k = 0; k < 32; ++k) {
-                const float a = Af[af_off(32 + r, k)];
-                const float4 tk = *reinterpret_cast<const float4 *>(Tf + af_off(k, c4));
-                x0 += a * tk.x; x1 += a * tk.y; x2 += a * tk.z; x3 += a * tk.w;
+            for (int k0 = 0; k0 < 32; k0 += 8) {
+                if (k0 + 8 <= n0) continue;  // rows k of T_AA above column n0 are zero
+                mma_tf32(d, to_tf32(Af[af_off(32 + m0 + fg, k0 + fc)]), to_tf32(Af[af_off(32 + m0 + fg + 8, k0 + fc)]),
+                         to_tf32(Af[af_off(32 + m0 + fg, k0 + fc + 4)]), to_tf32(Af[af_off(32 + m0 + fg + 8, k0 + fc + 4)]),
+                         to_tf32(Tf[af_off(k0 + fc, n0 + fg)]), to_tf32(Tf[af_off(k0 + fc + 4, n0 + fg)]));
             }
-            *reinterpret_cast<float4 *>(Xs + r * 32 + c4) = make_float4(x0, x1, x2, x3);
+            Xs[(m0 + fg) * 32 + n0 + 2 * fc] = d[0];
+            Xs[(m0 + fg) * 32 + n0 + 2 * fc + 1] = d[1];
+            Xs[(m0 + fg + 8) * 32 + n0 + 2 * fc] = d[2];
+            Xs[(m0 + fg + 8) * 32 + n0 + 2 * fc + 1] = d[3];
         }
         __syncthreads();
         {
-            const int r = tid >> 3, c4 = (tid & 7) * 4;
-            float y0 = 0.f, y1 = 0.f, y2 = 0.f, y3 = 0.f;
+            const int m0 = (warp >> 2) * 16, n0 = (warp & 3) * 8;
+            float d[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-            for (int k = 0; k < 32; ++k) {
-                const float tb = Tf[af_off(32 + r, 32 + k)];
-                const float4 x = *reinterpret_cast<const float4 *>(Xs + k * 32 + c4);
-                y0 += tb * x.x; y1 += tb * x.y; y2 += tb * x.z; y3 += tb * x.w;
+            for (int k0 = 0; k0 < 32; k0 += 8) {
+                if (k0 >= m0 + 16) continue;  // columns k of T_BB right of row m0 + 15 are zero
+                mma_tf32(d, to_tf32(Tf[af_off(32 + m0 + fg, 32 + k0 + fc)]),
+                         to_tf32(Tf[af_off(32 + m0 + fg + 8, 32 + k0 + fc)]),
+                         to_tf32(Tf[af_off(32 + m0 + fg, 32 + k0 + fc + 4)]),
+                         to_tf32(Tf[af_off(32 + m0 + fg + 8, 32 + k0 + fc + 4)]),
+                         to_tf32(Xs[(k0 + fc) * 32 + n0 + fg]), to_tf32(Xs[(k0 + fc + 4) * 32 + n0 + fg]));
             }
-            *reinterpret_cast<float4 *>(Tf + af_off(32 + r, c4)) = make_float4(-y0, -y1, -y2, -y3);
+            Tf[af_off(32 + m0 + fg, n0 + 2 * fc)] = -d[0];
+            Tf[af_off(32 + m0 + fg, n0 + 2 * fc + 1)] = -d[1];
+            Tf[af_off(32 + m0 + fg + 8, n0 + 2 * fc)] = -d[2];
+            Tf[af_off(32 + m0 + fg + 8, n0 + 2 * fc + 1)] = -d[3];
         }
         __syncthreads();
         // (d) T -> bf16 operand rows 0..63 of [T;PT] (A has served its purpose)
@@ -448,11 +476,14 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
             }
             umma_commit(bar_mma);
         }
-        const bool mine = mbar_wait(bar_mma, mma_phase, err);
+        bool mine = true;
+        if (tid == 0) {
+            mine = mbar_wait(bar_mma, mma_phase, err);
+            bulk_wait_read_all();  // PU0 has left TO before N is staged there
+        }
         mma_phase ^= 1;
-        if (tid == 0) bulk_wait_read_all();  // PU0 has left TO before N is staged there
-        tc_fence_after();
         ok = __syncthreads_and(mine) != 0;
+        tc_fence_after();
     }
 
     if (ok) {

@@ -5,8 +5,10 @@
 // part (the chain kernel, one CTA per (batch, head, value tile) walking the
 // chunks in order).  Prep records travel through a workspace in device memory.
 // The sequence is processed in windows of WC chunks so that the workspace of
-// one window stays small enough to live in L2 between the two kernels; the
-// state crosses window boundaries through a carry buffer (or S_T / S0).
+// one window stays small enough to live in L2 between the kernels; the state
+// crosses window boundaries through a carry buffer (or S_T / S0).  The
+// allocating entry point overlaps the windows on internal streams; the
+// no-allocation entry point runs them in order on the caller's stream.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -119,18 +121,119 @@ cudaError_t run_fwd_tc(const FwdArgs &a, const FwdTcPlan &p, uint8_t *ws)
     return cudaSuccess;
 }
 
+namespace {
+
+// Streams and events of the overlapped schedule, one set per device, created on
+// first use and kept for the life of the process.  The chain stream has the
+// highest priority so that its CTAs are dispatched ahead of pending prep CTAs.
+struct StreamSet {
+    std::mutex mu;
+    cudaStream_t prep = nullptr, chain = nullptr, out = nullptr;
+    cudaEvent_t start = nullptr, ev_p[4] = {}, ev_c[4] = {}, ev_o[4] = {};
+    bool ready = false;
+};
+
+StreamSet *stream_set(int dev)
+{
+    static StreamSet sets[64];
+    if (dev < 0 || dev >= 64) return nullptr;
+    StreamSet &ss = sets[dev];
+    std::lock_guard<std::mutex> lock(ss.mu);
+    if (!ss.ready) {
+        int lo = 0, hi = 0;
+        if (cudaDeviceGetStreamPriorityRange(&lo, &hi) != cudaSuccess) return nullptr;
+        if (cudaStreamCreateWithPriority(&ss.chain, cudaStreamNonBlocking, hi) != cudaSuccess ||
+            cudaStreamCreateWithFlags(&ss.prep, cudaStreamNonBlocking) != cudaSuccess ||
+            cudaStreamCreateWithFlags(&ss.out, cudaStreamNonBlocking) != cudaSuccess ||
+            cudaEventCreateWithFlags(&ss.start, cudaEventDisableTiming) != cudaSuccess)
+            return nullptr;
+        for (int i = 0; i < 4; ++i)
+            if (cudaEventCreateWithFlags(&ss.ev_p[i], cudaEventDisableTiming) != cudaSuccess ||
+                cudaEventCreateWithFlags(&ss.ev_c[i], cudaEventDisableTiming) != cudaSuccess ||
+                cudaEventCreateWithFlags(&ss.ev_o[i], cudaEventDisableTiming) != cudaSuccess)
+                return nullptr;
+        ss.ready = true;
+    }
+    return &ss;
+}
+
+// Overlapped schedule over two workspace halves (window w uses half w % 2):
+//   prep stream:   [wait chain(w-2), out(w-2)]  prep(w)  -> ev_p[w]
+//   chain stream:  [wait prep(w)]               chain(w) -> ev_c[w]
+//   out stream:    [wait chain(w)]              out(w)   -> ev_o[w]
+// so prep of the next window runs while the chain walks the current one.  The
+// caller's stream forks into the three at the start and joins them at the end.
+cudaError_t run_fwd_tc_overlapped(const FwdArgs &a, const FwdTcPlan &p, uint8_t *ws, StreamSet &ss)
+{
+    CUtensorMap maps[6];
+    const auto BF = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+    if (!make_map(&maps[0], a.q, BF, 2, 128, a.H, a.T, a.B, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map(&maps[1], a.k, BF, 2, 128, a.H, a.T, a.B, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map(&maps[2], a.b, BF, 2, 128, a.H, a.T, a.B, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map(&maps[3], a.log_alpha, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, 128, a.H, a.T, a.B, 128,
+                  CU_TENSOR_MAP_SWIZZLE_NONE) ||
+        !make_map(&maps[4], a.v, BF, 2, a.dv, a.H, a.T, a.B, a.dv, CU_TENSOR_MAP_SWIZZLE_NONE) ||
+        !make_map(&maps[5], a.w, BF, 2, a.dv, a.H, a.T, a.B, a.dv, CU_TENSOR_MAP_SWIZZLE_NONE))
+        return cudaErrorInvalidValue;
+    const size_t half = p.rec_total + p.sref_total;
+    float *carry = p.carry_bytes ? reinterpret_cast<float *>(ws + 2 * half) : nullptr;
+    cudaError_t e = cudaEventRecord(ss.start, a.stream);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(ss.prep, ss.start, 0);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(ss.chain, ss.start, 0);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(ss.out, ss.start, 0);
+    for (int w = 0; w < p.nwindows && e == cudaSuccess; ++w) {
+        const int c0 = w * p.wc, slot = w & 3;
+        const int ncw = (p.nchunks - c0 < p.wc) ? p.nchunks - c0 : p.wc;
+        uint8_t *recs = ws + (w & 1) * half, *srefs = recs + p.rec_total;
+        const float *S_in = (w == 0) ? a.S0 : carry;
+        float *S_out = (w == p.nwindows - 1) ? a.S_T : carry;
+        FwdArgs ap = a, ac = a, ao = a;
+        ap.stream = ss.prep;
+        ac.stream = ss.chain;
+        ao.stream = ss.out;
+        if (w >= 2) {
+            e = cudaStreamWaitEvent(ss.prep, ss.ev_c[(w - 2) & 3], 0);
+            if (e == cudaSuccess) e = cudaStreamWaitEvent(ss.prep, ss.ev_o[(w - 2) & 3], 0);
+        }
+        if (e == cudaSuccess) e = launch_prep(ap, maps, recs, c0, ncw, p.wc);
+        if (e == cudaSuccess) e = cudaEventRecord(ss.ev_p[slot], ss.prep);
+        if (e == cudaSuccess) e = cudaStreamWaitEvent(ss.chain, ss.ev_p[slot], 0);
+        if (e == cudaSuccess) e = launch_chain(ac, p.dvt, recs, srefs, S_in, S_out, ncw, p.wc);
+        if (e == cudaSuccess) e = cudaEventRecord(ss.ev_c[slot], ss.chain);
+        if (e == cudaSuccess) e = cudaStreamWaitEvent(ss.out, ss.ev_c[slot], 0);
+        if (e == cudaSuccess) e = launch_out(ao, recs, srefs, c0, ncw, p.wc);
+        if (e == cudaSuccess) e = cudaEventRecord(ss.ev_o[slot], ss.out);
+    }
+    // join: the caller's stream waits for the last chain and the last two outputs
+    if (e == cudaSuccess && p.nwindows > 0) {
+        const int last = p.nwindows - 1;
+        e = cudaStreamWaitEvent(a.stream, ss.ev_c[last & 3], 0);
+        if (e == cudaSuccess) e = cudaStreamWaitEvent(a.stream, ss.ev_o[last & 3], 0);
+        if (e == cudaSuccess && last >= 1) e = cudaStreamWaitEvent(a.stream, ss.ev_o[(last - 1) & 3], 0);
+    }
+    return e;
+}
+
+}  // namespace
+
 cudaError_t launch_fwd_tc(const FwdArgs &a)
 {
-    const FwdTcPlan p = plan_fwd_tc(a.B, a.T, a.H, a.dv, kWindowBudgetBytes);
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     cudaMemPool_t pool = workspace_pool(dev);
-    if (!pool) return cudaErrorMemoryAllocation;
+    StreamSet *ss = stream_set(dev);
+    if (!pool || !ss) return cudaErrorMemoryAllocation;
+    // two window halves of half the budget each
+    FwdTcPlan p = plan_fwd_tc(a.B, a.T, a.H, a.dv, kWindowBudgetBytes / 2);
+    const size_t bytes = 2 * (p.rec_total + p.sref_total) + p.carry_bytes;
     void *ws = nullptr;
-    e = cudaMallocFromPoolAsync(&ws, p.ws_bytes, pool, a.stream);
+    e = cudaMallocFromPoolAsync(&ws, bytes, pool, a.stream);
     if (e != cudaSuccess) return e;
-    e = run_fwd_tc(a, p, static_cast<uint8_t *>(ws));
+    {
+        std::lock_guard<std::mutex> lock(ss->mu);
+        e = run_fwd_tc_overlapped(a, p, static_cast<uint8_t *>(ws), *ss);
+    }
     const cudaError_t f = cudaFreeAsync(ws, a.stream);
     return e != cudaSuccess ? e : f;
 }

@@ -84,6 +84,26 @@ __device__ __forceinline__ float ex2_approx(float x)
     return y;
 }
 
+// Warp-level D += A B on tf32 operands, m16n8k8 (A row-major 16x8, B column-major
+// 8x8, fp32 accumulators).  Fragment of lane l (g = l / 4, c = l % 4):
+//   a0 = A[g][c], a1 = A[g+8][c], a2 = A[g][c+4], a3 = A[g+8][c+4]
+//   b0 = B[c][g], b1 = B[c+4][g]
+//   d0 = D[g][2c], d1 = D[g][2c+1], d2 = D[g+8][2c], d3 = D[g+8][2c+1]
+__device__ __forceinline__ uint32_t to_tf32(float x)
+{
+    uint32_t r;
+    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+    return r;
+}
+__device__ __forceinline__ void mma_tf32(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                         uint32_t b0, uint32_t b1)
+{
+    asm volatile("mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+                 "{%0,%1,%2,%3};"
+                 : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+                 : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
 // fp32 64x64 matrix in shared memory with 16-byte chunks XOR-swizzled by row,
 // so that row-per-thread float4 stores and column walks avoid bank conflicts.
 __device__ __forceinline__ int af_off(int t, int s) { return t * 64 + ((((s >> 2) ^ (t & 15)) << 2) | (s & 3)); }
