@@ -37,8 +37,10 @@ DEC = synth.DECODE_F32
 N_INPUT_SETS = 4  # rotating input sets: 4 x 136 MB > 126 MB of L2
 
 # dram__bytes_read.sum + dram__bytes_write.sum per launch from an ncu capture of
-# the current kernels (None once a kernel has changed since the capture).
-NCU_TRAFFIC_BYTES = {"fwd": None, "decode": None}
+# the current kernels (None once a kernel has changed since the capture).  The
+# forward is three kernels per window (profiles/*_layer_bf16.md hold each one);
+# decode: profiles/decode_kernel_decode_b256.md.
+NCU_TRAFFIC_BYTES = {"fwd": None, "decode": 281.03e6 + 215.97e6}
 
 
 def peaks():
@@ -357,7 +359,8 @@ def main():
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
                          "frac": achieved / hbm_peak, "traffic": NCU_TRAFFIC_BYTES["fwd"],
                          "peak_kind": peak_kind, "algorithmic_bytes_per_launch": alg_bytes,
-                         "mean_launch_us": mean_launch_ms * 1e3, "kernel": "gdn2_fwd_chunked"},
+                         "mean_launch_us": mean_launch_ms * 1e3,
+                         "kernel": "gdn2_fwd_chunked (prep + chain + output kernels per window)"},
             "decode": {"workload": dc.name, "us_per_step": dec_ms * 1e3, "hbm_gbs": dec_gbs,
                        "frac": dec_gbs / hbm_peak, "peak": hbm_peak,
                        "algorithmic_bytes_per_step": dec_bytes, "steps": args.decode_steps,
@@ -366,7 +369,7 @@ def main():
             "cpu_baseline": cpu,
             "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "steps": e2e_steps},
-            "gpu_launches": args.steps,
+            "gpu_launches": args.steps * g.gdn2_fwd_chunked_launches(c.B, c.T, c.H, c.dk, c.dv, c.dtype),
             "clocks": clk,
         }
         print(json.dumps(line), flush=True)

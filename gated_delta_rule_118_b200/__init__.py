@@ -31,7 +31,7 @@ GDN2_BF16 = 1
 
 # Every symbol include/gdn2.h declares.
 EXPORTED = ("gdn2_fwd_chunked", "gdn2_fwd_chunked_noalloc", "gdn2_decode_step",
-            "gdn2_check_device_error", "gdn2_status_string")
+            "gdn2_check_device_error", "gdn2_fwd_chunked_launches", "gdn2_status_string")
 
 _lib = None
 
@@ -59,6 +59,8 @@ def lib() -> ctypes.CDLL:
         L.gdn2_decode_step.restype = ci
         L.gdn2_check_device_error.argtypes = [vp]
         L.gdn2_check_device_error.restype = ci
+        L.gdn2_fwd_chunked_launches.argtypes = [ci] * 6
+        L.gdn2_fwd_chunked_launches.restype = ci
         L.gdn2_status_string.argtypes = [ci]
         L.gdn2_status_string.restype = ctypes.c_char_p
         _lib = L
@@ -152,6 +154,12 @@ def gdn2_decode_step(q, k, v, b, w, log_alpha, S, o=None, *, stream=None, check=
 def gdn2_check_device_error(stream=None) -> int:
     """Synchronise ``stream`` and return (and clear) the device error status."""
     return int(lib().gdn2_check_device_error(_stream(stream)))
+
+
+def gdn2_fwd_chunked_launches(B, T, H, dk, dv, dtype=torch.bfloat16) -> int:
+    """Kernel launches one gdn2_fwd_chunked call makes for this problem."""
+    code = GDN2_BF16 if dtype == torch.bfloat16 else GDN2_F32
+    return int(lib().gdn2_fwd_chunked_launches(B, T, H, dk, dv, code))
 
 
 def gdn2_status_string(status: int) -> str:

@@ -147,6 +147,15 @@ extern "C" gdn2_status gdn2_check_device_error(gdn2_stream_t stream)
     return GDN2_OK;
 }
 
+extern "C" int gdn2_fwd_chunked_launches(int B, int T, int H, int dk, int dv, gdn2_dtype dtype)
+{
+    if ((dtype != GDN2_F32 && dtype != GDN2_BF16) || B <= 0 || H <= 0 || T < 0) return -1;
+    if (check_dims(dk, dv) != GDN2_OK || B > 65535 || H > 65535) return -1;
+    if (T == 0) return 0;
+    if (dtype == GDN2_BF16 && dk == 128) return 3 * plan_fwd_tc(B, T, H, dv, kWindowBudgetBytes / 2).nwindows;
+    return 1;
+}
+
 extern "C" const char *gdn2_status_string(gdn2_status status)
 {
     switch (status) {

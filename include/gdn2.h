@@ -157,6 +157,14 @@ gdn2_status gdn2_decode_step(const void *q, const void *k, const void *v,
  */
 gdn2_status gdn2_check_device_error(gdn2_stream_t stream);
 
+/*
+ * gdn2_fwd_chunked_launches -- number of kernel launches one gdn2_fwd_chunked
+ * call makes for this problem (host-only arithmetic, no CUDA call; -1 for
+ * arguments gdn2_fwd_chunked would reject).  The bf16 path launches three
+ * kernels per window of chunks; the fp32 path launches one kernel.
+ */
+int gdn2_fwd_chunked_launches(int B, int T, int H, int dk, int dv, gdn2_dtype dtype);
+
 /* Human-readable name of a status code (static storage, never NULL). */
 const char *gdn2_status_string(gdn2_status status);
 

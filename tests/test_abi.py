@@ -35,6 +35,14 @@ def test_library_is_built_for_sm100a(lib):
     assert build.ARCH == ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 
+def test_launch_count_query(lib):
+    assert g.gdn2_fwd_chunked_launches(1, 4096, 16, 128, 128) % 3 == 0
+    assert g.gdn2_fwd_chunked_launches(1, 4096, 16, 128, 128) >= 3
+    assert g.gdn2_fwd_chunked_launches(1, 256, 2, 64, 64, __import__("torch").float32) == 1
+    assert g.gdn2_fwd_chunked_launches(1, 0, 2, 128, 128) == 0
+    assert g.gdn2_fwd_chunked_launches(0, 10, 2, 128, 128) == -1
+
+
 def test_status_strings(lib):
     for code in range(10):
         s = g.status_string(code)
