@@ -2,7 +2,7 @@
 // device allocation at all.
 //
 // gdn2_fwd_chunked draws the workspace of its bf16 tensor-core path (the
-// per-chunk prep records, the exported Sref images and the state carried
+// per-chunk prep records, the exported state images and the state carried
 // between windows) from a stream-ordered memory pool.  Some callers cannot let
 // a library allocate: a runtime that hands out all device memory itself at
 // start-up, code that must never enter the driver's allocator on its hot loop
@@ -88,8 +88,8 @@ extern "C" gdn2_status gdn2_fwd_chunked_noalloc(const void *q, const void *k, co
         // Records of as many chunks as fit, after room for the carried state.
         const size_t carry = (size_t)B * H * 128 * dv * sizeof(float);
         const size_t rec = (dv == 128) ? Record<128>::BYTES : Record<64>::BYTES;
-        const size_t sref = (dv == 128) ? SrefSlot<128>::BYTES : SrefSlot<64>::BYTES;
-        const size_t per_chunk = (size_t)B * H * (rec + sref);
+        const size_t sx = (dv == 128) ? SxSlot<128>::BYTES : SxSlot<64>::BYTES;
+        const size_t per_chunk = (size_t)B * H * (rec + sx);
         if (carry >= kNoAllocScratchBytes || per_chunk > kNoAllocScratchBytes - carry) return GDN2_ERR_SCRATCH_LIMIT;
         plan = plan_fwd_tc(B, T, H, dv, kNoAllocScratchBytes - carry);
         if (plan.ws_bytes > kNoAllocScratchBytes) return GDN2_ERR_SCRATCH_LIMIT;

@@ -3,11 +3,12 @@
 // The query reads the updated state ("Gated DeltaNet-2", iplexlaw.co.kr,
 // section "Decisiones independientes en dos ejes"); in the chunkwise form the
 // outputs of a chunk are
-//   O = P T Z + (Qhat - P T Ehat) Sref = PU0 + Q' Sref,
-// with PU0 and Q' from the chunk's prep record and Sref = e^{Gamma_r} S the
+//   O = P T Z + (Qhat - P T Ehat) Diag(e^{Gamma_r}) S = PT Z + QS Sx,
+// with PT, Z and QS from the chunk's prep record and Sx the bf16 image of the
 // incoming state exported by the chain kernel.  Nothing here is sequential in
-// the chunk index, so one CTA per (batch, head, chunk) runs one UMMA
-// (M = 64 tokens, N = dv, K = dk = 128) and writes its 64 output rows.
+// the chunk index, so one CTA per (batch, head, chunk) accumulates the two
+// products in tensor memory (M = 64 tokens, N = dv; K = 64 tokens, then K = dk)
+// and writes its 64 output rows.
 #include "launch.h"
 #include "tc_common.cuh"
 
@@ -20,18 +21,20 @@ constexpr int kOutThreads = 128;
 
 template <int DV>
 struct OutLayout {
-    static constexpr int QP = 0;                    // Q' [64][128] K-major, 2 blocks of 8 KB
-    static constexpr int SR = 16384;                // Sref, DV/64 blocks of [128][64]
-    static constexpr int PU = SR + 128 * DV * 2;    // PU0, DV/64 blocks of [64][64]
-    static constexpr int TX = PU + 64 * DV * 2;
+    static constexpr int QS = 0;                    // QS [64][128] K-major, 2 blocks of 8 KB
+    static constexpr int PT = 16384;                // PT [64][64] K-major, 8 KB
+    static constexpr int Z = 24576;                 // Z, DV/64 blocks of [64][64] (MN-major)
+    static constexpr int SX = Z + 64 * DV * 2;      // Sx, DV/64 blocks of [128][64] (MN-major)
+    static constexpr int TX = SX + 128 * DV * 2;
     static constexpr int BAR = TX;
     static constexpr int SLOT = BAR + 16;
     static constexpr int BYTES = SLOT + 16 + 1024;
+    static_assert(SX % 1024 == 0, "swizzle atoms");
 };
 
 template <int DV>
 __global__ void __launch_bounds__(kOutThreads)
-out_kernel(const uint8_t *__restrict__ ws, const uint8_t *__restrict__ sref, bf16 *__restrict__ o, int Tlen,
+out_kernel(const uint8_t *__restrict__ ws, const uint8_t *__restrict__ sx, bf16 *__restrict__ o, int Tlen,
            int H, int c0, int WC, unsigned int *err)
 {
     using L = OutLayout<DV>;
@@ -51,9 +54,10 @@ out_kernel(const uint8_t *__restrict__ ws, const uint8_t *__restrict__ sref, bf1
         fence_mbar_init();
         const uint8_t *rec = ws + idx * R::BYTES;
         mbar_arrive_expect_tx(bar, (uint32_t)L::TX);
-        bulk_load(sm + L::QP, rec + R::QP, 16384, bar);
-        bulk_load(sm + L::SR, sref + idx * SrefSlot<DV>::BYTES, 128 * DV * 2, bar);
-        bulk_load(sm + L::PU, rec + R::PU, 64 * DV * 2, bar);
+        bulk_load(sm + L::QS, rec + R::QS, 16384, bar);
+        bulk_load(sm + L::PT, rec + R::PT, 8192, bar);
+        bulk_load(sm + L::Z, rec + R::Z, 64 * DV * 2, bar);
+        bulk_load(sm + L::SX, sx + idx * SxSlot<DV>::BYTES, 128 * DV * 2, bar);
     }
     if (warp == 0) {
         tmem_alloc(slot, DV);
@@ -64,18 +68,22 @@ out_kernel(const uint8_t *__restrict__ ws, const uint8_t *__restrict__ sref, bf1
     tc_fence_after();
     const uint32_t tmem = *slot;
 
-    bool ok = mbar_wait(bar, 0, err);
+    bool ok = (tid == 0) ? mbar_wait(bar, 0, err) : true;
     if (tid == 0 && ok) {
         const uint32_t id = idesc_bf16(64, DV, 0, 1);
 #pragma unroll
+        for (int ks = 0; ks < 4; ++ks)
+            umma_bf16(tmem, smem_desc(sbase + L::PT + ks * 32, 16, 1024, kSw128),
+                      smem_desc(sbase + L::Z + ks * 2048, 8192, 1024, kSw128), id, ks > 0);
+#pragma unroll
         for (int ks = 0; ks < 8; ++ks)
-            umma_bf16(tmem, smem_desc(sbase + L::QP + (ks >> 2) * 8192 + (ks & 3) * 32, 16, 1024, kSw128),
-                      smem_desc(sbase + L::SR + ks * 2048, 16384, 1024, kSw128), id, ks > 0);
+            umma_bf16(tmem, smem_desc(sbase + L::QS + (ks >> 2) * 8192 + (ks & 3) * 32, 16, 1024, kSw128),
+                      smem_desc(sbase + L::SX + ks * 2048, 16384, 1024, kSw128), id, 1);
         umma_commit(bar + 1);
+        ok = mbar_wait(bar + 1, 0, err);
     }
     ok = __syncthreads_and(ok) != 0;
     if (ok) {
-        mbar_wait(bar + 1, 0, err);
         tc_fence_after();
         // M = 64 accumulator: row 16*warp + l sits in TMEM lane 32*warp + l (l < 16)
         const int t = warp * 16 + lane;
@@ -84,18 +92,16 @@ out_kernel(const uint8_t *__restrict__ ws, const uint8_t *__restrict__ sref, bf1
         bf16 *dst = o + (((long)bi * Tlen + ct0 + t) * H + h) * (long)DV;
         const uint32_t lane_addr = tmem + ((uint32_t)(warp * 32) << 16);
 #pragma unroll
-        for (int j = 0; j < DV; j += 16) {
-            float ov[16], pv[16];
-            tmem_ld16(lane_addr + j, ov);
+        for (int j = 0; j < DV; j += 32) {
+            float a[16], b[16];
+            tmem_ld16(lane_addr + j, a);
+            tmem_ld16(lane_addr + j + 16, b);
             tmem_ld_wait();
             if (live) {
-                const uint8_t *pb = sm + L::PU + (j >> 6) * 8192;
-                unpack8(*reinterpret_cast<const uint4 *>(pb + swz_off(t, (j & 63) * 2, 128)), pv);
-                unpack8(*reinterpret_cast<const uint4 *>(pb + swz_off(t, (j & 63) * 2 + 16, 128)), pv + 8);
-#pragma unroll
-                for (int u = 0; u < 16; ++u) ov[u] += pv[u];
-                *reinterpret_cast<uint4 *>(dst + j) = pack8(ov);
-                *reinterpret_cast<uint4 *>(dst + j + 8) = pack8(ov + 8);
+                *reinterpret_cast<uint4 *>(dst + j) = pack8(a);
+                *reinterpret_cast<uint4 *>(dst + j + 8) = pack8(a + 8);
+                *reinterpret_cast<uint4 *>(dst + j + 16) = pack8(b);
+                *reinterpret_cast<uint4 *>(dst + j + 24) = pack8(b + 8);
             }
         }
     }
@@ -108,22 +114,22 @@ out_kernel(const uint8_t *__restrict__ ws, const uint8_t *__restrict__ sref, bf1
 }
 
 template <int DV>
-cudaError_t launch_out_impl(const FwdArgs &a, const uint8_t *ws, const uint8_t *sref, int c0, int ncw, int WC)
+cudaError_t launch_out_impl(const FwdArgs &a, const uint8_t *ws, const uint8_t *sx, int c0, int ncw, int WC)
 {
     using L = OutLayout<DV>;
     auto kern = out_kernel<DV>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::BYTES);
     if (e != cudaSuccess) return e;
     dim3 grid(ncw, a.H, a.B);
-    kern<<<grid, kOutThreads, L::BYTES, a.stream>>>(ws, sref, (bf16 *)a.o, a.T, a.H, c0, WC, a.err);
+    kern<<<grid, kOutThreads, L::BYTES, a.stream>>>(ws, sx, (bf16 *)a.o, a.T, a.H, c0, WC, a.err);
     return cudaGetLastError();
 }
 
 }  // namespace
 
-cudaError_t launch_out(const FwdArgs &a, const uint8_t *ws, const uint8_t *sref, int c0, int ncw, int WC)
+cudaError_t launch_out(const FwdArgs &a, const uint8_t *ws, const uint8_t *sx, int c0, int ncw, int WC)
 {
-    return a.dv == 128 ? launch_out_impl<128>(a, ws, sref, c0, ncw, WC) : launch_out_impl<64>(a, ws, sref, c0, ncw, WC);
+    return a.dv == 128 ? launch_out_impl<128>(a, ws, sx, c0, ncw, WC) : launch_out_impl<64>(a, ws, sx, c0, ncw, WC);
 }
 
 }  // namespace gdn2

@@ -10,20 +10,22 @@
 //   Ehat = e^{Gamma-Gamma_r} b k    Qhat = e^{Gamma-Gamma_r} q
 //   Khat = e^{Gamma_r-Gamma} k      Ktil = e^{Gamma_C-Gamma} k    Z = w v
 //   A = strict_lower(Ehat Khat^T)   P = lower(Qhat Khat^T)   T = (I + A)^{-1}
-//   W = T Ehat   U0 = T Z   Q' = Qhat - P W   PU0 = P T Z
-//   G = Ktil^T W                    N = Ktil^T U0
-// so that, with Sref = e^{Gamma_r} S for the incoming state S,
-//   S_next = e^{Gamma_C} S + N - G Sref      O = PU0 + Q' Sref.
-// G, N, Q', PU0 and the decays form the chunk's record in the workspace.
+//   Y = Ktil^T T    PT = P T    G = Y Ehat    Q' = Qhat - PT Ehat
+// and the record keeps NG = -G Diag(e^{Gamma_r}), QS = Q' Diag(e^{Gamma_r}),
+// Y, PT, Z and e^{Gamma_C}, so that for the incoming state S
+//   S_next = e^{Gamma_C} S + NG S + Y Z        O = QS S + PT Z.
+// Nothing here depends on the values except Z, which is a plain product.
 //
 // Layout of the work on one SM: the CTA fits in half of the shared memory,
 // tensor memory and register file, so two chunks are in flight per SM and one
 // hides the other's load and UMMA latencies.  q, k, b and log_alpha arrive by
 // TMA straight into the operand buffers and the factors are formed in place;
-// v and w are read with plain vector loads.  Products are tcgen05 UMMAs with
-// fp32 accumulators in tensor memory; the solve is fp32 (16x16 diagonal blocks
-// by substitution on CUDA cores, then two levels of block merging whose small
-// products run as warp-level tf32 MMAs).  Record pieces leave through bulk copies from freed buffers.
+// v and w are read with plain vector loads and Z goes straight to the record.
+// Products are tcgen05 UMMAs with fp32 accumulators in tensor memory, three
+// round trips in all (Gram; Y and PT; G and P T Ehat); the solve is fp32
+// (16x16 diagonal blocks by substitution on CUDA cores, then two levels of
+// block merging whose small products run as warp-level tf32 MMAs).  Record
+// pieces leave through bulk copies as soon as they are final.
 #include <cuda.h>
 
 #include "launch.h"
@@ -38,20 +40,19 @@ constexpr int kPrepThreads = 256;
 constexpr int kDK = 128;
 
 struct PrepLayout {
-    static constexpr int EQ = 0;          // [Ehat;Qhat]; q and b arrive here; later [.;Q']
-    static constexpr int KH = 32768;      // Khat -> fp32 T -> W operand -> G block 0
-    static constexpr int KT = 49152;      // k arrives here -> Ktil -> G block 1
-    static constexpr int PO = 65536;      // P
-    static constexpr int TO = 73728;      // log_alpha (first half) -> fp32 A -> [T;PT] -> PU0 -> N block 1
-    static constexpr int ZO = 90112;      // log_alpha (second half) -> Z -> U0 operand -> N block 0
-    static constexpr int XS = 106496;     // solve scratch, 4 KB
-    static constexpr int DEC = 110592;    // e^{Gamma_C}, e^{Gamma_r}
-    static constexpr int TOT = 111616;    // quarter totals [4][128]
-    static constexpr int BAR = 113664;
+    static constexpr int EQ = 0;          // [Ehat;Qhat]: b, q arrive here; QS over Qhat at the end
+    static constexpr int KH = 32768;      // Khat -> solve scratch -> Y
+    static constexpr int KT = 49152;      // k arrives here -> Ktil -> PT
+    static constexpr int LA = 65536;      // log_alpha -> fp32 A | fp32 T -> bf16 T over A -> NG
+    static constexpr int PO = 98304;      // Gamma quarter totals -> P
+    static constexpr int DEC = 106496;    // e^{Gamma_C}[128], e^{Gamma_r}[128]
+    static constexpr int BAR = 107520;
     static constexpr int SLOT = BAR + 16;
     static constexpr int BYTES = SLOT + 16 + 1024;
     static constexpr int TX = 3 * 16384 + 32768;  // q, k, b, log_alpha
-    static constexpr uint32_t TM_G = 0, TM_PT = 64, TM_W = 0, TM_U = 128, TMEM_COLS = 256;
+    static constexpr int AF = LA, TF = LA + 16384, TB = LA, XS = KH, TOT = PO;
+    // tensor memory: Gram in [0, 64); then Y in [0, 64), PT in [64, 128); then G in [0, 128), P T Ehat in [128, 256)
+    static constexpr uint32_t TM_GRAM = 0, TM_Y = 0, TM_PT = 64, TM_G = 0, TM_PW = 128, TMEM_COLS = 256;
 };
 static_assert(PrepLayout::BYTES * 2 + 2048 <= 233472, "two CTAs per SM");
 
@@ -84,9 +85,9 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     uint64_t *bar_tma = reinterpret_cast<uint64_t *>(sm + L::BAR);
     uint64_t *bar_mma = bar_tma + 1;
     uint32_t *slot = reinterpret_cast<uint32_t *>(sm + L::SLOT);
-    float *la = reinterpret_cast<float *>(sm + L::TO);  // [64][128] fp32 over TO..ZO
-    float *Af = reinterpret_cast<float *>(sm + L::TO);
-    float *Tf = reinterpret_cast<float *>(sm + L::KH);
+    float *la = reinterpret_cast<float *>(sm + L::LA);  // [64][128] fp32
+    float *Af = reinterpret_cast<float *>(sm + L::AF);
+    float *Tf = reinterpret_cast<float *>(sm + L::TF);
     float *Xs = reinterpret_cast<float *>(sm + L::XS);
     float *dec = reinterpret_cast<float *>(sm + L::DEC);
     float *tot = reinterpret_cast<float *>(sm + L::TOT);
@@ -104,13 +105,14 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
             tma_load_4d(sm + L::EQ + kb * 16384, &tm_b, bar_tma, kb * 64, h, t0, bi);
             tma_load_4d(sm + L::KT + kb * 8192, &tm_k, bar_tma, kb * 64, h, t0, bi);
         }
-        tma_load_4d(sm + L::TO, &tm_la, bar_tma, 0, h, t0, bi);
+        tma_load_4d(sm + L::LA, &tm_la, bar_tma, 0, h, t0, bi);
     }
     if (warp == 0) {
         tmem_alloc(slot, L::TMEM_COLS);
         tmem_relinquish();
     }
     // v and w for Z = w v: plain vector loads, issued before anything waits
+    // (tokens past the sequence end give zero rows of Z)
     constexpr int ZV = 64 * DV / 8 / kPrepThreads;  // 16-byte vectors per thread
     uint4 vv[ZV], wv[ZV];
 #pragma unroll
@@ -208,7 +210,8 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
             }
             umma_commit(bar_mma);
         }
-        // Z = w v while the Gram runs (log_alpha in ZO is no longer needed)
+        // Z = w v while the Gram runs, straight into the record (MN-major operand
+        // blocks of 64 value columns; each warp fills whole 128-byte rows)
 #pragma unroll
         for (int m = 0; m < ZV; ++m) {
             const int idx = tid + m * kPrepThreads;
@@ -218,9 +221,8 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
             unpack8(wv[m], fw);
 #pragma unroll
             for (int u = 0; u < 8; ++u) fz[u] = fv[u] * fw[u];
-            *reinterpret_cast<uint4 *>(sm + L::ZO + (j >> 6) * 8192 + swz_off(t, (j & 63) * 2, 128)) = pack8(fz);
+            *reinterpret_cast<uint4 *>(rec + R::Z + (j >> 6) * 8192 + swz_off(t, (j & 63) * 2, 128)) = pack8(fz);
         }
-        fence_proxy_async_smem();
         ok = mma_done();
     }
 
@@ -229,7 +231,7 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         {
             const int r = wq * 32 + lane;
             float v[32];
-            tmem_ld32(tmem + lane_base + L::TM_G + wh * 32, v);
+            tmem_ld32(tmem + lane_base + L::TM_GRAM + wh * 32, v);
             if (r < 64) {
                 const int t = r;
 #pragma unroll
@@ -252,7 +254,7 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                     *reinterpret_cast<uint4 *>(sm + L::PO + swz_off(t, (wh * 32 + s8) * 2, 128)) = pack8(f);
                 }
             }
-            // T starts as zero; Khat (Gram operand, now consumed) gives its room to T
+            // T starts as zero (log_alpha, consumed by the Gamma scan, gives its room to A and T)
 #pragma unroll
             for (int m = 0; m < 4; ++m)
                 reinterpret_cast<float4 *>(Tf)[tid + m * kPrepThreads] = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -360,7 +362,7 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
             Tf[af_off(32 + m0 + fg + 8, n0 + 2 * fc + 1)] = -d[3];
         }
         __syncthreads();
-        // (d) T -> bf16 operand rows 0..63 of [T;PT] (A has served its purpose)
+        // (d) T -> bf16 operand over A (which has served its purpose)
         {
             const int t = tid >> 2, g = (tid & 3) * 16;
             float f[16];
@@ -369,160 +371,126 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                 const float4 v4 = *reinterpret_cast<const float4 *>(Tf + af_off(t, g + u));
                 f[u] = v4.x; f[u + 1] = v4.y; f[u + 2] = v4.z; f[u + 3] = v4.w;
             }
-            *reinterpret_cast<uint4 *>(sm + L::TO + swz_off(t, g * 2, 128)) = pack8(f);
-            *reinterpret_cast<uint4 *>(sm + L::TO + swz_off(t, g * 2 + 16, 128)) = pack8(f + 8);
+            *reinterpret_cast<uint4 *>(sm + L::TB + swz_off(t, g * 2, 128)) = pack8(f);
+            *reinterpret_cast<uint4 *>(sm + L::TB + swz_off(t, g * 2 + 16, 128)) = pack8(f + 8);
         }
         fence_proxy_async_smem();
         __syncthreads();
 
-        // ---------------------------------------------------------- PT = P T   (M = 64)
+        // ---------------------------------------------------------- Y = Ktil^T T (M = 128),  PT = P T (M = 64)
         if (tid == 0) {
             tc_fence_after();
-            const uint32_t id = idesc_bf16(64, 64, 0, 1);
+            const uint32_t idy = idesc_bf16(128, 64, 1, 1), idp = idesc_bf16(64, 64, 0, 1);
 #pragma unroll
-            for (int ks = 0; ks < 4; ++ks)
-                umma_bf16(tmem + L::TM_PT, smem_desc(sbase + L::PO + ks * 32, 16, 1024, kSw128),
-                          smem_desc(sbase + L::TO + ks * 2048, 8192, 1024, kSw128), id, ks > 0);
+            for (int ks = 0; ks < 4; ++ks) {
+                const uint64_t bt = smem_desc(sbase + L::TB + ks * 2048, 8192, 1024, kSw128);
+                umma_bf16(tmem + L::TM_Y, smem_desc(sbase + L::KT + ks * 2048, 8192, 1024, kSw128), bt, idy, ks > 0);
+                umma_bf16(tmem + L::TM_PT, smem_desc(sbase + L::PO + ks * 32, 16, 1024, kSw128), bt, idp, ks > 0);
+            }
             umma_commit(bar_mma);
         }
         ok = mma_done();
     }
 
     if (ok) {
-        {   // M = 64 accumulator: row 16*wq + l sits in TMEM lane 32*wq + l (l < 16)
-            float v[32];
-            tmem_ld32(tmem + lane_base + L::TM_PT + wh * 32, v);
+        {   // Y row i -> KH ([128][64] K-major);  PT (M = 64: row 16*wq + l in TMEM lane 32*wq + l) -> KT
+            float v0[16], v1[16], p0[16], p1[16];
+            tmem_ld16(tmem + lane_base + L::TM_Y + wh * 32, v0);
+            tmem_ld16(tmem + lane_base + L::TM_Y + wh * 32 + 16, v1);
+            tmem_ld16(tmem + lane_base + L::TM_PT + wh * 32, p0);
+            tmem_ld16(tmem + lane_base + L::TM_PT + wh * 32 + 16, p1);
+            tmem_ld_wait();
+            const int i = wq * 32 + lane;
+            uint8_t *yrow = sm + L::KH;
+            *reinterpret_cast<uint4 *>(yrow + swz_off(i, wh * 64, 128)) = pack8(v0);
+            *reinterpret_cast<uint4 *>(yrow + swz_off(i, wh * 64 + 16, 128)) = pack8(v0 + 8);
+            *reinterpret_cast<uint4 *>(yrow + swz_off(i, wh * 64 + 32, 128)) = pack8(v1);
+            *reinterpret_cast<uint4 *>(yrow + swz_off(i, wh * 64 + 48, 128)) = pack8(v1 + 8);
             if (lane < 16) {
-                const int row = 64 + wq * 16 + lane;
-#pragma unroll
-                for (int s8 = 0; s8 < 32; s8 += 8)
-                    *reinterpret_cast<uint4 *>(sm + L::TO + swz_off(row, (wh * 32 + s8) * 2, 128)) = pack8(v + s8);
+                const int t = wq * 16 + lane;
+                uint8_t *prow = sm + L::KT;
+                *reinterpret_cast<uint4 *>(prow + swz_off(t, wh * 64, 128)) = pack8(p0);
+                *reinterpret_cast<uint4 *>(prow + swz_off(t, wh * 64 + 16, 128)) = pack8(p0 + 8);
+                *reinterpret_cast<uint4 *>(prow + swz_off(t, wh * 64 + 32, 128)) = pack8(p1);
+                *reinterpret_cast<uint4 *>(prow + swz_off(t, wh * 64 + 48, 128)) = pack8(p1 + 8);
             }
         }
         tc_fence_before();
         fence_proxy_async_smem();
         __syncthreads();
 
-        // ---------------------------------------------------------- [W;PW] = [T;PT] Ehat,  [U0;PU0] = [T;PT] Z
+        // ---------------------------------------------------------- G = Y Ehat (M = 128),  PW = PT Ehat (M = 64)
         if (tid == 0) {
             tc_fence_after();
-            const uint32_t idw = idesc_bf16(128, kDK, 0, 1), idz = idesc_bf16(128, DV, 0, 1);
+            const uint32_t idg = idesc_bf16(128, kDK, 0, 1), idw = idesc_bf16(64, kDK, 0, 1);
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks) {
-                const uint64_t ad = smem_desc(sbase + L::TO + ks * 32, 16, 1024, kSw128);
-                umma_bf16(tmem + L::TM_W, ad, smem_desc(sbase + L::EQ + ks * 2048, 16384, 1024, kSw128), idw, ks > 0);
-                umma_bf16(tmem + L::TM_U, ad, smem_desc(sbase + L::ZO + ks * 2048, 8192, 1024, kSw128), idz, ks > 0);
+                const uint64_t be = smem_desc(sbase + L::EQ + ks * 2048, 16384, 1024, kSw128);
+                umma_bf16(tmem + L::TM_G, smem_desc(sbase + L::KH + ks * 32, 16, 1024, kSw128), be, idg, ks > 0);
+                umma_bf16(tmem + L::TM_PW, smem_desc(sbase + L::KT + ks * 32, 16, 1024, kSw128), be, idw, ks > 0);
             }
             umma_commit(bar_mma);
+            bulk_store(rec + R::Y, sm + L::KH, 16384);
+            bulk_store(rec + R::PT, sm + L::KT, 8192);
+            bulk_commit();
         }
         ok = mma_done();
     }
 
     if (ok) {
-        {
-            const int r = wq * 32 + lane;
-            const int t = r & 63;
-            // W rows -> W operand (KH); PW rows -> Q' = Qhat - PW, in place over Qhat
+        const float *er = dec + kDK;
+        {   // NG = -G Diag(e^{Gamma_r}): row i, columns [64*wh, +64) -> block wh of NG (over A/T)
+            const int i = wq * 32 + lane;
 #pragma unroll
             for (int part = 0; part < 64; part += 32) {
                 float v[32];
-                tmem_ld32(tmem + lane_base + L::TM_W + wh * 64 + part, v);
+                tmem_ld32(tmem + lane_base + L::TM_G + wh * 64 + part, v);
 #pragma unroll
                 for (int s8 = 0; s8 < 32; s8 += 8) {
-                    const uint32_t off = swz_off(t, (part + s8) * 2, 128);
-                    if (r < 64) {
-                        *reinterpret_cast<uint4 *>(sm + L::KH + wh * 8192 + off) = pack8(v + s8);
-                    } else {
-                        uint4 *qp = reinterpret_cast<uint4 *>(sm + L::EQ + wh * 16384 + 8192 + off);
+                    const int j = wh * 64 + part + s8;
+                    const float4 e0 = *reinterpret_cast<const float4 *>(er + j);
+                    const float4 e1 = *reinterpret_cast<const float4 *>(er + j + 4);
+                    float f[8] = {-v[s8] * e0.x,     -v[s8 + 1] * e0.y, -v[s8 + 2] * e0.z, -v[s8 + 3] * e0.w,
+                                  -v[s8 + 4] * e1.x, -v[s8 + 5] * e1.y, -v[s8 + 6] * e1.z, -v[s8 + 7] * e1.w};
+                    *reinterpret_cast<uint4 *>(sm + L::LA + wh * 16384 + swz_off(i, (part + s8) * 2, 128)) = pack8(f);
+                }
+            }
+        }
+        {   // QS = (Qhat - PT Ehat) Diag(e^{Gamma_r}), in place over Qhat (M = 64 accumulator)
+            const int t = wq * 16 + lane;
+#pragma unroll
+            for (int part = 0; part < 64; part += 32) {
+                float v[32];
+                tmem_ld32(tmem + lane_base + L::TM_PW + wh * 64 + part, v);
+                if (lane < 16) {
+#pragma unroll
+                    for (int s8 = 0; s8 < 32; s8 += 8) {
+                        const int j = wh * 64 + part + s8;
+                        uint4 *qp = reinterpret_cast<uint4 *>(sm + L::EQ + wh * 16384 + 8192 +
+                                                              swz_off(t, (part + s8) * 2, 128));
                         float qh[8], f[8];
                         unpack8(*qp, qh);
+                        const float4 e0 = *reinterpret_cast<const float4 *>(er + j);
+                        const float4 e1 = *reinterpret_cast<const float4 *>(er + j + 4);
+                        const float ev[8] = {e0.x, e0.y, e0.z, e0.w, e1.x, e1.y, e1.z, e1.w};
 #pragma unroll
-                        for (int u = 0; u < 8; ++u) f[u] = qh[u] - v[s8 + u];
+                        for (int u = 0; u < 8; ++u) f[u] = (qh[u] - v[s8 + u]) * ev[u];
                         *qp = pack8(f);
                     }
                 }
             }
-            // U0 rows -> U0 operand (ZO); PU0 rows -> PU0 (TO, the record's block layout)
-            constexpr int HALF = DV / 2;
-#pragma unroll
-            for (int part = 0; part < HALF; part += 32) {
-                float v[32];
-                tmem_ld32(tmem + lane_base + L::TM_U + wh * HALF + part, v);
-#pragma unroll
-                for (int s8 = 0; s8 < 32; s8 += 8) {
-                    const int col = wh * HALF + part + s8;
-                    const uint32_t off = (col >> 6) * 8192 + swz_off(t, (col & 63) * 2, 128);
-                    *reinterpret_cast<uint4 *>(sm + (r < 64 ? L::ZO : L::TO) + off) = pack8(v + s8);
-                }
-            }
-        }
-        tc_fence_before();
-        fence_proxy_async_smem();
-        __syncthreads();
-
-        // ---------------------------------------------------------- G = Ktil^T W,  N = Ktil^T U0
-        if (tid == 0) {
-            tc_fence_after();
-            bulk_store(rec + R::QP, sm + L::EQ + 8192, 8192);          // Q' (two 8 KB blocks)
-            bulk_store(rec + R::QP + 8192, sm + L::EQ + 24576, 8192);
-            bulk_store(rec + R::PU, sm + L::TO, 64 * DV * 2);          // PU0
-            bulk_commit();
-            const uint32_t idg = idesc_bf16(128, kDK, 1, 1), idn = idesc_bf16(128, DV, 1, 1);
-#pragma unroll
-            for (int ks = 0; ks < 4; ++ks) {
-                const uint64_t ad = smem_desc(sbase + L::KT + ks * 2048, 8192, 1024, kSw128);
-                umma_bf16(tmem + L::TM_W, ad, smem_desc(sbase + L::KH + ks * 2048, 8192, 1024, kSw128), idg, ks > 0);
-                umma_bf16(tmem + L::TM_U, ad, smem_desc(sbase + L::ZO + ks * 2048, 8192, 1024, kSw128), idn, ks > 0);
-            }
-            umma_commit(bar_mma);
-        }
-        bool mine = true;
-        if (tid == 0) {
-            mine = mbar_wait(bar_mma, mma_phase, err);
-            bulk_wait_read_all();  // PU0 has left TO before N is staged there
-        }
-        mma_phase ^= 1;
-        ok = __syncthreads_and(mine) != 0;
-        tc_fence_after();
-    }
-
-    if (ok) {
-        {   // G rows -> KH (block 0) / KT (block 1);  N rows -> ZO (block 0) / TO (block 1)
-            const int i = wq * 32 + lane;  // key channel
-#pragma unroll
-            for (int part = 0; part < 64; part += 32) {
-                float v[32];
-                tmem_ld32(tmem + lane_base + L::TM_W + wh * 64 + part, v);
-#pragma unroll
-                for (int s8 = 0; s8 < 32; s8 += 8)
-                    *reinterpret_cast<uint4 *>(sm + (wh ? L::KT : L::KH) + swz_off(i, (part + s8) * 2, 128)) =
-                        pack8(v + s8);
-            }
-            constexpr int HALF = DV / 2;
-#pragma unroll
-            for (int part = 0; part < HALF; part += 32) {
-                float v[32];
-                tmem_ld32(tmem + lane_base + L::TM_U + wh * HALF + part, v);
-#pragma unroll
-                for (int s8 = 0; s8 < 32; s8 += 8) {
-                    const int col = wh * HALF + part + s8;
-                    *reinterpret_cast<uint4 *>(sm + ((col >> 6) ? L::TO : L::ZO) + swz_off(i, (col & 63) * 2, 128)) =
-                        pack8(v + s8);
-                }
-            }
         }
         fence_proxy_async_smem();
         __syncthreads();
         if (tid == 0) {
-            bulk_store(rec + R::GC, sm + L::KH, 16384);
-            bulk_store(rec + R::GC + 16384, sm + L::KT, 16384);
-            bulk_store(rec + R::NC, sm + L::ZO, 16384);
-            if (DV > 64) bulk_store(rec + R::NC + 16384, sm + L::TO, 16384);
-            bulk_store(rec + R::DEC, sm + L::DEC, 1024);
+            bulk_store(rec + R::NG, sm + L::LA, 32768);
+            bulk_store(rec + R::QS, sm + L::EQ + 8192, 8192);
+            bulk_store(rec + R::QS + 8192, sm + L::EQ + 24576, 8192);
+            bulk_store(rec + R::DEC, sm + L::DEC, 512);
             bulk_commit();
-            bulk_wait_read_all();
         }
     }
+    if (tid == 0) bulk_wait_read_all();
     tc_fence_before();
     __syncthreads();
     if (warp == 0) {

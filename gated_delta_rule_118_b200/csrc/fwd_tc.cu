@@ -80,17 +80,17 @@ FwdTcPlan plan_fwd_tc(int B, int T, int H, int dv, size_t window_budget)
     p.dvt = (dv == 64 || bh * 2 <= 148) ? 64 : 128;
     p.nchunks = (T + kChunk - 1) / kChunk;
     p.rec_bytes = (dv == 128) ? Record<128>::BYTES : Record<64>::BYTES;
-    p.sref_bytes = (dv == 128) ? SrefSlot<128>::BYTES : SrefSlot<64>::BYTES;
-    const size_t per_chunk = (size_t)bh * (p.rec_bytes + p.sref_bytes);
+    p.sx_bytes = (dv == 128) ? SxSlot<128>::BYTES : SxSlot<64>::BYTES;
+    const size_t per_chunk = (size_t)bh * (p.rec_bytes + p.sx_bytes);
     long wc = per_chunk ? (long)(window_budget / per_chunk) : 0;
     if (wc < 1) wc = 1;
     if (wc > p.nchunks) wc = p.nchunks;
     p.wc = (int)wc;
     p.nwindows = p.nchunks ? (p.nchunks + p.wc - 1) / p.wc : 0;
     p.rec_total = (size_t)p.wc * bh * p.rec_bytes;
-    p.sref_total = (size_t)p.wc * bh * p.sref_bytes;
+    p.sx_total = (size_t)p.wc * bh * p.sx_bytes;
     p.carry_bytes = p.nwindows > 1 ? (size_t)bh * 128 * dv * sizeof(float) : 0;
-    p.ws_bytes = p.rec_total + p.sref_total + p.carry_bytes;
+    p.ws_bytes = p.rec_total + p.sx_total + p.carry_bytes;
     return p;
 }
 
@@ -106,16 +106,16 @@ cudaError_t run_fwd_tc(const FwdArgs &a, const FwdTcPlan &p, uint8_t *ws)
         !make_map(&maps[4], a.v, BF, 2, a.dv, a.H, a.T, a.B, a.dv, CU_TENSOR_MAP_SWIZZLE_NONE) ||
         !make_map(&maps[5], a.w, BF, 2, a.dv, a.H, a.T, a.B, a.dv, CU_TENSOR_MAP_SWIZZLE_NONE))
         return cudaErrorInvalidValue;
-    uint8_t *recs = ws, *srefs = ws + p.rec_total;
-    float *carry = p.carry_bytes ? reinterpret_cast<float *>(ws + p.rec_total + p.sref_total) : nullptr;
+    uint8_t *recs = ws, *sxs = ws + p.rec_total;
+    float *carry = p.carry_bytes ? reinterpret_cast<float *>(ws + p.rec_total + p.sx_total) : nullptr;
     for (int w = 0; w < p.nwindows; ++w) {
         const int c0 = w * p.wc;
         const int ncw = (p.nchunks - c0 < p.wc) ? p.nchunks - c0 : p.wc;
         const float *S_in = (w == 0) ? a.S0 : carry;
         float *S_out = (w == p.nwindows - 1) ? a.S_T : carry;
         cudaError_t e = launch_prep(a, maps, recs, c0, ncw, p.wc);
-        if (e == cudaSuccess) e = launch_chain(a, p.dvt, recs, srefs, S_in, S_out, ncw, p.wc);
-        if (e == cudaSuccess) e = launch_out(a, recs, srefs, c0, ncw, p.wc);
+        if (e == cudaSuccess) e = launch_chain(a, p.dvt, recs, sxs, S_in, S_out, ncw, p.wc);
+        if (e == cudaSuccess) e = launch_out(a, recs, sxs, c0, ncw, p.wc);
         if (e != cudaSuccess) return e;
     }
     return cudaSuccess;
@@ -175,7 +175,7 @@ cudaError_t run_fwd_tc_overlapped(const FwdArgs &a, const FwdTcPlan &p, uint8_t 
         !make_map(&maps[4], a.v, BF, 2, a.dv, a.H, a.T, a.B, a.dv, CU_TENSOR_MAP_SWIZZLE_NONE) ||
         !make_map(&maps[5], a.w, BF, 2, a.dv, a.H, a.T, a.B, a.dv, CU_TENSOR_MAP_SWIZZLE_NONE))
         return cudaErrorInvalidValue;
-    const size_t half = p.rec_total + p.sref_total;
+    const size_t half = p.rec_total + p.sx_total;
     float *carry = p.carry_bytes ? reinterpret_cast<float *>(ws + 2 * half) : nullptr;
     cudaError_t e = cudaEventRecord(ss.start, a.stream);
     if (e == cudaSuccess) e = cudaStreamWaitEvent(ss.prep, ss.start, 0);
@@ -184,7 +184,7 @@ cudaError_t run_fwd_tc_overlapped(const FwdArgs &a, const FwdTcPlan &p, uint8_t 
     for (int w = 0; w < p.nwindows && e == cudaSuccess; ++w) {
         const int c0 = w * p.wc, slot = w & 3;
         const int ncw = (p.nchunks - c0 < p.wc) ? p.nchunks - c0 : p.wc;
-        uint8_t *recs = ws + (w & 1) * half, *srefs = recs + p.rec_total;
+        uint8_t *recs = ws + (w & 1) * half, *sxs = recs + p.rec_total;
         const float *S_in = (w == 0) ? a.S0 : carry;
         float *S_out = (w == p.nwindows - 1) ? a.S_T : carry;
         FwdArgs ap = a, ac = a, ao = a;
@@ -198,10 +198,10 @@ cudaError_t run_fwd_tc_overlapped(const FwdArgs &a, const FwdTcPlan &p, uint8_t 
         if (e == cudaSuccess) e = launch_prep(ap, maps, recs, c0, ncw, p.wc);
         if (e == cudaSuccess) e = cudaEventRecord(ss.ev_p[slot], ss.prep);
         if (e == cudaSuccess) e = cudaStreamWaitEvent(ss.chain, ss.ev_p[slot], 0);
-        if (e == cudaSuccess) e = launch_chain(ac, p.dvt, recs, srefs, S_in, S_out, ncw, p.wc);
+        if (e == cudaSuccess) e = launch_chain(ac, p.dvt, recs, sxs, S_in, S_out, ncw, p.wc);
         if (e == cudaSuccess) e = cudaEventRecord(ss.ev_c[slot], ss.chain);
         if (e == cudaSuccess) e = cudaStreamWaitEvent(ss.out, ss.ev_c[slot], 0);
-        if (e == cudaSuccess) e = launch_out(ao, recs, srefs, c0, ncw, p.wc);
+        if (e == cudaSuccess) e = launch_out(ao, recs, sxs, c0, ncw, p.wc);
         if (e == cudaSuccess) e = cudaEventRecord(ss.ev_o[slot], ss.out);
     }
     // join: the caller's stream waits for the last chain and the last two outputs
@@ -226,7 +226,7 @@ cudaError_t launch_fwd_tc(const FwdArgs &a)
     if (!pool || !ss) return cudaErrorMemoryAllocation;
     // two window halves of half the budget each
     FwdTcPlan p = plan_fwd_tc(a.B, a.T, a.H, a.dv, kWindowBudgetBytes / 2);
-    const size_t bytes = 2 * (p.rec_total + p.sref_total) + p.carry_bytes;
+    const size_t bytes = 2 * (p.rec_total + p.sx_total) + p.carry_bytes;
     void *ws = nullptr;
     e = cudaMallocFromPoolAsync(&ws, bytes, pool, a.stream);
     if (e != cudaSuccess) return e;

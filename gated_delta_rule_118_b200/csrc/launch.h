@@ -37,16 +37,16 @@ cudaError_t launch_decode(const DecodeArgs &a);
 cudaError_t launch_fwd_simt(const FwdArgs &a);
 
 // bf16 tensor-core forward, per window of WC chunks:
-//   prep (per chunk) -> records -> chain (sequential, exports Sref) -> output (per chunk)
+//   prep (per chunk) -> records -> chain (sequential, exports the state image Sx) -> output (per chunk)
 struct FwdTcPlan {
     int dvt;            // value-tile width of a chain CTA
     int nchunks;        // chunks in the sequence
     int wc;             // chunks per window
     int nwindows;
     size_t rec_bytes;   // bytes of one prep record
-    size_t sref_bytes;  // bytes of one exported Sref
+    size_t sx_bytes;  // bytes of one exported state image
     size_t rec_total;   // records of one window
-    size_t sref_total;  // Sref slots of one window
+    size_t sx_total;  // state images of one window
     size_t carry_bytes; // state carried between windows
     size_t ws_bytes;    // total workspace
 };
@@ -55,8 +55,8 @@ FwdTcPlan plan_fwd_tc(int B, int T, int H, int dv, size_t window_budget);
 cudaError_t run_fwd_tc(const FwdArgs &a, const FwdTcPlan &p, uint8_t *ws);
 cudaError_t launch_fwd_tc(const FwdArgs &a);
 cudaError_t launch_prep(const FwdArgs &a, const CUtensorMap *maps, uint8_t *ws, int c0, int ncw, int WC);
-cudaError_t launch_chain(const FwdArgs &a, int dvt, const uint8_t *ws, uint8_t *sref, const float *S_in,
+cudaError_t launch_chain(const FwdArgs &a, int dvt, const uint8_t *ws, uint8_t *sx, const float *S_in,
                          float *S_out, int ncw, int WC);
-cudaError_t launch_out(const FwdArgs &a, const uint8_t *ws, const uint8_t *sref, int c0, int ncw, int WC);
+cudaError_t launch_out(const FwdArgs &a, const uint8_t *ws, const uint8_t *sx, int c0, int ncw, int WC);
 
 }  // namespace gdn2

@@ -1,7 +1,7 @@
 // tc_common.cuh -- helpers shared by the tensor-core forward kernels: bf16
-// packing, the shared-memory plan of one prep record, and the record layout in
-// the workspace that carries a chunk's state-independent quantities from the
-// prep kernel to the chain kernel.
+// packing, warp-level tf32 MMAs, and the layout of the workspace records that
+// carry a chunk's state-independent quantities from the prep kernel to the
+// chain and output kernels.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -18,31 +18,34 @@ constexpr float kLog2e = 1.4426950408889634f;
 
 __host__ __device__ constexpr int align_up(int x, int a) { return (x + a - 1) / a * a; }
 
-// One prep record per (batch, head, chunk), consumed by the chain and output kernels.
-//   GC  [128 rows = key channel][128 K = key channel] bf16, K-major, 128-byte
-//       swizzle, two 64-column blocks of 16 KB: G = Ktil^T T Ehat (the part of
-//       the chunk transition that the erase projection removes)
-//   QP  [64 rows = token][128 K] bf16, K-major, swizzled, blocks of 8 KB:
-//       Q' = Qhat - P T Ehat
-//   PU  [dv/64 blocks][64 tokens][64] bf16, rows swizzled: P T Z (the output's
-//       state-independent part)
-//   NC  [dv/64 blocks][128 key channels][64] bf16, rows swizzled: Ktil^T T Z
-//   DEC [2][128] fp32: e^{Gamma_C}, e^{Gamma_r} per key channel
+// One prep record per (batch, head, chunk), read by the chain and output kernels.
+// With Ebar = e^{Gamma} b k the erase keys decayed from the chunk start, the
+// chunk maps the incoming state S to
+//   S_next = Diag(e^{Gamma_C}) S + NG S + Y Z       NG = -Ktil^T T Ebar
+//   O      = QS S + PT Z                            QS = (Qhat - P T Ehat) Diag(e^{Gamma_r})
+// The parts, bf16 UMMA operands with the 128-byte swizzle:
+//   NG  [128 rows = key channel i][128 K = key channel j], K-major, two 16 KB blocks
+//   QS  [64 rows = token][128 K = key channel], K-major, two 8 KB blocks
+//   Y   [128 rows = key channel][64 K = token], K-major, 16 KB:  Y = Ktil^T T
+//   PT  [64 rows = token][64 K = token], K-major, 8 KB:          P T
+//   Z   [64 rows = token (K)][DV = value (N)], MN-major, DV/64 blocks of 8 KB: Z = w v
+//   DEC [128] fp32: e^{Gamma_C} per key channel
 template <int DV>
 struct Record {
-    static constexpr int GC = 0;
-    static constexpr int QP = GC + 32768;
-    static constexpr int PU = QP + 16384;
-    static constexpr int NC = PU + 64 * DV * 2;
-    static constexpr int DEC = NC + 128 * DV * 2;
+    static constexpr int NG = 0;
+    static constexpr int QS = 32768;
+    static constexpr int Y = 49152;
+    static constexpr int PT = 65536;
+    static constexpr int Z = 73728;
+    static constexpr int DEC = Z + 64 * DV * 2;
     static constexpr int BYTES = DEC + 1024;
 };
 
-// The chain kernel exports Sref = e^{Gamma_r} S of every chunk for the output
-// kernel: [128 key channels][DV] bf16 as dv/64 blocks of [128 rows][128 B],
-// 128-byte swizzle, i.e. the MN-major operand layout of the output UMMA.
+// The chain kernel exports the bf16 image Sx of the state entering every chunk
+// for the output kernel: [128 key channels][DV] as DV/64 blocks of [128 rows][128 B],
+// 128-byte swizzle, i.e. the MN-major B operand layout of the UMMA.
 template <int DV>
-struct SrefSlot {
+struct SxSlot {
     static constexpr int BYTES = 128 * DV * 2;
 };
 

@@ -14,19 +14,22 @@ reference point r inside the chunk (its midpoint):
     Khat_s = exp(Gamma_r - Gamma_s) (*) k_s
     Ktil_s = exp(Gamma_C - Gamma_s) (*) k_s
     A = strictly-lower(Ehat Khat^T),   P = lower-inclusive(Qhat Khat^T)
-    Sref = Diag(exp(Gamma_r)) S_0
-    U = (I + A)^{-1} (Z - Ehat Sref)                  (Z = w (*) v)
-    O = Qhat Sref + P U
-    S_C = Diag(exp(Gamma_C)) S_0 + Ktil^T U
-The decay is absorbed into asymmetric erase/key factors and the lower
-triangular system (I + T)^{-1} is solved per chunk, as the gist.science summary
-describes in section 3 ("Efficient chunkwise parallel training").
+    T = (I + A)^{-1},   Y = Ktil^T T,   PT = P T
+    NG = -Y Ehat Diag(exp(Gamma_r)),   QS = (Qhat - PT Ehat) Diag(exp(Gamma_r))
+and, with Z = w (*) v, the chunk maps the incoming state S to
+    S_C = Diag(exp(Gamma_C)) S + NG S + Y Z,      O = QS S + PT Z.
+(Equivalently U = T (Z - Ehat Diag(exp(Gamma_r)) S), O = Qhat Diag(exp(Gamma_r)) S
++ P U, S_C = Diag(exp(Gamma_C)) S + Ktil^T U.)  The decay is absorbed into
+asymmetric erase/key factors and the lower triangular system (I + T)^{-1} is
+solved per chunk, as the gist.science summary describes in section 3
+("Efficient chunkwise parallel training").  Only Z depends on the values, so
+every other part of the chunk's record is computed once for all value columns.
 """
 import numpy as np
 
 
-def chunk_step(q, k, v, b, w, la, S, C):
-    """One chunk of L <= C tokens for one (batch, head): returns (O, S_C)."""
+def chunk_record(q, k, b, la, C):
+    """State-independent part of one chunk of L <= C tokens: (gc, NG, QS, Y, PT)."""
     L = q.shape[0]
     G = np.cumsum(la, axis=0)                       # Gamma_1..Gamma_L
     r = min(C // 2, L)
@@ -36,13 +39,23 @@ def chunk_step(q, k, v, b, w, la, S, C):
     Qh = up * q
     Kh = np.exp(Gr - G) * k
     Kt = np.exp(G[-1] - G) * k
-    Z = w * v
     A = np.tril(Eh @ Kh.T, -1)
     P = np.tril(Qh @ Kh.T, 0)
-    Sref = np.exp(Gr)[:, None] * S
-    U = np.linalg.solve(np.eye(L) + A, Z - Eh @ Sref)
-    O = Qh @ Sref + P @ U
-    S_new = np.exp(G[-1])[:, None] * S + Kt.T @ U
+    T = np.linalg.inv(np.eye(L) + A)
+    Y = Kt.T @ T
+    PT = P @ T
+    er = np.exp(Gr)
+    NG = -(Y @ Eh) * er[None, :]
+    QS = (Qh - PT @ Eh) * er[None, :]
+    return np.exp(G[-1]), NG, QS, Y, PT
+
+
+def chunk_step(q, k, v, b, w, la, S, C):
+    """One chunk of L <= C tokens for one (batch, head): returns (O, S_C)."""
+    gc, NG, QS, Y, PT = chunk_record(q, k, b, la, C)
+    Z = w * v
+    O = QS @ S + PT @ Z
+    S_new = gc[:, None] * S + NG @ S + Y @ Z
     return O, S_new
 
 
