@@ -21,10 +21,10 @@ constexpr int kOutThreads = 128;
 
 template <int DV>
 struct OutLayout {
-    static constexpr int QS = 0;                    // QS [64][128] K-major, 2 blocks of 8 KB
-    static constexpr int PT = 16384;                // PT [64][64] K-major, 8 KB
+    static constexpr int QS = 0;                    // QS [64][128] K-major, no swizzle
+    static constexpr int PT = 16384;                // PT [64][64] K-major, no swizzle
     static constexpr int Z = 24576;                 // Z, DV/64 blocks of [64][64] (MN-major)
-    static constexpr int SX = Z + 64 * DV * 2;      // Sx, DV/64 blocks of [128][64] (MN-major)
+    static constexpr int SX = Z + 64 * DV * 2;      // Sx [128][DV] (MN-major, no swizzle)
     static constexpr int TX = SX + 128 * DV * 2;
     static constexpr int BAR = TX;
     static constexpr int SLOT = BAR + 16;
@@ -63,6 +63,8 @@ out_kernel(const uint8_t *__restrict__ ws, const uint8_t *__restrict__ sx, bf16 
         tmem_alloc(slot, DV);
         tmem_relinquish();
     }
+    // windows write disjoint outputs: the next window's output kernel may start early
+    allow_dependent_launch();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -73,12 +75,12 @@ out_kernel(const uint8_t *__restrict__ ws, const uint8_t *__restrict__ sx, bf16 
         const uint32_t id = idesc_bf16(64, DV, 0, 1);
 #pragma unroll
         for (int ks = 0; ks < 4; ++ks)
-            umma_bf16(tmem, smem_desc(sbase + L::PT + ks * 32, 16, 1024, kSw128),
+            umma_bf16(tmem, smem_desc(sbase + L::PT + ks * 2048, 1024, 128, kSwNone),
                       smem_desc(sbase + L::Z + ks * 2048, 8192, 1024, kSw128), id, ks > 0);
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks)
-            umma_bf16(tmem, smem_desc(sbase + L::QS + (ks >> 2) * 8192 + (ks & 3) * 32, 16, 1024, kSw128),
-                      smem_desc(sbase + L::SX + ks * 2048, 16384, 1024, kSw128), id, 1);
+            umma_bf16(tmem, smem_desc(sbase + L::QS + ks * 2048, 1024, 128, kSwNone),
+                      smem_desc(sbase + L::SX + ks * 256, 128, 2048, kSwNone), id, 1);
         umma_commit(bar + 1);
         ok = mbar_wait(bar + 1, 0, err);
     }
@@ -114,22 +116,23 @@ out_kernel(const uint8_t *__restrict__ ws, const uint8_t *__restrict__ sx, bf16 
 }
 
 template <int DV>
-cudaError_t launch_out_impl(const FwdArgs &a, const uint8_t *ws, const uint8_t *sx, int c0, int ncw, int WC)
+cudaError_t launch_out_impl(const FwdArgs &a, const uint8_t *ws, const uint8_t *sx, int c0, int ncw, int WC,
+                            bool overlap)
 {
     using L = OutLayout<DV>;
     auto kern = out_kernel<DV>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::BYTES);
     if (e != cudaSuccess) return e;
-    dim3 grid(ncw, a.H, a.B);
-    kern<<<grid, kOutThreads, L::BYTES, a.stream>>>(ws, sx, (bf16 *)a.o, a.T, a.H, c0, WC, a.err);
-    return cudaGetLastError();
+    LaunchCfg lc(dim3(ncw, a.H, a.B), dim3(kOutThreads), L::BYTES, a.stream, overlap);
+    return cudaLaunchKernelEx(&lc.cfg, kern, ws, sx, (bf16 *)a.o, a.T, a.H, c0, WC, a.err);
 }
 
 }  // namespace
 
-cudaError_t launch_out(const FwdArgs &a, const uint8_t *ws, const uint8_t *sx, int c0, int ncw, int WC)
+cudaError_t launch_out(const FwdArgs &a, const uint8_t *ws, const uint8_t *sx, int c0, int ncw, int WC, bool overlap)
 {
-    return a.dv == 128 ? launch_out_impl<128>(a, ws, sx, c0, ncw, WC) : launch_out_impl<64>(a, ws, sx, c0, ncw, WC);
+    return a.dv == 128 ? launch_out_impl<128>(a, ws, sx, c0, ncw, WC, overlap)
+                       : launch_out_impl<64>(a, ws, sx, c0, ncw, WC, overlap);
 }
 
 }  // namespace gdn2

@@ -8,9 +8,10 @@
 // system (I + T)^{-1} is solved per chunk).  With Gamma the chunk-local
 // cumulative log-decay (fp32) and r the chunk midpoint:
 //   Ehat = e^{Gamma-Gamma_r} b k    Qhat = e^{Gamma-Gamma_r} q
-//   Khat = e^{Gamma_r-Gamma} k      Ktil = e^{Gamma_C-Gamma} k    Z = w v
+//   Khat = e^{Gamma_r-Gamma} k      Z = w v
 //   A = strict_lower(Ehat Khat^T)   P = lower(Qhat Khat^T)   T = (I + A)^{-1}
-//   Y = Ktil^T T    PT = P T    G = Y Ehat    Q' = Qhat - PT Ehat
+//   Y = e^{Gamma_C-Gamma_r} Khat^T T  (= Ktil^T T with Ktil = e^{Gamma_C-Gamma} k)
+//   PT = P T    G = Y Ehat    Q' = Qhat - PT Ehat
 // and the record keeps NG = -G Diag(e^{Gamma_r}), QS = Q' Diag(e^{Gamma_r}),
 // Y, PT, Z and e^{Gamma_C}, so that for the incoming state S
 //   S_next = e^{Gamma_C} S + NG S + Y Z        O = QS S + PT Z.
@@ -25,7 +26,8 @@
 // round trips in all (Gram; Y and PT; G and P T Ehat); the solve is fp32
 // (16x16 diagonal blocks by substitution on CUDA cores, then two levels of
 // block merging whose small products run as warp-level tf32 MMAs).  Record
-// pieces leave through bulk copies as soon as they are final.
+// pieces go straight from the tensor-memory readouts to the record, each warp
+// store covering 512 contiguous bytes.
 #include <cuda.h>
 
 #include "launch.h"
@@ -40,12 +42,12 @@ constexpr int kPrepThreads = 256;
 constexpr int kDK = 128;
 
 struct PrepLayout {
-    static constexpr int EQ = 0;          // [Ehat;Qhat]: b, q arrive here; QS over Qhat at the end
-    static constexpr int KH = 32768;      // Khat -> solve scratch -> Y
-    static constexpr int KT = 49152;      // k arrives here -> Ktil -> PT
-    static constexpr int LA = 65536;      // log_alpha -> fp32 A | fp32 T -> bf16 T over A -> NG
+    static constexpr int EQ = 0;          // [Ehat;Qhat]: b, q arrive here
+    static constexpr int KH = 32768;      // solve scratch -> Y (no swizzle)
+    static constexpr int KT = 49152;      // k arrives here -> Khat -> PT (no swizzle)
+    static constexpr int LA = 65536;      // log_alpha -> fp32 A | fp32 T -> bf16 T over A
     static constexpr int PO = 98304;      // Gamma quarter totals -> P
-    static constexpr int DEC = 106496;    // e^{Gamma_C}[128], e^{Gamma_r}[128]
+    static constexpr int DEC = 106496;    // e^{Gamma_C-Gamma_r}[128], e^{Gamma_r}[128]
     static constexpr int BAR = 107520;
     static constexpr int SLOT = BAR + 16;
     static constexpr int BYTES = SLOT + 16 + 1024;
@@ -56,14 +58,10 @@ struct PrepLayout {
 };
 static_assert(PrepLayout::BYTES * 2 + 2048 <= 233472, "two CTAs per SM");
 
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&r)[32])
+__device__ __forceinline__ void tmem_ld32_wait(uint32_t taddr, float (&r)[32])
 {
-    float a[16], b[16];
-    tmem_ld16(taddr, a);
-    tmem_ld16(taddr + 16, b);
+    tmem_ld32(taddr, r);
     tmem_ld_wait();
-#pragma unroll
-    for (int u = 0; u < 16; ++u) { r[u] = a[u]; r[16 + u] = b[u]; }
 }
 
 template <int DV>
@@ -111,6 +109,8 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         tmem_alloc(slot, L::TMEM_COLS);
         tmem_relinquish();
     }
+    // chunks are independent: the next window's prep may start filling SMs
+    allow_dependent_launch();
     // v and w for Z = w v: plain vector loads, issued before anything waits
     // (tokens past the sequence end give zero rows of Z)
     constexpr int ZV = 64 * DV / 8 / kPrepThreads;  // 16-byte vectors per thread
@@ -171,13 +171,14 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         // midpoint reference: Gamma after 32 tokens (tokens past T carry log_alpha = 0)
         const float gr0 = tot[2 * p] + tot[kDK + 2 * p], gr1 = tot[2 * p + 1] + tot[kDK + 2 * p + 1];
         if (qr == 0) {
-            dec[2 * p] = expf(gc0);
-            dec[2 * p + 1] = expf(gc1);
+            const float e0 = expf(gc0), e1 = expf(gc1);
+            dec[2 * p] = expf(gc0 - gr0);
+            dec[2 * p + 1] = expf(gc1 - gr1);
             dec[kDK + 2 * p] = expf(gr0);
             dec[kDK + 2 * p + 1] = expf(gr1);
+            *reinterpret_cast<float2 *>(rec + R::DEC + 8 * p) = make_float2(e0, e1);
         }
-        const float ecr0 = ex2_approx((gc0 - gr0) * kLog2e), ecr1 = ex2_approx((gc1 - gr1) * kLog2e);
-        uint8_t *eq = sm + L::EQ + kb * 16384, *kh = sm + L::KH + kb * 8192, *kt = sm + L::KT + kb * 8192;
+        uint8_t *eq = sm + L::EQ + kb * 16384, *kt = sm + L::KT + kb * 8192;
         unsigned int bad = 0;
         const float sh0 = pre0 - gr0, sh1 = pre1 - gr1;
 #pragma unroll
@@ -191,8 +192,7 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
             const float2 kv = ld_bf16x2(kt + off), bv = ld_bf16x2(eq + off), qv = ld_bf16x2(eq + 8192 + off);
             st_bf16x2(eq + off, up0 * bv.x * kv.x, up1 * bv.y * kv.y);
             st_bf16x2(eq + 8192 + off, up0 * qv.x, up1 * qv.y);
-            st_bf16x2(kh + off, dn0 * kv.x, dn1 * kv.y);
-            st_bf16x2(kt + off, ecr0 * dn0 * kv.x, ecr1 * dn1 * kv.y);
+            st_bf16x2(kt + off, dn0 * kv.x, dn1 * kv.y);
         }
         if (bad) atomicOr(err, kErrRange);
         fence_proxy_async_smem();
@@ -206,7 +206,7 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
             for (int ks = 0; ks < kDK / 16; ++ks) {
                 const uint32_t kofs = (ks & 3) * 32;
                 umma_bf16(tmem + L::TM_G, smem_desc(sbase + L::EQ + (ks >> 2) * 16384 + kofs, 16, 1024, kSw128),
-                          smem_desc(sbase + L::KH + (ks >> 2) * 8192 + kofs, 16, 1024, kSw128), id, ks > 0);
+                          smem_desc(sbase + L::KT + (ks >> 2) * 8192 + kofs, 16, 1024, kSw128), id, ks > 0);
             }
             umma_commit(bar_mma);
         }
@@ -231,7 +231,7 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         {
             const int r = wq * 32 + lane;
             float v[32];
-            tmem_ld32(tmem + lane_base + L::TM_GRAM + wh * 32, v);
+            tmem_ld32_wait(tmem + lane_base + L::TM_GRAM + wh * 32, v);
             if (r < 64) {
                 const int t = r;
 #pragma unroll
@@ -377,7 +377,7 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         fence_proxy_async_smem();
         __syncthreads();
 
-        // ---------------------------------------------------------- Y = Ktil^T T (M = 128),  PT = P T (M = 64)
+        // ---------------------------------------------------------- Khat^T T (M = 128),  PT = P T (M = 64)
         if (tid == 0) {
             tc_fence_after();
             const uint32_t idy = idesc_bf16(128, 64, 1, 1), idp = idesc_bf16(64, 64, 0, 1);
@@ -393,26 +393,27 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     }
 
     if (ok) {
-        {   // Y row i -> KH ([128][64] K-major);  PT (M = 64: row 16*wq + l in TMEM lane 32*wq + l) -> KT
-            float v0[16], v1[16], p0[16], p1[16];
-            tmem_ld16(tmem + lane_base + L::TM_Y + wh * 32, v0);
-            tmem_ld16(tmem + lane_base + L::TM_Y + wh * 32 + 16, v1);
-            tmem_ld16(tmem + lane_base + L::TM_PT + wh * 32, p0);
-            tmem_ld16(tmem + lane_base + L::TM_PT + wh * 32 + 16, p1);
+        {   // Y row i, K chunks [4*wh, +4) -> KH and the record;  PT (M = 64: row 16*wq + l
+            // in TMEM lane 32*wq + l) -> KT and the record.  No-swizzle K-major tiles.
+            float v[32], p[32];
+            tmem_ld32(tmem + lane_base + L::TM_Y + wh * 32, v);
+            tmem_ld32(tmem + lane_base + L::TM_PT + wh * 32, p);
             tmem_ld_wait();
-            const int i = wq * 32 + lane;
-            uint8_t *yrow = sm + L::KH;
-            *reinterpret_cast<uint4 *>(yrow + swz_off(i, wh * 64, 128)) = pack8(v0);
-            *reinterpret_cast<uint4 *>(yrow + swz_off(i, wh * 64 + 16, 128)) = pack8(v0 + 8);
-            *reinterpret_cast<uint4 *>(yrow + swz_off(i, wh * 64 + 32, 128)) = pack8(v1);
-            *reinterpret_cast<uint4 *>(yrow + swz_off(i, wh * 64 + 48, 128)) = pack8(v1 + 8);
-            if (lane < 16) {
-                const int t = wq * 16 + lane;
-                uint8_t *prow = sm + L::KT;
-                *reinterpret_cast<uint4 *>(prow + swz_off(t, wh * 64, 128)) = pack8(p0);
-                *reinterpret_cast<uint4 *>(prow + swz_off(t, wh * 64 + 16, 128)) = pack8(p0 + 8);
-                *reinterpret_cast<uint4 *>(prow + swz_off(t, wh * 64 + 32, 128)) = pack8(p1);
-                *reinterpret_cast<uint4 *>(prow + swz_off(t, wh * 64 + 48, 128)) = pack8(p1 + 8);
+            const int i = wq * 32 + lane, t = wq * 16 + lane;
+            const float ecr = dec[i];
+#pragma unroll
+            for (int u = 0; u < 32; ++u) v[u] *= ecr;
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const int c = wh * 4 + q;
+                const uint4 y = pack8(v + 8 * q);
+                *reinterpret_cast<uint4 *>(sm + L::KH + kchunk_off(c, i, 128)) = y;
+                *reinterpret_cast<uint4 *>(rec + R::Y + kchunk_off(c, i, 128)) = y;
+                if (lane < 16) {
+                    const uint4 pt = pack8(p + 8 * q);
+                    *reinterpret_cast<uint4 *>(sm + L::KT + kchunk_off(c, t, 64)) = pt;
+                    *reinterpret_cast<uint4 *>(rec + R::PT + kchunk_off(c, t, 64)) = pt;
+                }
             }
         }
         tc_fence_before();
@@ -426,48 +427,44 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks) {
                 const uint64_t be = smem_desc(sbase + L::EQ + ks * 2048, 16384, 1024, kSw128);
-                umma_bf16(tmem + L::TM_G, smem_desc(sbase + L::KH + ks * 32, 16, 1024, kSw128), be, idg, ks > 0);
-                umma_bf16(tmem + L::TM_PW, smem_desc(sbase + L::KT + ks * 32, 16, 1024, kSw128), be, idw, ks > 0);
+                umma_bf16(tmem + L::TM_G, smem_desc(sbase + L::KH + ks * 4096, 2048, 128, kSwNone), be, idg, ks > 0);
+                umma_bf16(tmem + L::TM_PW, smem_desc(sbase + L::KT + ks * 2048, 1024, 128, kSwNone), be, idw, ks > 0);
             }
             umma_commit(bar_mma);
-            bulk_store(rec + R::Y, sm + L::KH, 16384);
-            bulk_store(rec + R::PT, sm + L::KT, 8192);
-            bulk_commit();
         }
         ok = mma_done();
     }
 
     if (ok) {
         const float *er = dec + kDK;
-        {   // NG = -G Diag(e^{Gamma_r}): row i, columns [64*wh, +64) -> block wh of NG (over A/T)
+        {   // NG = -G Diag(e^{Gamma_r}): row i, K chunks [8*wh, +8) -> the record
             const int i = wq * 32 + lane;
+            float v[64];
+            tmem_ld32(tmem + lane_base + L::TM_G + wh * 64, *reinterpret_cast<float(*)[32]>(v));
+            tmem_ld32(tmem + lane_base + L::TM_G + wh * 64 + 32, *reinterpret_cast<float(*)[32]>(v + 32));
+            tmem_ld_wait();
 #pragma unroll
-            for (int part = 0; part < 64; part += 32) {
-                float v[32];
-                tmem_ld32(tmem + lane_base + L::TM_G + wh * 64 + part, v);
-#pragma unroll
-                for (int s8 = 0; s8 < 32; s8 += 8) {
-                    const int j = wh * 64 + part + s8;
-                    const float4 e0 = *reinterpret_cast<const float4 *>(er + j);
-                    const float4 e1 = *reinterpret_cast<const float4 *>(er + j + 4);
-                    float f[8] = {-v[s8] * e0.x,     -v[s8 + 1] * e0.y, -v[s8 + 2] * e0.z, -v[s8 + 3] * e0.w,
-                                  -v[s8 + 4] * e1.x, -v[s8 + 5] * e1.y, -v[s8 + 6] * e1.z, -v[s8 + 7] * e1.w};
-                    *reinterpret_cast<uint4 *>(sm + L::LA + wh * 16384 + swz_off(i, (part + s8) * 2, 128)) = pack8(f);
-                }
+            for (int s8 = 0; s8 < 64; s8 += 8) {
+                const int j = wh * 64 + s8;
+                const float4 e0 = *reinterpret_cast<const float4 *>(er + j);
+                const float4 e1 = *reinterpret_cast<const float4 *>(er + j + 4);
+                float f[8] = {-v[s8] * e0.x,     -v[s8 + 1] * e0.y, -v[s8 + 2] * e0.z, -v[s8 + 3] * e0.w,
+                              -v[s8 + 4] * e1.x, -v[s8 + 5] * e1.y, -v[s8 + 6] * e1.z, -v[s8 + 7] * e1.w};
+                *reinterpret_cast<uint4 *>(rec + R::NG + kchunk_off(j >> 3, i, 128)) = pack8(f);
             }
         }
-        {   // QS = (Qhat - PT Ehat) Diag(e^{Gamma_r}), in place over Qhat (M = 64 accumulator)
+        {   // QS = (Qhat - PT Ehat) Diag(e^{Gamma_r}) -> the record (M = 64 accumulator)
             const int t = wq * 16 + lane;
 #pragma unroll
             for (int part = 0; part < 64; part += 32) {
                 float v[32];
-                tmem_ld32(tmem + lane_base + L::TM_PW + wh * 64 + part, v);
+                tmem_ld32_wait(tmem + lane_base + L::TM_PW + wh * 64 + part, v);
                 if (lane < 16) {
 #pragma unroll
                     for (int s8 = 0; s8 < 32; s8 += 8) {
                         const int j = wh * 64 + part + s8;
-                        uint4 *qp = reinterpret_cast<uint4 *>(sm + L::EQ + wh * 16384 + 8192 +
-                                                              swz_off(t, (part + s8) * 2, 128));
+                        const uint4 *qp = reinterpret_cast<const uint4 *>(sm + L::EQ + wh * 16384 + 8192 +
+                                                                          swz_off(t, (part + s8) * 2, 128));
                         float qh[8], f[8];
                         unpack8(*qp, qh);
                         const float4 e0 = *reinterpret_cast<const float4 *>(er + j);
@@ -475,22 +472,12 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                         const float ev[8] = {e0.x, e0.y, e0.z, e0.w, e1.x, e1.y, e1.z, e1.w};
 #pragma unroll
                         for (int u = 0; u < 8; ++u) f[u] = (qh[u] - v[s8 + u]) * ev[u];
-                        *qp = pack8(f);
+                        *reinterpret_cast<uint4 *>(rec + R::QS + kchunk_off(j >> 3, t, 64)) = pack8(f);
                     }
                 }
             }
         }
-        fence_proxy_async_smem();
-        __syncthreads();
-        if (tid == 0) {
-            bulk_store(rec + R::NG, sm + L::LA, 32768);
-            bulk_store(rec + R::QS, sm + L::EQ + 8192, 8192);
-            bulk_store(rec + R::QS + 8192, sm + L::EQ + 24576, 8192);
-            bulk_store(rec + R::DEC, sm + L::DEC, 512);
-            bulk_commit();
-        }
     }
-    if (tid == 0) bulk_wait_read_all();
     tc_fence_before();
     __syncthreads();
     if (warp == 0) {
@@ -502,21 +489,22 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
 }  // namespace
 
 template <int DV>
-cudaError_t launch_prep_impl(const FwdArgs &a, const CUtensorMap *maps, uint8_t *ws, int c0, int ncw, int WC)
+cudaError_t launch_prep_impl(const FwdArgs &a, const CUtensorMap *maps, uint8_t *ws, int c0, int ncw, int WC,
+                             bool overlap)
 {
     using L = PrepLayout;
     auto kern = prep_kernel<DV>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::BYTES);
     if (e != cudaSuccess) return e;
-    dim3 grid(ncw, a.H, a.B);
-    kern<<<grid, kPrepThreads, L::BYTES, a.stream>>>(maps[0], maps[1], maps[2], maps[3], (const bf16 *)a.v,
-                                                     (const bf16 *)a.w, ws, a.T, a.H, c0, WC, a.err);
-    return cudaGetLastError();
+    LaunchCfg lc(dim3(ncw, a.H, a.B), dim3(kPrepThreads), L::BYTES, a.stream, overlap);
+    return cudaLaunchKernelEx(&lc.cfg, kern, maps[0], maps[1], maps[2], maps[3], (const bf16 *)a.v,
+                              (const bf16 *)a.w, ws, a.T, a.H, c0, WC, a.err);
 }
 
-cudaError_t launch_prep(const FwdArgs &a, const CUtensorMap *maps, uint8_t *ws, int c0, int ncw, int WC)
+cudaError_t launch_prep(const FwdArgs &a, const CUtensorMap *maps, uint8_t *ws, int c0, int ncw, int WC, bool overlap)
 {
-    return a.dv == 128 ? launch_prep_impl<128>(a, maps, ws, c0, ncw, WC) : launch_prep_impl<64>(a, maps, ws, c0, ncw, WC);
+    return a.dv == 128 ? launch_prep_impl<128>(a, maps, ws, c0, ncw, WC, overlap)
+                       : launch_prep_impl<64>(a, maps, ws, c0, ncw, WC, overlap);
 }
 
 }  // namespace gdn2

@@ -113,9 +113,9 @@ cudaError_t run_fwd_tc(const FwdArgs &a, const FwdTcPlan &p, uint8_t *ws)
         const int ncw = (p.nchunks - c0 < p.wc) ? p.nchunks - c0 : p.wc;
         const float *S_in = (w == 0) ? a.S0 : carry;
         float *S_out = (w == p.nwindows - 1) ? a.S_T : carry;
-        cudaError_t e = launch_prep(a, maps, recs, c0, ncw, p.wc);
+        cudaError_t e = launch_prep(a, maps, recs, c0, ncw, p.wc, false);
         if (e == cudaSuccess) e = launch_chain(a, p.dvt, recs, sxs, S_in, S_out, ncw, p.wc);
-        if (e == cudaSuccess) e = launch_out(a, recs, sxs, c0, ncw, p.wc);
+        if (e == cudaSuccess) e = launch_out(a, recs, sxs, c0, ncw, p.wc, false);
         if (e != cudaSuccess) return e;
     }
     return cudaSuccess;
@@ -195,13 +195,15 @@ cudaError_t run_fwd_tc_overlapped(const FwdArgs &a, const FwdTcPlan &p, uint8_t 
             e = cudaStreamWaitEvent(ss.prep, ss.ev_c[(w - 2) & 3], 0);
             if (e == cudaSuccess) e = cudaStreamWaitEvent(ss.prep, ss.ev_o[(w - 2) & 3], 0);
         }
-        if (e == cudaSuccess) e = launch_prep(ap, maps, recs, c0, ncw, p.wc);
+        // prep and output launches of consecutive windows touch disjoint data, so
+        // each may start while the previous one of its stream drains
+        if (e == cudaSuccess) e = launch_prep(ap, maps, recs, c0, ncw, p.wc, true);
         if (e == cudaSuccess) e = cudaEventRecord(ss.ev_p[slot], ss.prep);
         if (e == cudaSuccess) e = cudaStreamWaitEvent(ss.chain, ss.ev_p[slot], 0);
         if (e == cudaSuccess) e = launch_chain(ac, p.dvt, recs, sxs, S_in, S_out, ncw, p.wc);
         if (e == cudaSuccess) e = cudaEventRecord(ss.ev_c[slot], ss.chain);
         if (e == cudaSuccess) e = cudaStreamWaitEvent(ss.out, ss.ev_c[slot], 0);
-        if (e == cudaSuccess) e = launch_out(ao, recs, sxs, c0, ncw, p.wc);
+        if (e == cudaSuccess) e = launch_out(ao, recs, sxs, c0, ncw, p.wc, true);
         if (e == cudaSuccess) e = cudaEventRecord(ss.ev_o[slot], ss.out);
     }
     // join: the caller's stream waits for the last chain and the last two outputs

@@ -54,9 +54,30 @@ constexpr size_t kWindowBudgetBytes = size_t(96) << 20;
 FwdTcPlan plan_fwd_tc(int B, int T, int H, int dv, size_t window_budget);
 cudaError_t run_fwd_tc(const FwdArgs &a, const FwdTcPlan &p, uint8_t *ws);
 cudaError_t launch_fwd_tc(const FwdArgs &a);
-cudaError_t launch_prep(const FwdArgs &a, const CUtensorMap *maps, uint8_t *ws, int c0, int ncw, int WC);
+// `overlap`: launch as a programmatic dependent of the previous kernel in the
+// stream, so that it may start before that kernel ends (only where the two
+// touch disjoint data).
+cudaError_t launch_prep(const FwdArgs &a, const CUtensorMap *maps, uint8_t *ws, int c0, int ncw, int WC,
+                        bool overlap);
 cudaError_t launch_chain(const FwdArgs &a, int dvt, const uint8_t *ws, uint8_t *sx, const float *S_in,
                          float *S_out, int ncw, int WC);
-cudaError_t launch_out(const FwdArgs &a, const uint8_t *ws, const uint8_t *sx, int c0, int ncw, int WC);
+cudaError_t launch_out(const FwdArgs &a, const uint8_t *ws, const uint8_t *sx, int c0, int ncw, int WC,
+                       bool overlap);
+// Launch configuration with the programmatic-dependent-launch attribute set when `overlap`.
+struct LaunchCfg {
+    cudaLaunchConfig_t cfg{};
+    cudaLaunchAttribute attr[1];
+    LaunchCfg(dim3 grid, dim3 block, size_t smem, cudaStream_t stream, bool overlap)
+    {
+        cfg.gridDim = grid;
+        cfg.blockDim = block;
+        cfg.dynamicSmemBytes = smem;
+        cfg.stream = stream;
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = overlap ? 1 : 0;
+    }
+};
 
 }  // namespace gdn2

@@ -23,12 +23,18 @@ __host__ __device__ constexpr int align_up(int x, int a) { return (x + a - 1) / 
 // chunk maps the incoming state S to
 //   S_next = Diag(e^{Gamma_C}) S + NG S + Y Z       NG = -Ktil^T T Ebar
 //   O      = QS S + PT Z                            QS = (Qhat - P T Ehat) Diag(e^{Gamma_r})
-// The parts, bf16 UMMA operands with the 128-byte swizzle:
-//   NG  [128 rows = key channel i][128 K = key channel j], K-major, two 16 KB blocks
-//   QS  [64 rows = token][128 K = key channel], K-major, two 8 KB blocks
-//   Y   [128 rows = key channel][64 K = token], K-major, 16 KB:  Y = Ktil^T T
-//   PT  [64 rows = token][64 K = token], K-major, 8 KB:          P T
-//   Z   [64 rows = token (K)][DV = value (N)], MN-major, DV/64 blocks of 8 KB: Z = w v
+// The A operands (NG, QS, Y, PT) are bf16 K-major without swizzle, stored as
+// 16-byte K chunks of all rows in turn: element (row m, k) at byte
+// (k / 8) * (16 * ROWS) + m * 16 + (k % 8) * 2, so that a warp writing one
+// K chunk of 32 consecutive rows stores 512 contiguous bytes, and the UMMA
+// reads the tile with a leading (K) byte offset of 16 * ROWS and a stride
+// (8-row) byte offset of 128.
+//   NG  [128 rows = key channel i][128 K = key channel j]
+//   QS  [64 rows = token][128 K = key channel]
+//   Y   [128 rows = key channel][64 K = token]:  Y = Ktil^T T
+//   PT  [64 rows = token][64 K = token]:         P T
+//   Z   [64 rows = token (K)][DV = value (N)], MN-major B operand with the
+//       128-byte swizzle, DV/64 blocks of 8 KB: Z = w v
 //   DEC [128] fp32: e^{Gamma_C} per key channel
 template <int DV>
 struct Record {
@@ -41,13 +47,20 @@ struct Record {
     static constexpr int BYTES = DEC + 1024;
 };
 
+// Byte offset of K chunk c (8 elements), row m, in a no-swizzle K-major tile of ROWS rows.
+__host__ __device__ constexpr uint32_t kchunk_off(int c, int m, int rows) { return (uint32_t)(c * 16 * rows + m * 16); }
+
 // The chain kernel exports the bf16 image Sx of the state entering every chunk
-// for the output kernel: [128 key channels][DV] as DV/64 blocks of [128 rows][128 B],
-// 128-byte swizzle, i.e. the MN-major B operand layout of the UMMA.
+// for the output kernel: [128 key channels (K)][DV values (N)], an MN-major B
+// operand without swizzle: element (j, n) at byte (n / 8) * 2048 + j * 16 + (n % 8) * 2.
+// A warp holding 8 value columns of 32 consecutive key rows stores 512
+// contiguous bytes; the UMMA reads it with a leading (8-row K group) byte
+// offset of 128 and a stride (8-column N chunk) byte offset of 2048.
 template <int DV>
 struct SxSlot {
     static constexpr int BYTES = 128 * DV * 2;
 };
+__host__ __device__ constexpr uint32_t sx_off(int j, int n) { return (uint32_t)((n >> 3) * 2048 + j * 16 + (n & 7) * 2); }
 
 __device__ __forceinline__ uint4 pack8(const float *f)
 {
