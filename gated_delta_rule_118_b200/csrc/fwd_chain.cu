@@ -48,11 +48,13 @@ struct ChainLayout {
     // one stage: NG | Y | Z tile (NB blocks of [64 tokens][64 values])
     static constexpr int S_NG = 0, S_Y = 32768, S_Z = 49152;
     static constexpr int STAGE = S_Z + NB * 8192;
-    static constexpr int SRB = DVT * 256;                     // one Sx buffer: [128][DVT], no swizzle
-    static constexpr int FIXED = 2 * SRB + 2048 + 1024;       // Sx buffers, barriers, alignment
+    // Sx buffer: [128][DVT], no swizzle.  One is enough: Sx of chunk c + 1 is
+    // written after the UMMA that read Sx of chunk c has completed.
+    static constexpr int SRB = DVT * 256;
+    static constexpr int FIXED = SRB + 2048 + 1024;           // Sx buffer, barriers, alignment
     static constexpr int NS = (4 * STAGE + FIXED <= 232448) ? 4 : (3 * STAGE + FIXED <= 232448) ? 3 : 2;
     static constexpr int SR = NS * STAGE;
-    static constexpr int BAR = SR + 2 * SRB;
+    static constexpr int BAR = SR + SRB;
     static constexpr int NBAR = 2 * NS + 5;  // full[NS], empty[NS], s_done, sx_full, yz_done[2], s_issued
     static constexpr int SLOT = BAR + 8 * NBAR;
     static constexpr int BYTES = SLOT + 16 + 1024;
@@ -102,6 +104,8 @@ chain_kernel(const uint8_t *__restrict__ ws, uint8_t *__restrict__ sx_out, const
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *slot;
+    // this window's chain is resident: the next window's prep may take the other SMs
+    allow_dependent_launch();
 
     if (warp == kProducerWarp) {
         // ------------------------------------------------------------ producer
@@ -158,12 +162,10 @@ chain_kernel(const uint8_t *__restrict__ ws, uint8_t *__restrict__ sx_out, const
                 tc_fence_after();
                 if (ok) {
                     const uint64_t so = (uint64_t)((s * L::STAGE) >> 4);
-                    const uint64_t bo = (uint64_t)((b * L::SRB) >> 4);
                     const uint32_t d = tmem + (uint32_t)(b * DVT);
 #pragma unroll
                     for (int ks = 0; ks < kDK / 16; ++ks)
-                        umma_bf16(d, ng0 + so + (uint64_t)((ks * 4096) >> 4), sx0 + bo + (uint64_t)((ks * 256) >> 4),
-                                  idd, 1);
+                        umma_bf16(d, ng0 + so + (uint64_t)((ks * 4096) >> 4), sx0 + (uint64_t)((ks * 256) >> 4), idd, 1);
                 }
                 umma_commit(s_done);
                 if (cw + NS < ncw) umma_commit(empty + s);
@@ -186,14 +188,14 @@ chain_kernel(const uint8_t *__restrict__ ws, uint8_t *__restrict__ sx_out, const
                 S[j] = v4.x; S[j + 1] = v4.y; S[j + 2] = v4.z; S[j + 3] = v4.w;
             }
         }
-        // Sx(cw) -> buffer cw & 1 (the next UMMA's operand), signal the MMA warp, then
-        // copy the same 16-byte pieces to the exported slot (every warp store covers
-        // 512 contiguous bytes).
+        // Sx(cw) -> the Sx buffer (the next UMMA's operand), signal the MMA warp,
+        // then copy the same 16-byte pieces to the exported slot (every warp store
+        // covers 512 contiguous bytes).
         auto publish_sx = [&](int cw) {
             uint4 px[COLS / 8];
 #pragma unroll
             for (int j = 0; j < COLS; j += 8) px[j / 8] = pack8(S + j);
-            uint8_t *sr = sm + L::SR + (cw & 1) * L::SRB;
+            uint8_t *sr = sm + L::SR;
 #pragma unroll
             for (int j = 0; j < COLS; j += 8) *reinterpret_cast<uint4 *>(sr + sx_off(i, col0 + j)) = px[j / 8];
             fence_proxy_async_smem();
@@ -258,7 +260,8 @@ cudaError_t launch_chain_impl(const FwdArgs &a, const uint8_t *ws, uint8_t *sx, 
 {
     using L = ChainLayout<DV, DVT>;
     auto kern = chain_kernel<DV, DVT>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::BYTES);
+    static std::atomic<unsigned long long> smem_set{0};
+    cudaError_t e = ensure_smem_limit(kern, L::BYTES, smem_set);
     if (e != cudaSuccess) return e;
     dim3 grid(DV / DVT, a.H, a.B);
     kern<<<grid, kChainThreads, L::BYTES, a.stream>>>(ws, sx, S_in, S_out, a.H, ncw, WC, a.err);

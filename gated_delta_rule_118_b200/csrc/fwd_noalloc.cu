@@ -91,7 +91,7 @@ extern "C" gdn2_status gdn2_fwd_chunked_noalloc(const void *q, const void *k, co
         const size_t sx = (dv == 128) ? SxSlot<128>::BYTES : SxSlot<64>::BYTES;
         const size_t per_chunk = (size_t)B * H * (rec + sx);
         if (carry >= kNoAllocScratchBytes || per_chunk > kNoAllocScratchBytes - carry) return GDN2_ERR_SCRATCH_LIMIT;
-        plan = plan_fwd_tc(B, T, H, dv, kNoAllocScratchBytes - carry);
+        plan = plan_fwd_tc(B, T, H, dv, kNoAllocScratchBytes - carry, 0);
         if (plan.ws_bytes > kNoAllocScratchBytes) return GDN2_ERR_SCRATCH_LIMIT;
     }
 

@@ -121,7 +121,8 @@ cudaError_t launch_out_impl(const FwdArgs &a, const uint8_t *ws, const uint8_t *
 {
     using L = OutLayout<DV>;
     auto kern = out_kernel<DV>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::BYTES);
+    static std::atomic<unsigned long long> smem_set{0};
+    cudaError_t e = ensure_smem_limit(kern, L::BYTES, smem_set);
     if (e != cudaSuccess) return e;
     LaunchCfg lc(dim3(ncw, a.H, a.B), dim3(kOutThreads), L::BYTES, a.stream, overlap);
     return cudaLaunchKernelEx(&lc.cfg, kern, ws, sx, (bf16 *)a.o, a.T, a.H, c0, WC, a.err);

@@ -494,7 +494,8 @@ cudaError_t launch_prep_impl(const FwdArgs &a, const CUtensorMap *maps, uint8_t 
 {
     using L = PrepLayout;
     auto kern = prep_kernel<DV>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::BYTES);
+    static std::atomic<unsigned long long> smem_set{0};
+    cudaError_t e = ensure_smem_limit(kern, L::BYTES, smem_set);
     if (e != cudaSuccess) return e;
     LaunchCfg lc(dim3(ncw, a.H, a.B), dim3(kPrepThreads), L::BYTES, a.stream, overlap);
     return cudaLaunchKernelEx(&lc.cfg, kern, maps[0], maps[1], maps[2], maps[3], (const bf16 *)a.v,

@@ -71,7 +71,7 @@ cudaMemPool_t workspace_pool(int dev)
 
 }  // namespace
 
-FwdTcPlan plan_fwd_tc(int B, int T, int H, int dv, size_t window_budget)
+FwdTcPlan plan_fwd_tc(int B, int T, int H, int dv, size_t budget, int num_sms)
 {
     FwdTcPlan p{};
     const long bh = (long)B * H;
@@ -81,8 +81,21 @@ FwdTcPlan plan_fwd_tc(int B, int T, int H, int dv, size_t window_budget)
     p.nchunks = (T + kChunk - 1) / kChunk;
     p.rec_bytes = (dv == 128) ? Record<128>::BYTES : Record<64>::BYTES;
     p.sx_bytes = (dv == 128) ? SxSlot<128>::BYTES : SxSlot<64>::BYTES;
+    // A chain CTA takes a whole SM.  When the chain leaves at least half of the
+    // SMs, a window's prep runs beside the previous window's chain (four windows
+    // in flight); otherwise prep and chain take turns on the whole GPU (two).
+    const long chain_ctas = bh * (dv / p.dvt);
+    p.overlap = num_sms > 0 && chain_ctas * 2 <= num_sms;
+    p.slots = num_sms > 0 ? (p.overlap ? kWindowSlots : 2) : 1;
+    if (num_sms > 0) budget = p.overlap ? kWindowBudgetBytes : kWideWindowBudgetBytes;
     const size_t per_chunk = (size_t)bh * (p.rec_bytes + p.sx_bytes);
-    long wc = per_chunk ? (long)(window_budget / per_chunk) : 0;
+    long wc = per_chunk ? (long)(budget / p.slots / per_chunk) : 0;
+    // beside the chain, a window whose prep CTAs (two per SM) fit the other SMs in
+    // one wave keeps the chain from waiting for a second wave
+    if (p.overlap) {
+        const long cap = 2 * (num_sms - chain_ctas) / bh;
+        if (cap >= 1 && wc > cap) wc = cap;
+    }
     if (wc < 1) wc = 1;
     if (wc > p.nchunks) wc = p.nchunks;
     p.wc = (int)wc;
@@ -90,7 +103,7 @@ FwdTcPlan plan_fwd_tc(int B, int T, int H, int dv, size_t window_budget)
     p.rec_total = (size_t)p.wc * bh * p.rec_bytes;
     p.sx_total = (size_t)p.wc * bh * p.sx_bytes;
     p.carry_bytes = p.nwindows > 1 ? (size_t)bh * 128 * dv * sizeof(float) : 0;
-    p.ws_bytes = p.rec_total + p.sx_total + p.carry_bytes;
+    p.ws_bytes = p.slots * (p.rec_total + p.sx_total) + p.carry_bytes;
     return p;
 }
 
@@ -123,13 +136,12 @@ cudaError_t run_fwd_tc(const FwdArgs &a, const FwdTcPlan &p, uint8_t *ws)
 
 namespace {
 
-// Streams and events of the overlapped schedule, one set per device, created on
-// first use and kept for the life of the process.  The chain stream has the
-// highest priority so that its CTAs are dispatched ahead of pending prep CTAs.
+// The output stream and the events of the overlapped schedule, one set per
+// device, created on first use and kept for the life of the process.
 struct StreamSet {
     std::mutex mu;
-    cudaStream_t prep = nullptr, chain = nullptr, out = nullptr;
-    cudaEvent_t start = nullptr, ev_p[4] = {}, ev_c[4] = {}, ev_o[4] = {};
+    cudaStream_t out = nullptr;
+    cudaEvent_t start = nullptr, ev_c[kWindowSlots] = {}, ev_o[kWindowSlots] = {};
     bool ready = false;
 };
 
@@ -142,14 +154,12 @@ StreamSet *stream_set(int dev)
     if (!ss.ready) {
         int lo = 0, hi = 0;
         if (cudaDeviceGetStreamPriorityRange(&lo, &hi) != cudaSuccess) return nullptr;
-        if (cudaStreamCreateWithPriority(&ss.chain, cudaStreamNonBlocking, hi) != cudaSuccess ||
-            cudaStreamCreateWithFlags(&ss.prep, cudaStreamNonBlocking) != cudaSuccess ||
-            cudaStreamCreateWithFlags(&ss.out, cudaStreamNonBlocking) != cudaSuccess ||
+        // lowest priority: the caller's stream (prep and chain) goes first
+        if (cudaStreamCreateWithPriority(&ss.out, cudaStreamNonBlocking, lo) != cudaSuccess ||
             cudaEventCreateWithFlags(&ss.start, cudaEventDisableTiming) != cudaSuccess)
             return nullptr;
-        for (int i = 0; i < 4; ++i)
-            if (cudaEventCreateWithFlags(&ss.ev_p[i], cudaEventDisableTiming) != cudaSuccess ||
-                cudaEventCreateWithFlags(&ss.ev_c[i], cudaEventDisableTiming) != cudaSuccess ||
+        for (int i = 0; i < kWindowSlots; ++i)
+            if (cudaEventCreateWithFlags(&ss.ev_c[i], cudaEventDisableTiming) != cudaSuccess ||
                 cudaEventCreateWithFlags(&ss.ev_o[i], cudaEventDisableTiming) != cudaSuccess)
                 return nullptr;
         ss.ready = true;
@@ -157,12 +167,19 @@ StreamSet *stream_set(int dev)
     return &ss;
 }
 
-// Overlapped schedule over two workspace halves (window w uses half w % 2):
-//   prep stream:   [wait chain(w-2), out(w-2)]  prep(w)  -> ev_p[w]
-//   chain stream:  [wait prep(w)]               chain(w) -> ev_c[w]
-//   out stream:    [wait chain(w)]              out(w)   -> ev_o[w]
-// so prep of the next window runs while the chain walks the current one.  The
-// caller's stream forks into the three at the start and joins them at the end.
+// Overlapped schedule over p.slots workspace slots (window w uses slot w % p.slots).
+// A chain CTA needs a whole SM, so the chain of a window must not queue behind
+// prep CTAs of later windows.  The caller's stream therefore carries
+//   prep(0), chain(0), prep(1), chain(1), ...
+// With p.overlap, prep(w + 1) is a programmatic dependent of chain(w): it starts
+// once every chain CTA of window w is resident and fills the other SMs while the
+// chain walks window w; chain(w + 1) starts when both are done.  Without it
+// (a chain that takes most SMs) prep and chain take turns.  The output kernels
+// run on their own stream, each after its window's chain:
+//   out stream:    [wait ev_c[w]]  out(w) -> ev_o[w]
+// and before chain(w) the caller's stream waits for the output kernel that last
+// used the slot prep(w + 1) is about to overwrite.  The output stream forks from
+// the caller's stream at the start and joins it at the end.
 cudaError_t run_fwd_tc_overlapped(const FwdArgs &a, const FwdTcPlan &p, uint8_t *ws, StreamSet &ss)
 {
     CUtensorMap maps[6];
@@ -175,44 +192,48 @@ cudaError_t run_fwd_tc_overlapped(const FwdArgs &a, const FwdTcPlan &p, uint8_t 
         !make_map(&maps[4], a.v, BF, 2, a.dv, a.H, a.T, a.B, a.dv, CU_TENSOR_MAP_SWIZZLE_NONE) ||
         !make_map(&maps[5], a.w, BF, 2, a.dv, a.H, a.T, a.B, a.dv, CU_TENSOR_MAP_SWIZZLE_NONE))
         return cudaErrorInvalidValue;
-    const size_t half = p.rec_total + p.sx_total;
-    float *carry = p.carry_bytes ? reinterpret_cast<float *>(ws + 2 * half) : nullptr;
+    const int nslots = p.slots;
+    const size_t slot_bytes = p.rec_total + p.sx_total;
+    float *carry = p.carry_bytes ? reinterpret_cast<float *>(ws + nslots * slot_bytes) : nullptr;
     cudaError_t e = cudaEventRecord(ss.start, a.stream);
-    if (e == cudaSuccess) e = cudaStreamWaitEvent(ss.prep, ss.start, 0);
-    if (e == cudaSuccess) e = cudaStreamWaitEvent(ss.chain, ss.start, 0);
     if (e == cudaSuccess) e = cudaStreamWaitEvent(ss.out, ss.start, 0);
+    auto window = [&](int w, int &c0, int &ncw, uint8_t *&recs, uint8_t *&sxs) {
+        c0 = w * p.wc;
+        ncw = (p.nchunks - c0 < p.wc) ? p.nchunks - c0 : p.wc;
+        recs = ws + (w % nslots) * slot_bytes;
+        sxs = recs + p.rec_total;
+    };
+    const FwdArgs &ac = a;
+    FwdArgs ao = a;
+    ao.stream = ss.out;
+    int c0, ncw;
+    uint8_t *recs, *sxs;
+    if (p.nwindows > 0) {
+        window(0, c0, ncw, recs, sxs);
+        e = launch_prep(ac, maps, recs, c0, ncw, p.wc, false);
+    }
     for (int w = 0; w < p.nwindows && e == cudaSuccess; ++w) {
-        const int c0 = w * p.wc, slot = w & 3;
-        const int ncw = (p.nchunks - c0 < p.wc) ? p.nchunks - c0 : p.wc;
-        uint8_t *recs = ws + (w & 1) * half, *sxs = recs + p.rec_total;
+        const int slot = w % nslots;
+        if (w + 1 < p.nwindows && w + 1 >= nslots) e = cudaStreamWaitEvent(a.stream, ss.ev_o[(w + 1) % nslots], 0);
+        window(w, c0, ncw, recs, sxs);
         const float *S_in = (w == 0) ? a.S0 : carry;
         float *S_out = (w == p.nwindows - 1) ? a.S_T : carry;
-        FwdArgs ap = a, ac = a, ao = a;
-        ap.stream = ss.prep;
-        ac.stream = ss.chain;
-        ao.stream = ss.out;
-        if (w >= 2) {
-            e = cudaStreamWaitEvent(ss.prep, ss.ev_c[(w - 2) & 3], 0);
-            if (e == cudaSuccess) e = cudaStreamWaitEvent(ss.prep, ss.ev_o[(w - 2) & 3], 0);
-        }
-        // prep and output launches of consecutive windows touch disjoint data, so
-        // each may start while the previous one of its stream drains
-        if (e == cudaSuccess) e = launch_prep(ap, maps, recs, c0, ncw, p.wc, true);
-        if (e == cudaSuccess) e = cudaEventRecord(ss.ev_p[slot], ss.prep);
-        if (e == cudaSuccess) e = cudaStreamWaitEvent(ss.chain, ss.ev_p[slot], 0);
         if (e == cudaSuccess) e = launch_chain(ac, p.dvt, recs, sxs, S_in, S_out, ncw, p.wc);
-        if (e == cudaSuccess) e = cudaEventRecord(ss.ev_c[slot], ss.chain);
+        if (e == cudaSuccess && w + 1 < p.nwindows) {
+            int c1, n1;
+            uint8_t *r1, *x1;
+            window(w + 1, c1, n1, r1, x1);
+            e = launch_prep(ac, maps, r1, c1, n1, p.wc, p.overlap);
+        }
+        if (e == cudaSuccess) e = cudaEventRecord(ss.ev_c[slot], a.stream);
         if (e == cudaSuccess) e = cudaStreamWaitEvent(ss.out, ss.ev_c[slot], 0);
+        // output launches of consecutive windows write disjoint rows
         if (e == cudaSuccess) e = launch_out(ao, recs, sxs, c0, ncw, p.wc, true);
         if (e == cudaSuccess) e = cudaEventRecord(ss.ev_o[slot], ss.out);
     }
-    // join: the caller's stream waits for the last chain and the last two outputs
-    if (e == cudaSuccess && p.nwindows > 0) {
-        const int last = p.nwindows - 1;
-        e = cudaStreamWaitEvent(a.stream, ss.ev_c[last & 3], 0);
-        if (e == cudaSuccess) e = cudaStreamWaitEvent(a.stream, ss.ev_o[last & 3], 0);
-        if (e == cudaSuccess && last >= 1) e = cudaStreamWaitEvent(a.stream, ss.ev_o[(last - 1) & 3], 0);
-    }
+    // join: the caller's stream waits for the last output (the output stream runs
+    // its windows in order)
+    if (e == cudaSuccess && p.nwindows > 0) e = cudaStreamWaitEvent(a.stream, ss.ev_o[(p.nwindows - 1) % nslots], 0);
     return e;
 }
 
@@ -226,9 +247,8 @@ cudaError_t launch_fwd_tc(const FwdArgs &a)
     cudaMemPool_t pool = workspace_pool(dev);
     StreamSet *ss = stream_set(dev);
     if (!pool || !ss) return cudaErrorMemoryAllocation;
-    // two window halves of half the budget each
-    FwdTcPlan p = plan_fwd_tc(a.B, a.T, a.H, a.dv, kWindowBudgetBytes / 2);
-    const size_t bytes = 2 * (p.rec_total + p.sx_total) + p.carry_bytes;
+    const FwdTcPlan p = plan_fwd_tc(a.B, a.T, a.H, a.dv, 0, a.num_sms);
+    const size_t bytes = p.ws_bytes;
     void *ws = nullptr;
     e = cudaMallocFromPoolAsync(&ws, bytes, pool, a.stream);
     if (e != cudaSuccess) return e;

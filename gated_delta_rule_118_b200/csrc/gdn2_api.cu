@@ -152,7 +152,16 @@ extern "C" int gdn2_fwd_chunked_launches(int B, int T, int H, int dk, int dv, gd
     if ((dtype != GDN2_F32 && dtype != GDN2_BF16) || B <= 0 || H <= 0 || T < 0) return -1;
     if (check_dims(dk, dv) != GDN2_OK || B > 65535 || H > 65535) return -1;
     if (T == 0) return 0;
-    if (dtype == GDN2_BF16 && dk == 128) return 3 * plan_fwd_tc(B, T, H, dv, kWindowBudgetBytes / 2).nwindows;
+    if (dtype == GDN2_BF16 && dk == 128) {
+        // the window plan depends on the SM count of the current device (none: plan for 148)
+        int dev = 0, sms = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+            sms = 0;
+            cudaGetLastError();
+        }
+        return 3 * plan_fwd_tc(B, T, H, dv, kWindowBudgetBytes, sms > 0 ? sms : 148).nwindows;
+    }
     return 1;
 }
 

@@ -7,6 +7,8 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include <atomic>
+
 namespace gdn2 {
 
 struct DecodeArgs {
@@ -49,9 +51,18 @@ struct FwdTcPlan {
     size_t sx_total;  // state images of one window
     size_t carry_bytes; // state carried between windows
     size_t ws_bytes;    // total workspace
+    int slots;          // windows in flight (workspace slots)
+    bool overlap;       // a window's prep runs beside the previous window's chain
 };
-constexpr size_t kWindowBudgetBytes = size_t(96) << 20;
-FwdTcPlan plan_fwd_tc(int B, int T, int H, int dv, size_t window_budget);
+// Workspace of the allocating entry point: kWindowSlots windows in flight when a
+// window's prep overlaps the previous chain, else two larger ones.
+constexpr size_t kWindowBudgetBytes = size_t(128) << 20;
+constexpr size_t kWideWindowBudgetBytes = size_t(512) << 20;
+constexpr int kWindowSlots = 4;
+// num_sms > 0: plan the overlapped schedule of the allocating entry point on a
+// device with num_sms SMs (budget ignored); num_sms == 0: one window slot of
+// `budget` bytes (the no-allocation entry point).
+FwdTcPlan plan_fwd_tc(int B, int T, int H, int dv, size_t budget, int num_sms);
 cudaError_t run_fwd_tc(const FwdArgs &a, const FwdTcPlan &p, uint8_t *ws);
 cudaError_t launch_fwd_tc(const FwdArgs &a);
 // `overlap`: launch as a programmatic dependent of the previous kernel in the
@@ -63,6 +74,21 @@ cudaError_t launch_chain(const FwdArgs &a, int dvt, const uint8_t *ws, uint8_t *
                          float *S_out, int ncw, int WC);
 cudaError_t launch_out(const FwdArgs &a, const uint8_t *ws, const uint8_t *sx, int c0, int ncw, int WC,
                        bool overlap);
+// Raise a kernel's dynamic shared-memory limit on the current device, once per
+// device (bit d of `done` records device d).
+template <typename Kernel>
+cudaError_t ensure_smem_limit(Kernel kern, int bytes, std::atomic<unsigned long long> &done)
+{
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    const unsigned long long bit = 1ull << (dev & 63);
+    if (done.load(std::memory_order_acquire) & bit) return cudaSuccess;
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e == cudaSuccess) done.fetch_or(bit, std::memory_order_release);
+    return e;
+}
+
 // Launch configuration with the programmatic-dependent-launch attribute set when `overlap`.
 struct LaunchCfg {
     cudaLaunchConfig_t cfg{};
