@@ -40,7 +40,14 @@ N_INPUT_SETS = 4  # rotating input sets: 4 x 136 MB > 126 MB of L2
 # the current kernels (None once a kernel has changed since the capture).  The
 # forward is three kernels per window (profiles/*_layer_bf16.md hold each one);
 # decode: profiles/decode_kernel_decode_b256.md.
-NCU_TRAFFIC_BYTES = {"fwd": None, "decode": 281.03e6 + 215.97e6}
+# DRAM bytes per launch from ncu captures (profiles/): the decode kernel, and one
+# forward call summed over its prep, chain and output launches, each scaled from
+# one captured window (14 chunks x 16 heads) by the chunks it processes.  ncu
+# captures each kernel cold, so the per-chunk records that prep writes and the
+# chain and output kernels read back count as DRAM traffic here.
+NCU_TRAFFIC_BYTES = {"fwd": round((25.769728e6 + 17.152e3) / 224 * 1024 + 15.874560e6 / 14 * 64
+                                  + 16.534016e6 / 224 * 1024),
+                     "decode": 281.078016e6 + 213.638144e6}
 
 
 def peaks():
