@@ -104,8 +104,11 @@ chain_kernel(const uint8_t *__restrict__ ws, uint8_t *__restrict__ sx_out, const
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *slot;
-    // this window's chain is resident: the next window's prep may take the other SMs
+    // This window's chain is resident: the next window's prep may take the other
+    // SMs.  Then wait for this window's prep (its records, and through its own
+    // final wait the previous chain and the state it carries).
     allow_dependent_launch();
+    wait_prior_grid();
 
     if (warp == kProducerWarp) {
         // ------------------------------------------------------------ producer
@@ -256,7 +259,7 @@ chain_kernel(const uint8_t *__restrict__ ws, uint8_t *__restrict__ sx_out, const
 
 template <int DV, int DVT>
 cudaError_t launch_chain_impl(const FwdArgs &a, const uint8_t *ws, uint8_t *sx, const float *S_in, float *S_out,
-                              int ncw, int WC)
+                              int ncw, int WC, bool overlap)
 {
     using L = ChainLayout<DV, DVT>;
     auto kern = chain_kernel<DV, DVT>;
@@ -264,18 +267,18 @@ cudaError_t launch_chain_impl(const FwdArgs &a, const uint8_t *ws, uint8_t *sx, 
     cudaError_t e = ensure_smem_limit(kern, L::BYTES, smem_set);
     if (e != cudaSuccess) return e;
     dim3 grid(DV / DVT, a.H, a.B);
-    kern<<<grid, kChainThreads, L::BYTES, a.stream>>>(ws, sx, S_in, S_out, a.H, ncw, WC, a.err);
-    return cudaGetLastError();
+    LaunchCfg lc(grid, dim3(kChainThreads), L::BYTES, a.stream, overlap);
+    return cudaLaunchKernelEx(&lc.cfg, kern, ws, sx, S_in, S_out, a.H, ncw, WC, a.err);
 }
 
 cudaError_t launch_chain(const FwdArgs &a, int dvt, const uint8_t *ws, uint8_t *sx, const float *S_in,
-                         float *S_out, int ncw, int WC)
+                         float *S_out, int ncw, int WC, bool overlap)
 {
     if (a.dv == 128) {
-        if (dvt == 128) return launch_chain_impl<128, 128>(a, ws, sx, S_in, S_out, ncw, WC);
-        return launch_chain_impl<128, 64>(a, ws, sx, S_in, S_out, ncw, WC);
+        if (dvt == 128) return launch_chain_impl<128, 128>(a, ws, sx, S_in, S_out, ncw, WC, overlap);
+        return launch_chain_impl<128, 64>(a, ws, sx, S_in, S_out, ncw, WC, overlap);
     }
-    return launch_chain_impl<64, 64>(a, ws, sx, S_in, S_out, ncw, WC);
+    return launch_chain_impl<64, 64>(a, ws, sx, S_in, S_out, ncw, WC, overlap);
 }
 
 }  // namespace gdn2

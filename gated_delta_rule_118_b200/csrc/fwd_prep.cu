@@ -484,6 +484,9 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         tc_fence_after();
         tmem_dealloc(tmem, L::TMEM_COLS);
     }
+    // When launched behind the previous window's chain, end only after it: the
+    // next chain waits for this grid and so also for the state it carries.
+    wait_prior_grid();
 }
 
 }  // namespace

@@ -127,7 +127,7 @@ cudaError_t run_fwd_tc(const FwdArgs &a, const FwdTcPlan &p, uint8_t *ws)
         const float *S_in = (w == 0) ? a.S0 : carry;
         float *S_out = (w == p.nwindows - 1) ? a.S_T : carry;
         cudaError_t e = launch_prep(a, maps, recs, c0, ncw, p.wc, false);
-        if (e == cudaSuccess) e = launch_chain(a, p.dvt, recs, sxs, S_in, S_out, ncw, p.wc);
+        if (e == cudaSuccess) e = launch_chain(a, p.dvt, recs, sxs, S_in, S_out, ncw, p.wc, false);
         if (e == cudaSuccess) e = launch_out(a, recs, sxs, c0, ncw, p.wc, false);
         if (e != cudaSuccess) return e;
     }
@@ -218,7 +218,7 @@ cudaError_t run_fwd_tc_overlapped(const FwdArgs &a, const FwdTcPlan &p, uint8_t 
         window(w, c0, ncw, recs, sxs);
         const float *S_in = (w == 0) ? a.S0 : carry;
         float *S_out = (w == p.nwindows - 1) ? a.S_T : carry;
-        if (e == cudaSuccess) e = launch_chain(ac, p.dvt, recs, sxs, S_in, S_out, ncw, p.wc);
+        if (e == cudaSuccess) e = launch_chain(ac, p.dvt, recs, sxs, S_in, S_out, ncw, p.wc, p.overlap);
         if (e == cudaSuccess && w + 1 < p.nwindows) {
             int c1, n1;
             uint8_t *r1, *x1;

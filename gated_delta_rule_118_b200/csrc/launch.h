@@ -71,7 +71,7 @@ cudaError_t launch_fwd_tc(const FwdArgs &a);
 cudaError_t launch_prep(const FwdArgs &a, const CUtensorMap *maps, uint8_t *ws, int c0, int ncw, int WC,
                         bool overlap);
 cudaError_t launch_chain(const FwdArgs &a, int dvt, const uint8_t *ws, uint8_t *sx, const float *S_in,
-                         float *S_out, int ncw, int WC);
+                         float *S_out, int ncw, int WC, bool overlap);
 cudaError_t launch_out(const FwdArgs &a, const uint8_t *ws, const uint8_t *sx, int c0, int ncw, int WC,
                        bool overlap);
 // Raise a kernel's dynamic shared-memory limit on the current device, once per

@@ -122,6 +122,10 @@ __device__ __forceinline__ void fence_proxy_async_smem()
 // dependent, start while this grid is still running (a no-op otherwise).
 __device__ __forceinline__ void allow_dependent_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 
+// Wait until the grid this one was launched as a programmatic dependent of has
+// completed and its memory operations are visible (returns at once otherwise).
+__device__ __forceinline__ void wait_prior_grid() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // ---------------------------------------------------------------- tcgen05
 __device__ __forceinline__ void tmem_alloc(uint32_t *dst_smem, uint32_t ncols)
 {
