@@ -1,68 +1,16 @@
-// fwd_prep.cu -- the state-independent part of the chunkwise forward (bf16 inputs).
-//
-// One CTA per (batch, head, chunk) computes every quantity of the chunkwise WY
-// form that does not depend on the state carried in from earlier chunks
-// ("Gated DeltaNet-2", iplexlaw.co.kr, section "Procesamiento del token y
-// entrenamiento paralelo"; gist.science, section 3: the cumulative per-channel
-// decay is folded into asymmetric erase/key factors and a lower triangular
-// system (I + T)^{-1} is solved per chunk).  With Gamma the chunk-local
-// cumulative log-decay (fp32) and r the chunk midpoint:
-//   Ehat = e^{Gamma-Gamma_r} b k    Qhat = e^{Gamma-Gamma_r} q
-//   Khat = e^{Gamma_r-Gamma} k      Z = w v
-//   A = strict_lower(Ehat Khat^T)   P = lower(Qhat Khat^T)   T = (I + A)^{-1}
-//   Y = e^{Gamma_C-Gamma_r} Khat^T T  (= Ktil^T T with Ktil = e^{Gamma_C-Gamma} k)
-//   PT = P T    G = Y Ehat    Q' = Qhat - PT Ehat
-// and the record keeps NG = -G Diag(e^{Gamma_r}), QS = Q' Diag(e^{Gamma_r}),
-// Y, PT, Z and e^{Gamma_C}, so that for the incoming state S
-//   S_next = e^{Gamma_C} S + NG S + Y Z        O = QS S + PT Z.
-// Nothing here depends on the values except Z, which is a plain product.
-//
-// Layout of the work on one SM: the CTA fits in half of the shared memory,
-// tensor memory and register file, so two chunks are in flight per SM and one
-// hides the other's load and UMMA latencies.  q, k, b and log_alpha arrive by
-// TMA straight into the operand buffers and the factors are formed in place;
-// v and w are read with plain vector loads and Z goes straight to the record.
-// Products are tcgen05 UMMAs with fp32 accumulators in tensor memory, three
-// round trips in all (Gram; Y and PT; G and P T Ehat); the solve is fp32
-// (16x16 diagonal blocks by substitution on CUDA cores, then two levels of
-// block merging whose small products run as warp-level tf32 MMAs).  Record
-// pieces go straight from the tensor-memory readouts to the record, each warp
-// store covering 512 contiguous bytes.
+// fwd_prep.cu -- the windowed prep kernel: one CTA of 256 threads per
+// (batch, head, chunk) of a window, two CTAs per SM, running the chunk prep of
+// prep_body.cuh (the state-independent part of the chunkwise forward).
 #include <cuda.h>
 
 #include "launch.h"
-#include "tc_common.cuh"
+#include "prep_body.cuh"
 
 namespace gdn2 {
 namespace {
 
 using namespace sm100;
-
-constexpr int kPrepThreads = 256;
-constexpr int kDK = 128;
-
-struct PrepLayout {
-    static constexpr int EQ = 0;          // [Ehat;Qhat]: b, q arrive here
-    static constexpr int KH = 32768;      // solve scratch -> Y (no swizzle)
-    static constexpr int KT = 49152;      // k arrives here -> Khat -> PT (no swizzle)
-    static constexpr int LA = 65536;      // log_alpha -> fp32 A | fp32 T -> bf16 T over A
-    static constexpr int PO = 98304;      // Gamma quarter totals -> P
-    static constexpr int DEC = 106496;    // e^{Gamma_C-Gamma_r}[128], e^{Gamma_r}[128]
-    static constexpr int BAR = 107520;
-    static constexpr int SLOT = BAR + 16;
-    static constexpr int BYTES = SLOT + 16 + 1024;
-    static constexpr int TX = 3 * 16384 + 32768;  // q, k, b, log_alpha
-    static constexpr int AF = LA, TF = LA + 16384, TB = LA, XS = KH, TOT = PO;
-    // tensor memory: Gram in [0, 64); then Y in [0, 64), PT in [64, 128); then G in [0, 128), P T Ehat in [128, 256)
-    static constexpr uint32_t TM_GRAM = 0, TM_Y = 0, TM_PT = 64, TM_G = 0, TM_PW = 128, TMEM_COLS = 256;
-};
-static_assert(PrepLayout::BYTES * 2 + 2048 <= 233472, "two CTAs per SM");
-
-__device__ __forceinline__ void tmem_ld32_wait(uint32_t taddr, float (&r)[32])
-{
-    tmem_ld32(taddr, r);
-    tmem_ld_wait();
-}
+using namespace prep;
 
 template <int DV>
 __global__ void __launch_bounds__(kPrepThreads, 2)
@@ -75,35 +23,19 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     using R = Record<DV>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int wq = warp & 3, wh = warp >> 2;  // TMEM lane quarter, column half
+    const int tid = threadIdx.x, warp = tid >> 5;
     const int cw = blockIdx.x, h = blockIdx.y, bi = blockIdx.z;
     const int t0 = (c0 + cw) * kChunk;
-    const int Lc = min(kChunk, Tlen - t0);
     uint64_t *bar_tma = reinterpret_cast<uint64_t *>(sm + L::BAR);
     uint64_t *bar_mma = bar_tma + 1;
     uint32_t *slot = reinterpret_cast<uint32_t *>(sm + L::SLOT);
-    float *la = reinterpret_cast<float *>(sm + L::LA);  // [64][128] fp32
-    float *Af = reinterpret_cast<float *>(sm + L::AF);
-    float *Tf = reinterpret_cast<float *>(sm + L::TF);
-    float *Xs = reinterpret_cast<float *>(sm + L::XS);
-    float *dec = reinterpret_cast<float *>(sm + L::DEC);
-    float *tot = reinterpret_cast<float *>(sm + L::TOT);
-    const uint32_t sbase = smem_u32(sm);
     uint8_t *rec = ws + (((long)bi * H + h) * WC + cw) * (long)R::BYTES;
-    uint32_t mma_phase = 0;
 
     if (tid == 0) {
         mbar_init(bar_tma, 1);
         mbar_init(bar_mma, 1);
         fence_mbar_init();
-        mbar_arrive_expect_tx(bar_tma, (uint32_t)L::TX);
-        for (int kb = 0; kb < 2; ++kb) {
-            tma_load_4d(sm + L::EQ + kb * 16384 + 8192, &tm_q, bar_tma, kb * 64, h, t0, bi);
-            tma_load_4d(sm + L::EQ + kb * 16384, &tm_b, bar_tma, kb * 64, h, t0, bi);
-            tma_load_4d(sm + L::KT + kb * 8192, &tm_k, bar_tma, kb * 64, h, t0, bi);
-        }
-        tma_load_4d(sm + L::LA, &tm_la, bar_tma, 0, h, t0, bi);
+        prep_issue_loads(sm, bar_tma, &tm_q, &tm_k, &tm_b, &tm_la, t0, h, bi);
     }
     if (warp == 0) {
         tmem_alloc(slot, L::TMEM_COLS);
@@ -111,373 +43,12 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     }
     // chunks are independent: the next window's prep may start filling SMs
     allow_dependent_launch();
-    // v and w for Z = w v: plain vector loads, issued before anything waits
-    // (tokens past the sequence end give zero rows of Z)
-    constexpr int ZV = 64 * DV / 8 / kPrepThreads;  // 16-byte vectors per thread
-    uint4 vv[ZV], wv[ZV];
-#pragma unroll
-    for (int m = 0; m < ZV; ++m) {
-        const int idx = tid + m * kPrepThreads;
-        const int t = idx / (DV / 8), j = (idx % (DV / 8)) * 8;
-        vv[m] = make_uint4(0, 0, 0, 0);
-        wv[m] = make_uint4(0, 0, 0, 0);
-        if (t < Lc) {
-            const long off = (((long)bi * Tlen + t0 + t) * H + h) * DV + j;
-            vv[m] = __ldg(reinterpret_cast<const uint4 *>(vg + off));
-            wv[m] = __ldg(reinterpret_cast<const uint4 *>(wg + off));
-        }
-    }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *slot;
-    const uint32_t lane_base = (uint32_t)(wq * 32) << 16;
-
-    // One thread polls each barrier; the others park on the CTA barrier, which
-    // leaves the issue slots to the co-resident CTA.  tcgen05.fence::after
-    // orders the tensor-memory reads after that barrier.
-    auto mma_done = [&]() {
-        const bool mine = (tid == 0) ? mbar_wait(bar_mma, mma_phase, err) : true;
-        mma_phase ^= 1;
-        const bool all = __syncthreads_and(mine) != 0;
-        tc_fence_after();
-        return all;
-    };
-    bool ok = __syncthreads_and((tid == 0) ? mbar_wait(bar_tma, 0, err) : true) != 0;
-
-    if (ok) {
-        // ---------------------------------------------------------- Gamma and factors (in place)
-        const int p = tid & 63, qr = tid >> 6;           // channel pair, token quarter
-        const int kb = p >> 5, cb = (p & 31) * 4;
-        float2 lv[16];
-#pragma unroll
-        for (int u = 0; u < 16; ++u) lv[u] = *reinterpret_cast<const float2 *>(la + (qr * 16 + u) * kDK + 2 * p);
-        float g0 = 0.f, g1 = 0.f;
-#pragma unroll
-        for (int u = 0; u < 16; ++u) {
-            g0 += lv[u].x; g1 += lv[u].y;
-            lv[u] = make_float2(g0, g1);
-        }
-        tot[qr * kDK + 2 * p] = g0;
-        tot[qr * kDK + 2 * p + 1] = g1;
-        __syncthreads();
-        float pre0 = 0.f, pre1 = 0.f, gc0 = 0.f, gc1 = 0.f;
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            const float a0 = tot[q * kDK + 2 * p], a1 = tot[q * kDK + 2 * p + 1];
-            if (q < qr) { pre0 += a0; pre1 += a1; }
-            gc0 += a0; gc1 += a1;
-        }
-        // midpoint reference: Gamma after 32 tokens (tokens past T carry log_alpha = 0)
-        const float gr0 = tot[2 * p] + tot[kDK + 2 * p], gr1 = tot[2 * p + 1] + tot[kDK + 2 * p + 1];
-        if (qr == 0) {
-            const float e0 = expf(gc0), e1 = expf(gc1);
-            dec[2 * p] = expf(gc0 - gr0);
-            dec[2 * p + 1] = expf(gc1 - gr1);
-            dec[kDK + 2 * p] = expf(gr0);
-            dec[kDK + 2 * p + 1] = expf(gr1);
-            *reinterpret_cast<float2 *>(rec + R::DEC + 8 * p) = make_float2(e0, e1);
-        }
-        uint8_t *eq = sm + L::EQ + kb * 16384, *kt = sm + L::KT + kb * 8192;
-        unsigned int bad = 0;
-        const float sh0 = pre0 - gr0, sh1 = pre1 - gr1;
-#pragma unroll
-        for (int u = 0; u < 16; ++u) {
-            const int t = qr * 16 + u;
-            const float x0 = lv[u].x + sh0, x1 = lv[u].y + sh1;
-            bad |= (fabsf(x0) > kMaxHalfChunkLogDecay) | (fabsf(x1) > kMaxHalfChunkLogDecay);
-            const float up0 = ex2_approx(x0 * kLog2e), up1 = ex2_approx(x1 * kLog2e);
-            const float dn0 = ex2_approx(-x0 * kLog2e), dn1 = ex2_approx(-x1 * kLog2e);
-            const uint32_t off = swz_off(t, cb, 128);
-            const float2 kv = ld_bf16x2(kt + off), bv = ld_bf16x2(eq + off), qv = ld_bf16x2(eq + 8192 + off);
-            st_bf16x2(eq + off, up0 * bv.x * kv.x, up1 * bv.y * kv.y);
-            st_bf16x2(eq + 8192 + off, up0 * qv.x, up1 * qv.y);
-            st_bf16x2(kt + off, dn0 * kv.x, dn1 * kv.y);
-        }
-        if (bad) atomicOr(err, kErrRange);
-        fence_proxy_async_smem();
-        __syncthreads();
-
-        // ---------------------------------------------------------- Gram: [Ehat;Qhat] Khat^T
-        if (tid == 0) {
-            tc_fence_after();
-            const uint32_t id = idesc_bf16(128, 64, 0, 0);
-#pragma unroll
-            for (int ks = 0; ks < kDK / 16; ++ks) {
-                const uint32_t kofs = (ks & 3) * 32;
-                umma_bf16(tmem + L::TM_G, smem_desc(sbase + L::EQ + (ks >> 2) * 16384 + kofs, 16, 1024, kSw128),
-                          smem_desc(sbase + L::KT + (ks >> 2) * 8192 + kofs, 16, 1024, kSw128), id, ks > 0);
-            }
-            umma_commit(bar_mma);
-        }
-        // Z = w v while the Gram runs, straight into the record (MN-major operand
-        // blocks of 64 value columns; each warp fills whole 128-byte rows)
-#pragma unroll
-        for (int m = 0; m < ZV; ++m) {
-            const int idx = tid + m * kPrepThreads;
-            const int t = idx / (DV / 8), j = (idx % (DV / 8)) * 8;
-            float fv[8], fw[8], fz[8];
-            unpack8(vv[m], fv);
-            unpack8(wv[m], fw);
-#pragma unroll
-            for (int u = 0; u < 8; ++u) fz[u] = fv[u] * fw[u];
-            *reinterpret_cast<uint4 *>(rec + R::Z + (j >> 6) * 8192 + swz_off(t, (j & 63) * 2, 128)) = pack8(fz);
-        }
-        ok = mma_done();
-    }
-
-    if (ok) {
-        // ---------------------------------------------------------- A (fp32) and P (bf16)
-        {
-            const int r = wq * 32 + lane;
-            float v[32];
-            tmem_ld32_wait(tmem + lane_base + L::TM_GRAM + wh * 32, v);
-            if (r < 64) {
-                const int t = r;
-#pragma unroll
-                for (int s4 = 0; s4 < 32; s4 += 4) {
-                    const int s = wh * 32 + s4;
-                    float4 a4;
-                    a4.x = (s + 0 < t) ? v[s4 + 0] : 0.f;
-                    a4.y = (s + 1 < t) ? v[s4 + 1] : 0.f;
-                    a4.z = (s + 2 < t) ? v[s4 + 2] : 0.f;
-                    a4.w = (s + 3 < t) ? v[s4 + 3] : 0.f;
-                    *reinterpret_cast<float4 *>(Af + af_off(t, s)) = a4;
-                }
-            } else {
-                const int t = r - 64;
-#pragma unroll
-                for (int s8 = 0; s8 < 32; s8 += 8) {
-                    float f[8];
-#pragma unroll
-                    for (int u = 0; u < 8; ++u) f[u] = (wh * 32 + s8 + u <= t) ? v[s8 + u] : 0.f;
-                    *reinterpret_cast<uint4 *>(sm + L::PO + swz_off(t, (wh * 32 + s8) * 2, 128)) = pack8(f);
-                }
-            }
-            // T starts as zero (log_alpha, consumed by the Gamma scan, gives its room to A and T)
-#pragma unroll
-            for (int m = 0; m < 4; ++m)
-                reinterpret_cast<float4 *>(Tf)[tid + m * kPrepThreads] = make_float4(0.f, 0.f, 0.f, 0.f);
-        }
-        tc_fence_before();
-        __syncthreads();
-
-        // ---------------------------------------------------------- T = (I + A)^{-1}
-        // (a) diagonal 16x16 blocks: one column per thread, rows of A read as float4
-        if (tid < 64) {
-            const int b0 = (tid >> 4) * 16, j = tid & 15;
-            float x[16];
-#pragma unroll
-            for (int t = 0; t < 16; ++t) {
-                float a[16];
-#pragma unroll
-                for (int s4 = 0; s4 < 16; s4 += 4) {
-                    const float4 a4 = *reinterpret_cast<const float4 *>(Af + af_off(b0 + t, b0 + s4));
-                    a[s4] = a4.x; a[s4 + 1] = a4.y; a[s4 + 2] = a4.z; a[s4 + 3] = a4.w;
-                }
-                float acc0 = (t == j) ? 1.f : 0.f, acc1 = 0.f;
-#pragma unroll
-                for (int s = 0; s < t; ++s) {
-                    if (s & 1) acc1 -= a[s] * x[s];
-                    else acc0 -= a[s] * x[s];
-                }
-                x[t] = acc0 + acc1;
-                Tf[af_off(b0 + t, b0 + j)] = x[t];
-            }
-        }
-        __syncthreads();
-        // (b), (c): the merges are small products inside a dependency chain; they
-        // run as warp-level tf32 MMAs (m16n8k8) on the fp32 blocks.  g, c: fragment
-        // coordinates of this lane.
-        const int fg = lane >> 2, fc = lane & 3;
-        // (b) T_{b+1,b} = -D_{b+1} (A_{b+1,b} D_b) for the pairs (0,1), (2,3).
-        //     Warp w < 4: pair w >> 1, 8-column tile w & 1 of the 16x16 block.
-        if (warp < 4) {
-            const int which = warp >> 1, n0 = (warp & 1) * 8;
-            const int R0 = 16 + 32 * which, C0 = 32 * which;
-            float d[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-            for (int k0 = 0; k0 < 16; k0 += 8) {
-                mma_tf32(d, to_tf32(Af[af_off(R0 + fg, C0 + k0 + fc)]), to_tf32(Af[af_off(R0 + fg + 8, C0 + k0 + fc)]),
-                         to_tf32(Af[af_off(R0 + fg, C0 + k0 + fc + 4)]), to_tf32(Af[af_off(R0 + fg + 8, C0 + k0 + fc + 4)]),
-                         to_tf32(Tf[af_off(C0 + k0 + fc, C0 + n0 + fg)]), to_tf32(Tf[af_off(C0 + k0 + fc + 4, C0 + n0 + fg)]));
-            }
-            float *x = Xs + which * 256;  // X[16][16]
-            x[fg * 16 + n0 + 2 * fc] = d[0];
-            x[fg * 16 + n0 + 2 * fc + 1] = d[1];
-            x[(fg + 8) * 16 + n0 + 2 * fc] = d[2];
-            x[(fg + 8) * 16 + n0 + 2 * fc + 1] = d[3];
-        }
-        __syncthreads();
-        if (warp < 4) {
-            const int which = warp >> 1, n0 = (warp & 1) * 8;
-            const int R0 = 16 + 32 * which, C0 = 32 * which;
-            const float *x = Xs + which * 256;
-            float d[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-            for (int k0 = 0; k0 < 16; k0 += 8) {
-                mma_tf32(d, to_tf32(Tf[af_off(R0 + fg, R0 + k0 + fc)]), to_tf32(Tf[af_off(R0 + fg + 8, R0 + k0 + fc)]),
-                         to_tf32(Tf[af_off(R0 + fg, R0 + k0 + fc + 4)]), to_tf32(Tf[af_off(R0 + fg + 8, R0 + k0 + fc + 4)]),
-                         to_tf32(x[(k0 + fc) * 16 + n0 + fg]), to_tf32(x[(k0 + fc + 4) * 16 + n0 + fg]));
-            }
-            Tf[af_off(R0 + fg, C0 + n0 + 2 * fc)] = -d[0];
-            Tf[af_off(R0 + fg, C0 + n0 + 2 * fc + 1)] = -d[1];
-            Tf[af_off(R0 + fg + 8, C0 + n0 + 2 * fc)] = -d[2];
-            Tf[af_off(R0 + fg + 8, C0 + n0 + 2 * fc + 1)] = -d[3];
-        }
-        __syncthreads();
-        // (c) T[32:64, 0:32] = -T_BB (A[32:64, 0:32] T_AA).  Warp w: 16-row tile w >> 2,
-        //     8-column tile w & 3 of the 32x32 block; T_AA and T_BB are lower triangular.
-        {
-            const int m0 = (warp >> 2) * 16, n0 = (warp & 3) * 8;
-            float d[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-            for (int k0 = 0; k0 < 32; k0 += 8) {
-                if (k0 + 8 <= n0) continue;  // rows k of T_AA above column n0 are zero
-                mma_tf32(d, to_tf32(Af[af_off(32 + m0 + fg, k0 + fc)]), to_tf32(Af[af_off(32 + m0 + fg + 8, k0 + fc)]),
-                         to_tf32(Af[af_off(32 + m0 + fg, k0 + fc + 4)]), to_tf32(Af[af_off(32 + m0 + fg + 8, k0 + fc + 4)]),
-                         to_tf32(Tf[af_off(k0 + fc, n0 + fg)]), to_tf32(Tf[af_off(k0 + fc + 4, n0 + fg)]));
-            }
-            Xs[(m0 + fg) * 32 + n0 + 2 * fc] = d[0];
-            Xs[(m0 + fg) * 32 + n0 + 2 * fc + 1] = d[1];
-            Xs[(m0 + fg + 8) * 32 + n0 + 2 * fc] = d[2];
-            Xs[(m0 + fg + 8) * 32 + n0 + 2 * fc + 1] = d[3];
-        }
-        __syncthreads();
-        {
-            const int m0 = (warp >> 2) * 16, n0 = (warp & 3) * 8;
-            float d[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-            for (int k0 = 0; k0 < 32; k0 += 8) {
-                if (k0 >= m0 + 16) continue;  // columns k of T_BB right of row m0 + 15 are zero
-                mma_tf32(d, to_tf32(Tf[af_off(32 + m0 + fg, 32 + k0 + fc)]),
-                         to_tf32(Tf[af_off(32 + m0 + fg + 8, 32 + k0 + fc)]),
-                         to_tf32(Tf[af_off(32 + m0 + fg, 32 + k0 + fc + 4)]),
-                         to_tf32(Tf[af_off(32 + m0 + fg + 8, 32 + k0 + fc + 4)]),
-                         to_tf32(Xs[(k0 + fc) * 32 + n0 + fg]), to_tf32(Xs[(k0 + fc + 4) * 32 + n0 + fg]));
-            }
-            Tf[af_off(32 + m0 + fg, n0 + 2 * fc)] = -d[0];
-            Tf[af_off(32 + m0 + fg, n0 + 2 * fc + 1)] = -d[1];
-            Tf[af_off(32 + m0 + fg + 8, n0 + 2 * fc)] = -d[2];
-            Tf[af_off(32 + m0 + fg + 8, n0 + 2 * fc + 1)] = -d[3];
-        }
-        __syncthreads();
-        // (d) T -> bf16 operand over A (which has served its purpose)
-        {
-            const int t = tid >> 2, g = (tid & 3) * 16;
-            float f[16];
-#pragma unroll
-            for (int u = 0; u < 16; u += 4) {
-                const float4 v4 = *reinterpret_cast<const float4 *>(Tf + af_off(t, g + u));
-                f[u] = v4.x; f[u + 1] = v4.y; f[u + 2] = v4.z; f[u + 3] = v4.w;
-            }
-            *reinterpret_cast<uint4 *>(sm + L::TB + swz_off(t, g * 2, 128)) = pack8(f);
-            *reinterpret_cast<uint4 *>(sm + L::TB + swz_off(t, g * 2 + 16, 128)) = pack8(f + 8);
-        }
-        fence_proxy_async_smem();
-        __syncthreads();
-
-        // ---------------------------------------------------------- Khat^T T (M = 128),  PT = P T (M = 64)
-        if (tid == 0) {
-            tc_fence_after();
-            const uint32_t idy = idesc_bf16(128, 64, 1, 1), idp = idesc_bf16(64, 64, 0, 1);
-#pragma unroll
-            for (int ks = 0; ks < 4; ++ks) {
-                const uint64_t bt = smem_desc(sbase + L::TB + ks * 2048, 8192, 1024, kSw128);
-                umma_bf16(tmem + L::TM_Y, smem_desc(sbase + L::KT + ks * 2048, 8192, 1024, kSw128), bt, idy, ks > 0);
-                umma_bf16(tmem + L::TM_PT, smem_desc(sbase + L::PO + ks * 32, 16, 1024, kSw128), bt, idp, ks > 0);
-            }
-            umma_commit(bar_mma);
-        }
-        ok = mma_done();
-    }
-
-    if (ok) {
-        {   // Y row i, K chunks [4*wh, +4) -> KH and the record;  PT (M = 64: row 16*wq + l
-            // in TMEM lane 32*wq + l) -> KT and the record.  No-swizzle K-major tiles.
-            float v[32], p[32];
-            tmem_ld32(tmem + lane_base + L::TM_Y + wh * 32, v);
-            tmem_ld32(tmem + lane_base + L::TM_PT + wh * 32, p);
-            tmem_ld_wait();
-            const int i = wq * 32 + lane, t = wq * 16 + lane;
-            const float ecr = dec[i];
-#pragma unroll
-            for (int u = 0; u < 32; ++u) v[u] *= ecr;
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                const int c = wh * 4 + q;
-                const uint4 y = pack8(v + 8 * q);
-                *reinterpret_cast<uint4 *>(sm + L::KH + kchunk_off(c, i, 128)) = y;
-                *reinterpret_cast<uint4 *>(rec + R::Y + kchunk_off(c, i, 128)) = y;
-                if (lane < 16) {
-                    const uint4 pt = pack8(p + 8 * q);
-                    *reinterpret_cast<uint4 *>(sm + L::KT + kchunk_off(c, t, 64)) = pt;
-                    *reinterpret_cast<uint4 *>(rec + R::PT + kchunk_off(c, t, 64)) = pt;
-                }
-            }
-        }
-        tc_fence_before();
-        fence_proxy_async_smem();
-        __syncthreads();
-
-        // ---------------------------------------------------------- G = Y Ehat (M = 128),  PW = PT Ehat (M = 64)
-        if (tid == 0) {
-            tc_fence_after();
-            const uint32_t idg = idesc_bf16(128, kDK, 0, 1), idw = idesc_bf16(64, kDK, 0, 1);
-#pragma unroll
-            for (int ks = 0; ks < 4; ++ks) {
-                const uint64_t be = smem_desc(sbase + L::EQ + ks * 2048, 16384, 1024, kSw128);
-                umma_bf16(tmem + L::TM_G, smem_desc(sbase + L::KH + ks * 4096, 2048, 128, kSwNone), be, idg, ks > 0);
-                umma_bf16(tmem + L::TM_PW, smem_desc(sbase + L::KT + ks * 2048, 1024, 128, kSwNone), be, idw, ks > 0);
-            }
-            umma_commit(bar_mma);
-        }
-        ok = mma_done();
-    }
-
-    if (ok) {
-        const float *er = dec + kDK;
-        {   // NG = -G Diag(e^{Gamma_r}): row i, K chunks [8*wh, +8) -> the record
-            const int i = wq * 32 + lane;
-            float v[64];
-            tmem_ld32(tmem + lane_base + L::TM_G + wh * 64, *reinterpret_cast<float(*)[32]>(v));
-            tmem_ld32(tmem + lane_base + L::TM_G + wh * 64 + 32, *reinterpret_cast<float(*)[32]>(v + 32));
-            tmem_ld_wait();
-#pragma unroll
-            for (int s8 = 0; s8 < 64; s8 += 8) {
-                const int j = wh * 64 + s8;
-                const float4 e0 = *reinterpret_cast<const float4 *>(er + j);
-                const float4 e1 = *reinterpret_cast<const float4 *>(er + j + 4);
-                float f[8] = {-v[s8] * e0.x,     -v[s8 + 1] * e0.y, -v[s8 + 2] * e0.z, -v[s8 + 3] * e0.w,
-                              -v[s8 + 4] * e1.x, -v[s8 + 5] * e1.y, -v[s8 + 6] * e1.z, -v[s8 + 7] * e1.w};
-                *reinterpret_cast<uint4 *>(rec + R::NG + kchunk_off(j >> 3, i, 128)) = pack8(f);
-            }
-        }
-        {   // QS = (Qhat - PT Ehat) Diag(e^{Gamma_r}) -> the record (M = 64 accumulator)
-            const int t = wq * 16 + lane;
-#pragma unroll
-            for (int part = 0; part < 64; part += 32) {
-                float v[32];
-                tmem_ld32_wait(tmem + lane_base + L::TM_PW + wh * 64 + part, v);
-                if (lane < 16) {
-#pragma unroll
-                    for (int s8 = 0; s8 < 32; s8 += 8) {
-                        const int j = wh * 64 + part + s8;
-                        const uint4 *qp = reinterpret_cast<const uint4 *>(sm + L::EQ + wh * 16384 + 8192 +
-                                                                          swz_off(t, (part + s8) * 2, 128));
-                        float qh[8], f[8];
-                        unpack8(*qp, qh);
-                        const float4 e0 = *reinterpret_cast<const float4 *>(er + j);
-                        const float4 e1 = *reinterpret_cast<const float4 *>(er + j + 4);
-                        const float ev[8] = {e0.x, e0.y, e0.z, e0.w, e1.x, e1.y, e1.z, e1.w};
-#pragma unroll
-                        for (int u = 0; u < 8; ++u) f[u] = (qh[u] - v[s8 + u]) * ev[u];
-                        *reinterpret_cast<uint4 *>(rec + R::QS + kchunk_off(j >> 3, t, 64)) = pack8(f);
-                    }
-                }
-            }
-        }
-    }
+    uint32_t mma_phase = 0;
+    prep_chunk<DV>(sm, tmem, tid, 0, bar_tma, 0, bar_mma, mma_phase, vg, wg, rec, Tlen, H, t0, h, bi, err);
     tc_fence_before();
     __syncthreads();
     if (warp == 0) {

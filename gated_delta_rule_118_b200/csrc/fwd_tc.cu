@@ -237,6 +237,39 @@ cudaError_t run_fwd_tc_overlapped(const FwdArgs &a, const FwdTcPlan &p, uint8_t 
     return e;
 }
 
+// The persistent launch (fwd_persist.cu) for shapes whose chains leave most
+// SMs free; returns false (nothing enqueued) when the device cannot hold the
+// cooperative grid, so that the windowed schedule runs instead.
+bool try_fwd_persist(const FwdArgs &a, cudaMemPool_t pool, cudaError_t *status)
+{
+    const PersistPlan p = plan_fwd_persist(a.B, a.T, a.H, a.dv, a.num_sms);
+    if (!p.use) return false;
+    CUtensorMap maps[4];
+    const auto BF = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+    if (!make_map(&maps[0], a.q, BF, 2, 128, a.H, a.T, a.B, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map(&maps[1], a.k, BF, 2, 128, a.H, a.T, a.B, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map(&maps[2], a.b, BF, 2, 128, a.H, a.T, a.B, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map(&maps[3], a.log_alpha, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, 128, a.H, a.T, a.B, 128,
+                  CU_TENSOR_MAP_SWIZZLE_NONE)) {
+        *status = cudaErrorInvalidValue;
+        return true;
+    }
+    void *ws = nullptr;
+    cudaError_t e = cudaMallocFromPoolAsync(&ws, p.ws_bytes, pool, a.stream);
+    if (e != cudaSuccess) {
+        *status = e;
+        return true;
+    }
+    e = launch_persist(a, maps, static_cast<uint8_t *>(ws), p);
+    const cudaError_t f = cudaFreeAsync(ws, a.stream);
+    if (e == cudaErrorCooperativeLaunchTooLarge) {
+        (void)cudaGetLastError();
+        return false;
+    }
+    *status = e != cudaSuccess ? e : f;
+    return true;
+}
+
 }  // namespace
 
 cudaError_t launch_fwd_tc(const FwdArgs &a)
@@ -247,6 +280,7 @@ cudaError_t launch_fwd_tc(const FwdArgs &a)
     cudaMemPool_t pool = workspace_pool(dev);
     StreamSet *ss = stream_set(dev);
     if (!pool || !ss) return cudaErrorMemoryAllocation;
+    if (try_fwd_persist(a, pool, &e)) return e;
     const FwdTcPlan p = plan_fwd_tc(a.B, a.T, a.H, a.dv, 0, a.num_sms);
     const size_t bytes = p.ws_bytes;
     void *ws = nullptr;

@@ -160,7 +160,9 @@ extern "C" int gdn2_fwd_chunked_launches(int B, int T, int H, int dk, int dv, gd
             sms = 0;
             cudaGetLastError();
         }
-        return 3 * plan_fwd_tc(B, T, H, dv, kWindowBudgetBytes, sms > 0 ? sms : 148).nwindows;
+        if (sms <= 0) sms = 148;
+        if (plan_fwd_persist(B, T, H, dv, sms).use) return 1;
+        return 3 * plan_fwd_tc(B, T, H, dv, kWindowBudgetBytes, sms).nwindows;
     }
     return 1;
 }

@@ -74,6 +74,25 @@ cudaError_t launch_chain(const FwdArgs &a, int dvt, const uint8_t *ws, uint8_t *
                          float *S_out, int ncw, int WC, bool overlap);
 cudaError_t launch_out(const FwdArgs &a, const uint8_t *ws, const uint8_t *sx, int c0, int ncw, int WC,
                        bool overlap);
+// Persistent forward (fwd_persist.cu): prep, chain and output work in one
+// cooperative launch of one CTA per SM, records and state images in rings of
+// kRing chunks per (batch, head); the outputs of chunk c are handed out after
+// the prep of chunk c + kLag (kLag < kRing).
+// A prep takes about as long as a dozen chain steps, so prep runs that far ahead
+// of the chain; outputs are handed out kLag chunks behind it, when they can run.
+constexpr int kRing = 24;
+constexpr int kLag = 16;
+struct PersistPlan {
+    bool use;           // the shape suits the persistent launch
+    int nchain;         // chain CTAs (the others are workers)
+    int grid;           // CTAs (one per SM)
+    size_t rec_total;   // record rings
+    size_t sx_total;    // state-image rings
+    size_t flag_bytes;  // flags and counters (zeroed before the launch)
+    size_t ws_bytes;    // total workspace
+};
+PersistPlan plan_fwd_persist(int B, int T, int H, int dv, int num_sms);
+cudaError_t launch_persist(const FwdArgs &a, const CUtensorMap *maps, uint8_t *ws, const PersistPlan &p);
 // Raise a kernel's dynamic shared-memory limit on the current device, once per
 // device (bit d of `done` records device d).
 template <typename Kernel>

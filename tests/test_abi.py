@@ -36,8 +36,12 @@ def test_library_is_built_for_sm100a(lib):
 
 
 def test_launch_count_query(lib):
-    assert g.gdn2_fwd_chunked_launches(1, 4096, 16, 128, 128) % 3 == 0
-    assert g.gdn2_fwd_chunked_launches(1, 4096, 16, 128, 128) >= 3
+    # one persistent launch where the chains take at most a quarter of the SMs
+    # (16 heads x 2 value tiles of 64 of 148), else three per window of chunks
+    assert g.gdn2_fwd_chunked_launches(1, 4096, 16, 128, 128) == 1
+    assert g.gdn2_fwd_chunked_launches(1, 65536, 16, 128, 128) == 1
+    assert g.gdn2_fwd_chunked_launches(8, 4096, 16, 128, 128) % 3 == 0
+    assert g.gdn2_fwd_chunked_launches(8, 4096, 16, 128, 128) >= 3
     assert g.gdn2_fwd_chunked_launches(1, 256, 2, 64, 64, __import__("torch").float32) == 1
     assert g.gdn2_fwd_chunked_launches(1, 0, 2, 128, 128) == 0
     assert g.gdn2_fwd_chunked_launches(0, 10, 2, 128, 128) == -1

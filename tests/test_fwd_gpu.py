@@ -91,6 +91,31 @@ def test_full_size_sampled_pairs(case, pairs):
         assert eo <= TOL_BF16 and es <= TOL_BF16, (case.name, bi, h, eo, es)
 
 
+# The bf16 forward has two schedules: one persistent launch whose chain CTAs
+# (batch * heads * dv / 64) take at most a quarter of the SMs, with records in
+# rings of 16 chunks per head, and windows of three launches otherwise.
+SCHEDULES = [
+    # B, T, H, dv, pairs checked, what it covers
+    (1, 2600, 3, 128, None, "persistent, rings wrap twice, ragged tail"),
+    (1, 1500, 2, 64, None, "persistent, dv = 64 (one chain CTA per head)"),
+    (2, 700, 12, 128, [(0, 0), (1, 11)], "windows beside the chain (24 heads)"),
+]
+
+
+@pytest.mark.parametrize("B,T,H,dv,pairs,what", SCHEDULES, ids=[c[5] for c in SCHEDULES])
+def test_schedules(B, T, H, dv, pairs, what):
+    d = synth.draw_fwd(B, T, H, 128, dv, seed=31 + T, dtype=torch.bfloat16, s0_sigma=0.02)
+    o, st = run_gpu(d)
+    if pairs is None:
+        o_ref, s_ref = oracle_ref(d)
+        assert rel_err(o, o_ref) <= TOL_BF16 and rel_err(st, s_ref) <= TOL_BF16, what
+        return
+    for (bi, h), (o_ref, s_ref) in zip(pairs, oracle_ref(d, pairs)):
+        eo = rel_err(o[bi:bi + 1, :, h:h + 1], o_ref)
+        es = rel_err(st[bi:bi + 1, h:h + 1], s_ref)
+        assert eo <= TOL_BF16 and es <= TOL_BF16, (what, bi, h, eo, es)
+
+
 def test_state_in_place_and_optional_outputs():
     d = synth.draw_fwd(2, 150, 2, 128, 128, seed=7, dtype=torch.bfloat16, s0_sigma=0.05)
     o_ref, s_ref = oracle_ref(d)
