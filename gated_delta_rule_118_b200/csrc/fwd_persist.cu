@@ -124,6 +124,7 @@ struct Item {
 
 __device__ __forceinline__ Item decode_item(int n, int P, int bh)
 {
+    if (n < 0) return {-1, 0, 0};  // no item (the abort flag was up)
     const int lag = min(kLag, P);
     const int head = lag * bh;
     if (n < head) return {0, n / bh, n % bh};
@@ -189,42 +190,48 @@ persist_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         }
     } else {
         // ---------------------------------------------------------------- worker
-        const int half = tid >> 8, lt = tid & 255, bar_id = 2 + half;
+        const int half = tid >> 8, lt = tid & 255, bar_id = 2 + half, bcast_id = 4 + half;
         uint8_t *hs = sm + half * kHalf;
         uint64_t *hb = reinterpret_cast<uint64_t *>(hs + kHalfData);
         volatile int *item_slot = reinterpret_cast<volatile int *>(hs + kHalfData + 64);
         const uint32_t ht = tmem + (uint32_t)(half * 256);
         uint32_t tma_phase = 0, mma_phase = 0, out_phase = 0;
         for (;;) {
-            if (lt == 0) item_slot[0] = *reinterpret_cast<volatile uint32_t *>(abort) ? -1 : (int)atomicAdd(next, 1u);
-            named_bar(bar_id, 256);
-            const Item it = decode_item(item_slot[0], P, bh);
-            if (it.kind < 0) break;
-            const int c = it.c, r = it.r, h = r % H, bi = r / H, slot = c % kRing;
-            uint8_t *rec = recs + ((long)r * kRing + slot) * Record<DV>::BYTES;
+            // Warp 1 takes the next item, checks its dependencies (one flag per
+            // lane) and issues its loads while warp 0 may still be releasing the
+            // last item (a GPU-scope fence); warp 0 joins at the barrier after.
+            if (lt == 32) item_slot[0] = *reinterpret_cast<volatile uint32_t *>(abort) ? -1 : (int)atomicAdd(next, 1u);
+            if (lt >= 32) named_bar(bcast_id, 224);
             bool ok = true;
-            if (lt == 0) {
-                // dependencies (see the top of this file)
+            if (lt >= 32 && lt < 64) {
+                const Item it = decode_item(item_slot[0], P, bh);
+                const int c = it.c, r = it.r, slot = c % kRing, lane = lt - 32;
+                const uint32_t *fp = nullptr;
+                uint32_t target = 0;
                 if (it.kind == 0) {
-                    if (c >= kRing) {
-                        ok = wait_flag(out_gen + r * kRing + slot, (uint32_t)(c / kRing), abort, err);
-                        for (int t = 0; t < NT && ok; ++t)
-                            ok = wait_flag(prog + r * NT + t, (uint32_t)(c - kRing + 2), abort, err);
-                    }
-                } else {
-                    ok = wait_flag(rec_gen + r * kRing + slot, (uint32_t)(c / kRing + 1), abort, err);
-                    for (int t = 0; t < NT && ok; ++t) ok = wait_flag(prog + r * NT + t, (uint32_t)(c + 1), abort, err);
+                    if (c >= kRing && lane == 0) fp = out_gen + r * kRing + slot, target = (uint32_t)(c / kRing);
+                    if (c >= kRing && lane >= 1 && lane <= NT) fp = prog + r * NT + lane - 1, target = (uint32_t)(c - kRing + 2);
+                } else if (it.kind == 1) {
+                    if (lane == 0) fp = rec_gen + r * kRing + slot, target = (uint32_t)(c / kRing + 1);
+                    if (lane >= 1 && lane <= NT) fp = prog + r * NT + lane - 1, target = (uint32_t)(c + 1);
                 }
-                fence_proxy_async_global();
-                if (ok) {
-                    if (it.kind == 0)
-                        prep::prep_issue_loads(hs, hb, &tm_q, &tm_k, &tm_b, &tm_la, c * kChunk, h, bi);
-                    else
-                        outp::out_issue_loads<DV>(hs, hb + 2, rec,
-                                                  sxs + ((long)r * kRing + slot) * SxSlot<DV>::BYTES);
+                ok = __all_sync(0xffffffffu, fp == nullptr || wait_flag(fp, target, abort, err)) != 0;
+                if (lane == 0 && it.kind >= 0) {
+                    fence_proxy_async_global();
+                    if (ok) {
+                        if (it.kind == 0)
+                            prep::prep_issue_loads(hs, hb, &tm_q, &tm_k, &tm_b, &tm_la, c * kChunk, r % H, r / H);
+                        else
+                            outp::out_issue_loads<DV>(hs, hb + 2, recs + ((long)r * kRing + slot) * Record<DV>::BYTES,
+                                                      sxs + ((long)r * kRing + slot) * SxSlot<DV>::BYTES);
+                    }
                 }
             }
-            if (!named_bar_and(bar_id, 256, ok)) break;
+            ok = named_bar_and(bar_id, 256, ok);
+            const Item it = decode_item(item_slot[0], P, bh);
+            if (it.kind < 0 || !ok) break;
+            const int c = it.c, r = it.r, h = r % H, bi = r / H, slot = c % kRing;
+            uint8_t *rec = recs + ((long)r * kRing + slot) * Record<DV>::BYTES;
             uint64_t *ld_bar = it.kind == 0 ? hb : hb + 2;
             const uint32_t ld_phase = it.kind == 0 ? tma_phase : out_phase;
             if (it.kind == 0) {
@@ -243,7 +250,6 @@ persist_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             ok = named_bar_and(bar_id, 256, ok);
             if (lt == 0) {
                 if (ok) {
-                    __threadfence();
                     st_release_gpu((it.kind == 0 ? rec_gen : out_gen) + r * kRing + slot, (uint32_t)(c / kRing + 1));
                 } else {
                     atomicExch(abort, 1u);
