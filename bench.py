@@ -38,16 +38,10 @@ N_INPUT_SETS = 4  # rotating input sets: 4 x 136 MB > 126 MB of L2
 
 # dram__bytes_read.sum + dram__bytes_write.sum per launch from an ncu capture of
 # the current kernels (None once a kernel has changed since the capture).  The
-# forward is three kernels per window (profiles/*_layer_bf16.md hold each one);
-# decode: profiles/decode_kernel_decode_b256.md.
-# DRAM bytes per launch from ncu captures (profiles/): the decode kernel, and one
-# forward call summed over its prep, chain and output launches, each scaled from
-# one captured window (14 chunks x 16 heads) by the chunks it processes.  ncu
-# captures each kernel cold, so the per-chunk records that prep writes and the
-# chain and output kernels read back count as DRAM traffic here.
-NCU_TRAFFIC_BYTES = {"fwd": round((25.769728e6 + 17.152e3) / 224 * 1024 + 15.874560e6 / 14 * 64
-                                  + 16.534016e6 / 224 * 1024),
-                     "decode": 281.078016e6 + 213.638144e6}
+# layer-workload forward is one persistent launch
+# (profiles/persist_kernel_layer_bf16.md); decode:
+# profiles/decode_kernel_decode_b256.md.
+NCU_TRAFFIC_BYTES = {"fwd": 117.755648e6 + 59.421696e6, "decode": 281.078016e6 + 213.638144e6}
 
 
 def peaks():
@@ -186,8 +180,8 @@ def run_profile_case(args):
     torch.cuda.set_device(0)
     dev = torch.device("cuda", 0)
     names = ("q", "k", "v", "b", "w", "log_alpha")
-    if args.profile == "fwd":
-        c = CASE
+    if args.profile in ("fwd", "fwd_train"):
+        c = CASE if args.profile == "fwd" else synth.TRAIN_BF16
         d = synth.draw_fwd_device(c.B, c.T, c.H, c.dk, c.dv, seed=0, device=dev, dtype=c.dtype,
                                   log_alpha_range=c.log_alpha_range, gate_sigma=c.gate_sigma)
         for _ in range(args.warmup + args.steps):
@@ -212,7 +206,7 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--decode-steps", type=int, default=1000)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--profile", choices=["fwd", "decode"], default=None,
+    ap.add_argument("--profile", choices=["fwd", "fwd_train", "decode"], default=None,
                     help="run a few launches of one operator on the bench workload for an ncu "
                          "capture (no timing, no JSON line)")
     args = ap.parse_args()
@@ -367,7 +361,7 @@ def main():
                          "frac": achieved / hbm_peak, "traffic": NCU_TRAFFIC_BYTES["fwd"],
                          "peak_kind": peak_kind, "algorithmic_bytes_per_launch": alg_bytes,
                          "mean_launch_us": mean_launch_ms * 1e3,
-                         "kernel": "gdn2_fwd_chunked (prep + chain + output kernels per window)"},
+                         "kernel": "gdn2_fwd_chunked (one persistent launch: prep, chain and output work)"},
             "decode": {"workload": dc.name, "us_per_step": dec_ms * 1e3, "hbm_gbs": dec_gbs,
                        "frac": dec_gbs / hbm_peak, "peak": hbm_peak,
                        "algorithmic_bytes_per_step": dec_bytes, "steps": args.decode_steps,
