@@ -142,7 +142,6 @@ __device__ __forceinline__ bool prep_chunk(uint8_t *sm, uint32_t tmem, int tid, 
     if (ok) {
         // ---------------------------------------------------------- Gamma and factors (in place)
         const int p = tid & 63, qr = tid >> 6;           // channel pair, token quarter
-        const int kb = p >> 5, cb = (p & 31) * 4;
         float2 lv[16];
 #pragma unroll
         for (int u = 0; u < 16; ++u) lv[u] = *reinterpret_cast<const float2 *>(la + (qr * 16 + u) * kDK + 2 * p);
@@ -172,23 +171,43 @@ __device__ __forceinline__ bool prep_chunk(uint8_t *sm, uint32_t tmem, int tid, 
             dec[kDK + 2 * p + 1] = expf(gr1);
             *reinterpret_cast<float2 *>(rec + R::DEC + 8 * p) = make_float2(e0, e1);
         }
-        uint8_t *eq = sm + L::EQ + kb * 16384, *kt = sm + L::KT + kb * 8192;
+        // x = Gamma_t - Gamma_r of this thread's tokens and channels, over log_alpha
         unsigned int bad = 0;
         const float sh0 = pre0 - gr0, sh1 = pre1 - gr1;
 #pragma unroll
         for (int u = 0; u < 16; ++u) {
-            const int t = qr * 16 + u;
             const float x0 = lv[u].x + sh0, x1 = lv[u].y + sh1;
             bad |= (fabsf(x0) > kMaxHalfChunkLogDecay) | (fabsf(x1) > kMaxHalfChunkLogDecay);
-            const float up0 = ex2_approx(x0 * kLog2e), up1 = ex2_approx(x1 * kLog2e);
-            const float dn0 = ex2_approx(-x0 * kLog2e), dn1 = ex2_approx(-x1 * kLog2e);
-            const uint32_t off = swz_off(t, cb, 128);
-            const float2 kv = ld_bf16x2(kt + off), bv = ld_bf16x2(eq + off), qv = ld_bf16x2(eq + 8192 + off);
-            st_bf16x2(eq + off, up0 * bv.x * kv.x, up1 * bv.y * kv.y);
-            st_bf16x2(eq + 8192 + off, up0 * qv.x, up1 * qv.y);
-            st_bf16x2(kt + off, dn0 * kv.x, dn1 * kv.y);
+            *reinterpret_cast<float2 *>(la + (qr * 16 + u) * kDK + 2 * p) = make_float2(x0, x1);
         }
         if (bad) atomicOr(err, kErrRange);
+        named_bar(bar_id, kPrepThreads);
+        // the factors in place, one 16-byte piece (8 channels of one token) of
+        // each swizzled tile per step: Ehat over b, Qhat over q, Khat over k
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+            const int idx = tid + m * kPrepThreads;
+            const int t = idx >> 4, g = idx & 15, hb = g >> 3;  // token, channel group, 64-channel half tile
+            const uint32_t off = swz_off(t, (g & 7) * 16, 128);
+            uint8_t *ep = sm + L::EQ + hb * 16384 + off, *qp = ep + 8192, *kp = sm + L::KT + hb * 8192 + off;
+            const float4 xa = *reinterpret_cast<const float4 *>(la + t * kDK + 8 * g);
+            const float4 xb = *reinterpret_cast<const float4 *>(la + t * kDK + 8 * g + 4);
+            const float x[8] = {xa.x, xa.y, xa.z, xa.w, xb.x, xb.y, xb.z, xb.w};
+            float kv[8], bv[8], qv[8], fe[8], fq[8], fk[8];
+            unpack8(*reinterpret_cast<const uint4 *>(kp), kv);
+            unpack8(*reinterpret_cast<const uint4 *>(ep), bv);
+            unpack8(*reinterpret_cast<const uint4 *>(qp), qv);
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const float up = ex2_approx(x[u] * kLog2e), dn = ex2_approx(-x[u] * kLog2e);
+                fe[u] = up * bv[u] * kv[u];
+                fq[u] = up * qv[u];
+                fk[u] = dn * kv[u];
+            }
+            *reinterpret_cast<uint4 *>(ep) = pack8(fe);
+            *reinterpret_cast<uint4 *>(qp) = pack8(fq);
+            *reinterpret_cast<uint4 *>(kp) = pack8(fk);
+        }
         fence_proxy_async_smem();
         named_bar(bar_id, kPrepThreads);
 

@@ -26,3 +26,27 @@ def test_wy_model_strong_decay_and_wide_erase():
     o, s = wy_forward(q, k, v, 2 * b, w, la, S0=s0, C=64)
     assert np.abs(o - o_ref).max() <= 1e-11 * np.abs(o_ref).max()
     assert np.abs(s - s_ref).max() <= 1e-11 * np.abs(s_ref).max()
+
+
+@pytest.mark.parametrize("C,T", [(4, 37), (8, 64), (16, 150), (64, 200)])
+def test_pair_composition_matches_oracle(C, T):
+    """Two chunk records composed into one state map (the form the persistent
+    forward's chain steps over) equal the token recurrence; an odd last chunk
+    (T = 37 with C = 4: ten chunks, T = 150 with C = 16: ten, T = 200 with C = 64: four)
+    and a lone pair (T = 64 with C = 8: eight chunks)."""
+    from wy_model import wy_forward_pairs
+    q, k, v, b, w, la, s0 = _inputs(T, 8, 6, seed=300 + C, B=1, H=2)
+    o_ref, s_ref = oracle.fwd(q, k, v, b, w, la, S0=s0)
+    o, s = wy_forward_pairs(q, k, v, b, w, la, S0=s0, C=C)
+    assert np.abs(o - o_ref).max() <= 1e-11 * np.abs(o_ref).max()
+    assert np.abs(s - s_ref).max() <= 1e-11 * np.abs(s_ref).max()
+
+
+def test_pair_composition_odd_chunk_count():
+    """Three chunks: one composed pair and a lone last chunk."""
+    from wy_model import wy_forward_pairs
+    q, k, v, b, w, la, s0 = _inputs(40, 8, 6, seed=401, B=1, H=1)
+    o_ref, s_ref = oracle.fwd(q, k, v, b, w, la, S0=s0)
+    o, s = wy_forward_pairs(q, k, v, b, w, la, S0=s0, C=16)
+    assert np.abs(o - o_ref).max() <= 1e-11 * np.abs(o_ref).max()
+    assert np.abs(s - s_ref).max() <= 1e-11 * np.abs(s_ref).max()

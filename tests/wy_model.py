@@ -76,3 +76,50 @@ def wy_forward(q, k, v, b, w, log_alpha, S0=None, C=64):
                 o[bi, sl, h] = O
             ST[bi, h] = S
     return o, ST
+
+
+def pair_record(r1, r2):
+    """Two consecutive chunk records (gc, NG, QS, Y, PT) composed into one map of
+    the state entering the first chunk.  With A = Diag(gc) + NG the transition of
+    a chunk, S_1 = A_1 S + Y_1 Z_1 and S_2 = A_2 S_1 + Y_2 Z_2 give
+        S_2 = Diag(gc_1 gc_2) S + NG' S + [Y_1' | Y_2] [Z_1; Z_2]
+        NG' = Diag(gc_2) NG_1 + NG_2 Diag(gc_1) + NG_2 NG_1,   Y_1' = Diag(gc_2) Y_1 + NG_2 Y_1
+    and the second chunk's outputs O_2 = QS_2 S_1 + PT_2 Z_2 become
+        O_2 = QS_2' S + PT_21 Z_1 + PT_2 Z_2,   QS_2' = QS_2 Diag(gc_1) + QS_2 NG_1,   PT_21 = QS_2 Y_1.
+    Returns (gc', NG', Y_1', QS_2', PT_21)."""
+    g1, NG1, _, Y1, _ = r1
+    g2, NG2, QS2, _, _ = r2
+    NGp = g2[:, None] * NG1 + NG2 * g1[None, :] + NG2 @ NG1
+    Y1p = g2[:, None] * Y1 + NG2 @ Y1
+    QS2p = QS2 * g1[None, :] + QS2 @ NG1
+    return g1 * g2, NGp, Y1p, QS2p, QS2 @ Y1
+
+
+def wy_forward_pairs(q, k, v, b, w, log_alpha, S0=None, C=64):
+    """wy_forward with the state carried over pairs of chunks (pair_record); an
+    odd last chunk is a step of its own."""
+    q, k, v, b, w, la = (np.asarray(x, dtype=np.float64) for x in (q, k, v, b, w, log_alpha))
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    o = np.zeros((B, T, H, dv))
+    ST = np.zeros((B, H, dk, dv))
+    for bi in range(B):
+        for h in range(H):
+            S = np.zeros((dk, dv)) if S0 is None else np.array(S0[bi, h], dtype=np.float64)
+            chunks = [slice(t0, min(T, t0 + C)) for t0 in range(0, T, C)]
+            for i in range(0, len(chunks), 2):
+                s1 = chunks[i]
+                r1 = chunk_record(q[bi, s1, h], k[bi, s1, h], b[bi, s1, h], la[bi, s1, h], C)
+                Z1 = w[bi, s1, h] * v[bi, s1, h]
+                o[bi, s1, h] = r1[2] @ S + r1[4] @ Z1
+                if i + 1 == len(chunks):
+                    S = r1[0][:, None] * S + r1[1] @ S + r1[3] @ Z1
+                    break
+                s2 = chunks[i + 1]
+                r2 = chunk_record(q[bi, s2, h], k[bi, s2, h], b[bi, s2, h], la[bi, s2, h], C)
+                Z2 = w[bi, s2, h] * v[bi, s2, h]
+                gp, NGp, Y1p, QS2p, PT21 = pair_record(r1, r2)
+                o[bi, s2, h] = QS2p @ S + PT21 @ Z1 + r2[4] @ Z2
+                S = gp[:, None] * S + NGp @ S + Y1p @ Z1 + r2[3] @ Z2
+            ST[bi, h] = S
+    return o, ST
