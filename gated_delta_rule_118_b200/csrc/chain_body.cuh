@@ -58,7 +58,8 @@ constexpr int kChainThreads = 32 * (kStateWarps + 4);
 constexpr int kPublishEvery = 2;  // chunks per progress release (each costs a GPU-scope fence)
 constexpr int kDK = 128;
 
-template <int DV, int DVT>
+// MAX: the dynamic shared memory the CTA has (the ring takes as many stages as fit).
+template <int DV, int DVT, int MAX = 232448>
 struct ChainLayout {
     static constexpr int NB = DVT / 64;                       // 64-column blocks of Z in the tile
     static constexpr int COLS = DVT / (kStateWarps / 4);      // columns per state thread
@@ -71,7 +72,7 @@ struct ChainLayout {
     static constexpr int SRB = DVT * 256;
     static constexpr int DEC_BYTES = kDK * 4;
     static constexpr int bytes(int ns) { return ns * (STAGE + DEC_BYTES) + SRB + 8 * (2 * ns + 5) + 16 + 1024; }
-    static constexpr int NS = bytes(4) <= 232448 ? 4 : bytes(3) <= 232448 ? 3 : 2;
+    static constexpr int NS = bytes(4) <= MAX ? 4 : bytes(3) <= MAX ? 3 : 2;
     static constexpr int SR = NS * STAGE;
     static constexpr int DECR = SR + SRB;
     static constexpr int BAR = DECR + NS * DEC_BYTES;
@@ -80,7 +81,8 @@ struct ChainLayout {
     static constexpr int DATA = SLOT + 16;   // bytes used from the 1024-aligned base
     static constexpr int BYTES = DATA + 1024;
     static constexpr uint32_t TMEM_COLS = 2 * DVT;            // two D buffers
-    static_assert(BYTES <= 232448, "shared memory");
+    static_assert(BYTES <= MAX, "shared memory");
+    static_assert(COLS % 32 == 0, "state columns per thread: whole 32-column tensor-memory loads");
     static_assert(STAGE % 1024 == 0 && SR % 1024 == 0, "swizzle atoms");
 };
 
@@ -247,13 +249,9 @@ __device__ __forceinline__ void chain_run(uint8_t *sm, uint32_t tmem, int tid, c
         // the same 16-byte pieces to the slot (every warp store covers 512
         // contiguous bytes) and count the warp's export.
         auto publish_sx = [&](int cw, bool ok) {
-            uint4 px[COLS / 8];
             uint8_t *sr = sm + L::SR;
 #pragma unroll
-            for (int j = 0; j < COLS; j += 8) {
-                px[j / 8] = pack8(S + j);
-                *reinterpret_cast<uint4 *>(sr + sx_off(i, col0 + j)) = px[j / 8];
-            }
+            for (int j = 0; j < COLS; j += 8) *reinterpret_cast<uint4 *>(sr + sx_off(i, col0 + j)) = pack8(S + j);
             fence_proxy_async_smem();
             tc_fence_before();
             __syncwarp();
@@ -270,7 +268,8 @@ __device__ __forceinline__ void chain_run(uint8_t *sm, uint32_t tmem, int tid, c
                 uint8_t *dst = f.sx_slot(cw);
 #pragma unroll
                 for (int j = 0; j < COLS; j += 8)
-                    *reinterpret_cast<uint4 *>(dst + sx_off(i, tile * DVT + col0 + j)) = px[j / 8];
+                    *reinterpret_cast<uint4 *>(dst + sx_off(i, tile * DVT + col0 + j)) =
+                        *reinterpret_cast<const uint4 *>(sr + sx_off(i, col0 + j));  // this thread's own pieces
                 if (Flow::kPublishes) {
                     __syncwarp();
                     if (lane == 0) smem_add_release(exports, 1);
@@ -288,21 +287,17 @@ __device__ __forceinline__ void chain_run(uint8_t *sm, uint32_t tmem, int tid, c
             ok = ok && mbar_wait(full + s, (cw / NS) & 1, err);
             tc_fence_after();
             const float gc = decr[s * kDK + i];
-            {
-                float d[COLS];
-                const uint32_t da = lane_addr + (uint32_t)((cw & 1) * DVT);
-                if constexpr (COLS % 32 == 0) {
+            __syncwarp();
+            if (lane == 0 && cw + NS < ncw) mbar_arrive(empty + s);
+            // the update in 32-column pieces (one tensor-memory load each)
+            const uint32_t da = lane_addr + (uint32_t)((cw & 1) * DVT);
 #pragma unroll
-                    for (int j = 0; j < COLS; j += 32) tmem_ld32(da + j, *reinterpret_cast<float(*)[32]>(d + j));
-                } else {
-#pragma unroll
-                    for (int j = 0; j < COLS; j += 16) tmem_ld16(da + j, *reinterpret_cast<float(*)[16]>(d + j));
-                }
+            for (int h = 0; h < COLS; h += 32) {
+                float d[32];
+                tmem_ld32(da + h, d);
                 tmem_ld_wait();
-                __syncwarp();
-                if (lane == 0 && cw + NS < ncw) mbar_arrive(empty + s);
 #pragma unroll
-                for (int u = 0; u < COLS; ++u) S[u] = gc * S[u] + d[u];
+                for (int u = 0; u < 32; ++u) S[h + u] = gc * S[h + u] + d[u];
             }
             if (cw + 1 < ncw) ok = publish_sx(cw + 1, ok);
         }

@@ -40,19 +40,24 @@ namespace {
 using namespace sm100;
 
 constexpr int kPersistThreads = 512;
-constexpr int kChainDvt = 64;            // value tile of a chain CTA (fits the 128-register budget)
 constexpr uint64_t kFlagWaitNs = 1000000000ull;
 
 // Shared memory of a persistent CTA (from its 1024-aligned base): two worker
-// regions, each with its mbarriers and item slot at the end, or a chain layout;
-// the tensor-memory address slot after both.
+// regions, each with its mbarriers and item slot at the end, and the workers'
+// tensor-memory address slot after them; or the layout of a chain over a DVT-wide
+// value tile, which keeps its own slot.
 constexpr int kHalfData = align_up(prep::PrepLayout::DATA, 1024);
 constexpr int kHalf = kHalfData + 1024;  // + mbarriers (prep TMA, prep UMMA, output loads, output UMMA), item
 constexpr int kTmemSlot = 2 * kHalf;
-constexpr int kPersistSmem = kTmemSlot + 16 + 1024;
+template <int DV, int DVT>
+constexpr int persist_smem()
+{
+    return chain::ChainLayout<DV, DVT>::BYTES > kTmemSlot + 16 + 1024 ? chain::ChainLayout<DV, DVT>::BYTES
+                                                                         : kTmemSlot + 16 + 1024;
+}
 static_assert(outp::OutLayout<128>::DATA <= kHalfData, "output region");
-static_assert(chain::ChainLayout<128, kChainDvt>::DATA <= kTmemSlot, "chain layout");
-static_assert(kPersistSmem <= 232448, "shared memory");
+static_assert(chain::ChainLayout<128, 128>::NS >= 3 && chain::ChainLayout<128, 64>::NS >= 3, "chain ring depth");
+static_assert(persist_smem<128, 128>() <= 232448, "shared memory");
 
 struct FlagLayout {
     int bh, nt;
@@ -139,7 +144,7 @@ __device__ __forceinline__ Item decode_item(int n, int P, int bh)
     return {-1, 0, 0};
 }
 
-template <int DV>
+template <int DV, int DVT>
 __global__ void __launch_bounds__(kPersistThreads, 1)
 persist_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ CUtensorMap tm_la,
@@ -147,8 +152,8 @@ persist_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                float *S_T, uint8_t *__restrict__ recs, uint8_t *__restrict__ sxs, uint32_t *flags, int B, int T,
                int H, int nchain, unsigned int *err)
 {
-    using CL = chain::ChainLayout<DV, kChainDvt>;
-    constexpr int NT = DV / kChainDvt;
+    using CL = chain::ChainLayout<DV, DVT>;
+    constexpr int NT = DV / DVT;  // chain CTAs per head
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int tid = threadIdx.x, warp = tid >> 5;
@@ -157,11 +162,11 @@ persist_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     const FlagLayout fl{bh, NT};
     uint32_t *rec_gen = flags + fl.rec_gen(), *out_gen = flags + fl.out_gen(), *prog = flags + fl.prog();
     uint32_t *next = flags + fl.next(), *abort = flags + fl.abort();
-    uint32_t *tslot = reinterpret_cast<uint32_t *>(sm + kTmemSlot);
+    uint32_t *tslot = reinterpret_cast<uint32_t *>(sm + (is_chain ? CL::SLOT : kTmemSlot));
     const uint32_t tcols = is_chain ? CL::TMEM_COLS : 512;
 
     if (is_chain) {
-        if (tid == 0) chain::chain_init<DV, kChainDvt>(sm);
+        if (tid == 0) chain::chain_init<DV, DVT>(sm);
     } else if ((tid & 255) == 0) {
         uint64_t *hb = reinterpret_cast<uint64_t *>(sm + (tid >> 8) * kHalf + kHalfData);
         for (int k = 0; k < 4; ++k) mbar_init(hb + k, 1);
@@ -186,7 +191,7 @@ persist_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                                  prog + pair * NT + tile,
                                  abort,
                                  err};
-            chain::chain_run<DV, kChainDvt>(sm, tmem, tid, f, S0, S_T, pair, tile, P, err);
+            chain::chain_run<DV, DVT>(sm, tmem, tid, f, S0, S_T, pair, tile, P, err);
         }
     } else {
         // ---------------------------------------------------------------- worker
@@ -275,7 +280,11 @@ PersistPlan plan_fwd_persist(int B, int T, int H, int dv, int num_sms)
 {
     PersistPlan p{};
     const long bh = (long)B * H;
-    const int nt = dv / kChainDvt;
+    // Value tile of a chain CTA: a 128-wide tile leaves SMs to the workers (long
+    // sequences are worker-bound: B1 H16 T65536 1.49 -> 1.39 ms), a 64-wide one
+    // steps faster (B1 H16 T4096: 121.6 -> 117.6 us).
+    p.dvt = (dv == 128 && T >= kPersistWideT) ? 128 : 64;
+    const int nt = dv / p.dvt;
     p.nchain = (int)(bh * nt);
     // the chain CTAs must leave most SMs to the workers
     p.use = (dv == 64 || dv == 128) && num_sms > 0 && T > 0 && p.nchain * 4 <= num_sms;
@@ -293,15 +302,16 @@ cudaError_t launch_persist(const FwdArgs &a, const CUtensorMap *maps, uint8_t *w
     uint32_t *flags = reinterpret_cast<uint32_t *>(ws + p.rec_total + p.sx_total);
     cudaError_t e = cudaMemsetAsync(flags, 0, p.flag_bytes, a.stream);
     if (e != cudaSuccess) return e;
-    auto kern = a.dv == 128 ? persist_kernel<128> : persist_kernel<64>;
-    static std::atomic<unsigned long long> smem_set[2] = {};
-    e = ensure_smem_limit(kern, kPersistSmem, smem_set[a.dv == 128]);
+    auto kern = a.dv == 64 ? persist_kernel<64, 64> : p.dvt == 128 ? persist_kernel<128, 128> : persist_kernel<128, 64>;
+    const int smem = a.dv == 64 ? persist_smem<64, 64>() : p.dvt == 128 ? persist_smem<128, 128>() : persist_smem<128, 64>();
+    static std::atomic<unsigned long long> smem_set[3] = {};
+    e = ensure_smem_limit(kern, smem, smem_set[a.dv == 64 ? 0 : p.dvt == 128 ? 1 : 2]);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg{};
     cudaLaunchAttribute attr[1];
     cfg.gridDim = dim3(p.grid);
     cfg.blockDim = dim3(kPersistThreads);
-    cfg.dynamicSmemBytes = kPersistSmem;
+    cfg.dynamicSmemBytes = smem;
     cfg.stream = a.stream;
     // every CTA resident at once: the CTAs wait for one another
     attr[0].id = cudaLaunchAttributeCooperative;

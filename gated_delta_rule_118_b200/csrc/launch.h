@@ -82,8 +82,10 @@ cudaError_t launch_out(const FwdArgs &a, const uint8_t *ws, const uint8_t *sx, i
 // of the chain; outputs are handed out kLag chunks behind it, when they can run.
 constexpr int kRing = 24;
 constexpr int kLag = 16;
+constexpr int kPersistWideT = 16384;  // from this sequence length on, 128-wide chain tiles
 struct PersistPlan {
     bool use;           // the shape suits the persistent launch
+    int dvt;            // value tile of a chain CTA
     int nchain;         // chain CTAs (the others are workers)
     int grid;           // CTAs (one per SM)
     size_t rec_total;   // record rings
