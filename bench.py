@@ -41,7 +41,7 @@ N_INPUT_SETS = 4  # rotating input sets: 4 x 136 MB > 126 MB of L2
 # layer-workload forward is one persistent launch
 # (profiles/persist_kernel_layer_bf16.md); decode:
 # profiles/decode_kernel_decode_b256.md.
-NCU_TRAFFIC_BYTES = {"fwd": 117.755648e6 + 59.421696e6, "decode": 281.078016e6 + 213.638144e6}
+NCU_TRAFFIC_BYTES = {"fwd": 117.728e6 + 56.744192e6, "decode": 281.078016e6 + 213.638144e6}
 
 
 def peaks():
