@@ -84,14 +84,6 @@ __device__ __forceinline__ void unpack8(uint4 v, float *f)
     }
 }
 
-__device__ __forceinline__ float2 ld_bf16x2(const uint8_t *p)
-{
-    return __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(p));
-}
-__device__ __forceinline__ void st_bf16x2(uint8_t *p, float a, float b)
-{
-    *reinterpret_cast<__nv_bfloat162 *>(p) = __floats2bfloat162_rn(a, b);
-}
 
 __device__ __forceinline__ float ex2_approx(float x)
 {
