@@ -92,6 +92,16 @@ typedef struct CUstream_st *gdn2_stream_t;
  * channel is split at the chunk midpoint and each half must stay above -80
  * (any log_alpha >= -2.5 satisfies this).  A chunk outside this range sets
  * GDN2_ERR_RANGE in the device error word and its results are not valid.
+ *
+ * Execution (bf16, dk = 128): when the sequences' state chains take at most a
+ * quarter of the SMs (see gdn2_fwd_chunked_launches) the call is one
+ * cooperative kernel with one CTA on every SM, whose CTAs hand work to one
+ * another (each such wait gives up after one second and reports
+ * GDN2_ERR_DEVICE_TIMEOUT); it starts once every SM is free, so kernels of
+ * other streams delay it or wait for it.  If the device cannot hold that grid
+ * the call falls back to the windowed schedule: three kernels per window of
+ * chunks on `stream`, the output kernels on a library-owned side stream that
+ * forks from and joins back into `stream`.
  */
 gdn2_status gdn2_fwd_chunked(const void *q, const void *k, const void *v,
                              const void *b, const void *w, const float *log_alpha,
