@@ -131,16 +131,17 @@ def max_over_ranks(x: float, ws: int) -> float:
     return float(t.item())
 
 
-def cpu_oracle_tokens_per_s(sample_T: int, heads: int):
-    """Oracle (fp64, OpenMP over heads) on a bounded sample of the workload."""
+def cpu_oracle_tokens_per_s(sample_T: int, heads: int, nthreads: int = 0):
+    """Oracle (fp64, OpenMP over heads; nthreads 0 = every host core) on a bounded
+    sample of the workload."""
     import oracle
     d = synth.draw_fwd(1, sample_T, heads, CASE.dk, CASE.dv, seed=CASE.seed, dtype=CASE.dtype,
                        log_alpha_range=CASE.log_alpha_range, gate_sigma=CASE.gate_sigma)
     args = [d[n] for n in ("q", "k", "v", "b", "w", "log_alpha")]
     orc = oracle.load()
-    cores = orc.max_threads()
+    cores = nthreads if nthreads > 0 else orc.max_threads()
     t = time.perf_counter()
-    orc.fwd(*args, S0=None)
+    orc.fwd(*args, S0=None, nthreads=nthreads)
     dt = time.perf_counter() - t
     return sample_T * heads / dt, cores, dt
 
@@ -342,9 +343,13 @@ def main():
     cpu = None
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
         v, cores, dt = cpu_oracle_tokens_per_s(c.T, c.H)
+        v1, _, dt1 = cpu_oracle_tokens_per_s(1024, c.H, nthreads=1)
         cpu = {"value": v, "unit": "tokens/s", "cores": cores, "kind": "oracle",
                "sample": f"the whole workload (B=1 H=16 T=4096 d=128, 65,536 head-tokens), fp64, "
-                         f"{dt:.1f} s"}
+                         f"{dt:.1f} s",
+               "single_core": {"value": v1, "unit": "tokens/s",
+                               "sample": f"the first 1024 tokens of the workload, 16 heads, one thread, "
+                                         f"{dt1:.1f} s"}}
 
     if rank == 0:
         line = {
