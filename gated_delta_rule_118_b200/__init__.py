@@ -31,7 +31,8 @@ GDN2_BF16 = 1
 
 # Every symbol include/gdn2.h declares.
 EXPORTED = ("gdn2_fwd_chunked", "gdn2_fwd_chunked_noalloc", "gdn2_decode_step",
-            "gdn2_check_device_error", "gdn2_fwd_chunked_launches", "gdn2_status_string")
+            "gdn2_check_device_error", "gdn2_selftest_bounded_wait", "gdn2_fwd_chunked_launches",
+            "gdn2_status_string")
 
 _lib = None
 
@@ -59,6 +60,8 @@ def lib() -> ctypes.CDLL:
         L.gdn2_decode_step.restype = ci
         L.gdn2_check_device_error.argtypes = [vp]
         L.gdn2_check_device_error.restype = ci
+        L.gdn2_selftest_bounded_wait.argtypes = [vp]
+        L.gdn2_selftest_bounded_wait.restype = ci
         L.gdn2_fwd_chunked_launches.argtypes = [ci] * 6
         L.gdn2_fwd_chunked_launches.restype = ci
         L.gdn2_status_string.argtypes = [ci]
@@ -154,6 +157,11 @@ def gdn2_decode_step(q, k, v, b, w, log_alpha, S, o=None, *, stream=None, check=
 def gdn2_check_device_error(stream=None) -> int:
     """Synchronise ``stream`` and return (and clear) the device error status."""
     return int(lib().gdn2_check_device_error(_stream(stream)))
+
+
+def gdn2_selftest_bounded_wait(stream=None) -> int:
+    """Queue the bounded-wait self-test (a wait that runs out after one second)."""
+    return int(lib().gdn2_selftest_bounded_wait(_stream(stream)))
 
 
 def gdn2_fwd_chunked_launches(B, T, H, dk, dv, dtype=torch.bfloat16) -> int:

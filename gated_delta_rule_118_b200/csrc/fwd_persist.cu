@@ -86,6 +86,14 @@ __device__ __noinline__ bool wait_flag(const uint32_t *p, uint32_t target, uint3
     return false;
 }
 
+// A flag that nothing sets and its abort word, for the bounded-wait self-test.
+__device__ uint32_t g_selftest_words[2];
+
+__global__ void selftest_wait_kernel(unsigned int *err)
+{
+    if (threadIdx.x == 0) wait_flag(&g_selftest_words[0], 1u, &g_selftest_words[1], err);
+}
+
 // The chain's view of the rings of one (batch, head) and of its own progress counter.
 template <int DV>
 struct RingFlow {
@@ -275,6 +283,16 @@ persist_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
 }
 
 }  // namespace
+
+cudaError_t launch_selftest_wait(cudaStream_t stream, unsigned int *err)
+{
+    void *words = nullptr;
+    cudaError_t e = cudaGetSymbolAddress(&words, g_selftest_words);
+    if (e == cudaSuccess) e = cudaMemsetAsync(words, 0, sizeof(uint32_t) * 2, stream);
+    if (e != cudaSuccess) return e;
+    selftest_wait_kernel<<<1, 32, 0, stream>>>(err);
+    return cudaGetLastError();
+}
 
 PersistPlan plan_fwd_persist(int B, int T, int H, int dv, int num_sms)
 {

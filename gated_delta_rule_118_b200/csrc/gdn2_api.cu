@@ -147,6 +147,15 @@ extern "C" gdn2_status gdn2_check_device_error(gdn2_stream_t stream)
     return GDN2_OK;
 }
 
+extern "C" gdn2_status gdn2_selftest_bounded_wait(gdn2_stream_t stream)
+{
+    unsigned int *err = nullptr;
+    int sms = 0;
+    if (device_context(&err, &sms) != GDN2_OK) return GDN2_ERR_CUDA;
+    return launch_selftest_wait(reinterpret_cast<cudaStream_t>(stream), err) == cudaSuccess ? GDN2_OK
+                                                                                            : GDN2_ERR_CUDA;
+}
+
 extern "C" int gdn2_fwd_chunked_launches(int B, int T, int H, int dk, int dv, gdn2_dtype dtype)
 {
     if ((dtype != GDN2_F32 && dtype != GDN2_BF16) || B <= 0 || H <= 0 || T < 0) return -1;

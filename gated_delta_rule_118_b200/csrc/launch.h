@@ -95,6 +95,8 @@ struct PersistPlan {
 };
 PersistPlan plan_fwd_persist(int B, int T, int H, int dv, int num_sms);
 cudaError_t launch_persist(const FwdArgs &a, const CUtensorMap *maps, uint8_t *ws, const PersistPlan &p);
+// One-warp kernel whose flag wait (the persistent forward's) runs out: kErrTimeout after one second.
+cudaError_t launch_selftest_wait(cudaStream_t stream, unsigned int *err);
 // Raise a kernel's dynamic shared-memory limit on the current device, once per
 // device (bit d of `done` records device d).
 template <typename Kernel>

@@ -181,6 +181,16 @@ gdn2_status gdn2_check_device_error(gdn2_stream_t stream);
  */
 int gdn2_fwd_chunked_launches(int B, int T, int H, int dk, int dv, gdn2_dtype dtype);
 
+/*
+ * gdn2_selftest_bounded_wait -- queue on `stream` a one-warp kernel that waits
+ * for a device flag nothing sets, with the bounded wait the persistent forward
+ * uses between its CTAs.  The wait gives up after one second and records
+ * GDN2_ERR_DEVICE_TIMEOUT in the device error word, so the next
+ * gdn2_check_device_error(stream) returns it, and the context stays usable.
+ * Returns GDN2_OK once queued (GDN2_ERR_CUDA if queuing failed).
+ */
+gdn2_status gdn2_selftest_bounded_wait(gdn2_stream_t stream);
+
 /* Human-readable name of a status code (static storage, never NULL). */
 const char *gdn2_status_string(gdn2_status status);
 

@@ -187,3 +187,19 @@ def test_decay_outside_range_is_reported(dtype):
     assert g.gdn2_check_device_error() == g.GDN2_ERR_RANGE
     g.gdn2_fwd_chunked(*(d[n] for n in names))
     assert g.gdn2_check_device_error() == g.GDN2_OK
+
+
+def test_bounded_wait_gives_up_and_reports():
+    """A device wait on a flag nothing sets gives up after about a second and
+    reports GDN2_ERR_DEVICE_TIMEOUT; the context stays usable (a forward after it
+    runs and reports no error)."""
+    import time
+    assert g.gdn2_selftest_bounded_wait() == g.GDN2_OK
+    t0 = time.perf_counter()
+    assert g.gdn2_check_device_error() == g.GDN2_ERR_DEVICE_TIMEOUT
+    assert 0.5 < time.perf_counter() - t0 < 10.0
+    assert g.gdn2_check_device_error() == g.GDN2_OK  # the word was cleared
+    d = synth.draw_fwd(1, 130, 2, 128, 128, seed=11, dtype=torch.bfloat16, s0_sigma=0.02)
+    o, st = run_gpu(d)
+    o_ref, s_ref = oracle_ref(d)
+    assert rel_err(o, o_ref) <= TOL_BF16 and rel_err(st, s_ref) <= TOL_BF16
