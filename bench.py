@@ -101,17 +101,23 @@ class ClockSampler:
                 "sm_max_mhz": max(mx) if mx else None, "reasons": reasons, "samples": len(rows)}
 
 
-def dist_setup(args):
+def dist_setup(backend="nccl"):
+    """One process per GPU (RANK / WORLD_SIZE / LOCAL_RANK from the launcher); the
+    process group only carries the barrier and the max over ranks (replicas, no
+    data exchange).  `backend` "gloo" runs the same logic on the host."""
     ws = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     if ws > 1:
         import datetime
         import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
-    else:
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                    device_id=torch.device("cuda", local))
+        else:
+            dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    elif backend == "nccl":
         torch.cuda.set_device(0)
     return ws, rank, local
 
@@ -122,11 +128,11 @@ def barrier(ws):
         dist.barrier()
 
 
-def max_over_ranks(x: float, ws: int) -> float:
+def max_over_ranks(x: float, ws: int, device: str = "cuda") -> float:
     if ws == 1:
         return x
     import torch.distributed as dist
-    t = torch.tensor([x], device="cuda", dtype=torch.float64)
+    t = torch.tensor([x], device=device, dtype=torch.float64)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
 
@@ -223,7 +229,7 @@ def main():
     if args.profile:
         run_profile_case(args)
         return
-    ws, rank, local = dist_setup(args)
+    ws, rank, local = dist_setup()
     dev = torch.device("cuda", torch.cuda.current_device())
     stream = torch.cuda.current_stream()
     hbm_peak, peak_kind = peaks()
