@@ -5,22 +5,26 @@
 // (chain_body.cuh) and the outputs of a chunk (out_body.cuh) -- run in one
 // cooperative grid of one CTA per SM, so that every CTA is resident and may
 // wait for another:
-//   * CTAs [0, nchain) each run one chain over the whole sequence;
+//   * CTAs [0, nchain) each run one chain (a 64- or 128-wide value tile of one
+//     (batch, head)) over the whole sequence;
 //   * every other CTA is two independent workers of 256 threads, each with half
 //     of the SM's shared and tensor memory, which take items from one counter
 //     in a fixed order: the prep of chunk c for all heads, then the outputs of
 //     chunk c - kLag for all heads, for c = 0, 1, ...
 // Records and state images live in rings of kRing chunks per (batch, head).
 // Hand-offs go through flags in global memory (release / acquire at GPU scope):
-//   prep(c)   -> rec_gen    : record c is written          (chain, outputs wait)
-//   chain     -> prog       : state images up to c exported (outputs wait for c + 1;
-//                             prep(c + kRing) waits for c + 2, the chain being done
-//                             with record c)
-//   out(c)    -> out_gen    : ring slots of c are read      (prep(c + kRing) and the
-//                             chain's export of c + kRing wait)
-// Every item waits only for items earlier in the order or for chain progress
-// that those items make possible, and kLag < kRing, so the order cannot
-// deadlock.  Every wait is bounded: a wait that gives up raises kErrTimeout and
+//   prep(c)   -> rec_gen    : record c is written
+//                             (the chain's producer and output(c) wait for it)
+//   chain     -> prog = n   : the state images of chunks [0, n) are exported
+//                             (output(c) waits for n > c; prep(c + kRing) waits for
+//                             n > c + 1, the chain being done with record c then)
+//   out(c)    -> out_gen    : the ring slots of chunk c have been read
+//                             (prep(c + kRing) waits for it)
+// The chain exports the state image of chunk c into its slot once its producer
+// has seen record c ready: prep(c) waited for output(c - kRing), the slot's last
+// reader.  Every item waits only for items earlier in the order or for chain
+// progress that those items make possible, and kLag < kRing, so the order
+// cannot deadlock (tests/test_persist_schedule.py replays these rules).  Every wait is bounded: a wait that gives up raises kErrTimeout and
 // an abort flag that ends every other wait, and the CTA leaves once its
 // copies in flight have landed.
 //
