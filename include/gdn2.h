@@ -123,7 +123,7 @@ gdn2_status gdn2_fwd_chunked(const void *q, const void *k, const void *v,
  * the library's device image (held on every GPU that loads the library, until
  * the process exits) and processes the sequence in as many windows as needed
  * to fit it.  A problem whose single chunk of records does not fit (about
- * 193 KiB per (batch, head) pair for dv = 128, so B*H up to 169) returns
+ * 185 KiB per (batch, head) pair for dv = 128, so B*H up to 177) returns
  * GDN2_ERR_SCRATCH_LIMIT and launches nothing.
  *
  * The first call on a device looks the buffer's device address up

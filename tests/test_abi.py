@@ -96,3 +96,12 @@ def test_fwd_rejects_bad_arguments(lib, kw, code):
 ])
 def test_decode_rejects_bad_arguments(lib, kw, code):
     assert dec(lib, **kw) == code
+
+
+def test_noalloc_rejects_pairs_beyond_its_scratch(lib):
+    # One chunk of records and state image plus the carried state take 185 KiB per
+    # (batch, head) pair at dv = 128: 178 pairs exceed the 32 MiB buffer.  (Only
+    # the rejection is checked here: an accepted call would launch.)
+    for B, H in ((1, 178), (2, 89), (178, 1)):
+        st = lib.gdn2_fwd_chunked_noalloc(P, P, P, P, P, P, None, P, None, B, 64, H, 128, 128, 1, None)
+        assert st == g.GDN2_ERR_SCRATCH_LIMIT, (B, H)
