@@ -235,7 +235,51 @@ def pin_batch_head_independence(orc):
             _close(st[bi:bi + 1, h:h + 1], ss, 0.0, f"pair ({bi},{h}) S_T")
 
 
+# ---------------------------------------------------------------------------
+# 12. Orthonormal keys (alpha = 1, b = w = 1, S_0 = 0): each write lands in a
+#     direction no earlier key reads, so nothing is erased; querying an earlier
+#     key returns its value, a later key returns zero, and S_T = sum_i k_i v_i^T.
+def pin_orthonormal_keys(orc):
+    dk, dv = 6, 4
+    r = _rng(121)
+    K = np.linalg.qr(r.standard_normal((dk, dk)))[0].T          # rows: orthonormal keys
+    v = r.standard_normal((1, dk, 1, dv))
+    k = K.reshape(1, dk, 1, dk)
+    q = np.empty_like(k)
+    for t in range(dk):
+        q[0, t, 0] = K[(t * 5 + 2) % dk]                         # a key written before, at t, or later
+    one_k, one_v = np.ones((1, dk, 1, dk)), np.ones((1, dk, 1, dv))
+    o, st = orc.fwd(q, k, v, one_k, one_v, np.zeros((1, dk, 1, dk)), S0=None)
+    for t in range(dk):
+        j = (t * 5 + 2) % dk
+        _close(o[0, t, 0], v[0, j, 0] if j <= t else np.zeros(dv), 1e-13, f"orthonormal keys o[{t}]")
+    _close(st[0, 0], K.T @ v[0, :, 0], 1e-13, "orthonormal keys S_T")
+
+
+# ---------------------------------------------------------------------------
+# 13. One basis key e_i, erase gate beta on channel i, write gate omega, decay
+#     alpha_i: x_t = S_t^T e_i obeys x_t = alpha_i (1 - beta) x_{t-1} + omega v,
+#     so x_t = omega v (1 - rho^t) / (1 - rho) with rho = alpha_i (1 - beta).  The
+#     decay acts before the erase reads, the erase uses b and the write uses w.
+def pin_gated_geometric(orc):
+    T, dk, dv, i = 12, 5, 3, 2
+    beta, omega, alpha = 0.3, 0.7, 0.9
+    r = _rng(131)
+    vv = r.standard_normal(dv)
+    k = np.zeros((1, T, 1, dk)); k[..., i] = 1.0
+    b = np.full((1, T, 1, dk), 0.55); b[..., i] = beta          # other channels' gates never act
+    w = np.full((1, T, 1, dv), omega)
+    la = np.full((1, T, 1, dk), np.log(0.5)); la[..., i] = np.log(alpha)
+    v = np.broadcast_to(vv, (1, T, 1, dv)).copy()
+    o, st = orc.fwd(k, k, v, b, w, la, S0=None)
+    rho = alpha * (1.0 - beta)
+    for t in range(T):
+        _close(o[0, t, 0], omega * vv * (1.0 - rho ** (t + 1)) / (1.0 - rho), 1e-13, f"gated geometric o[{t}]")
+    want = np.zeros((dk, dv)); want[i] = omega * vv * (1.0 - rho ** T) / (1.0 - rho)
+    _close(st[0, 0], want, 1e-13, "gated geometric S_T")
+
+
 ALL_PINS = [pin_scalar_hand, pin_reduces_to_kda, pin_reduces_to_gated_deltanet,
             pin_reduces_to_deltanet, pin_exact_recall, pin_pure_decay, pin_product_form,
             pin_linearity, pin_column_permutation, pin_sequence_split,
-            pin_batch_head_independence]
+            pin_batch_head_independence, pin_orthonormal_keys, pin_gated_geometric]
