@@ -10,12 +10,17 @@ namespace gdn2 {
 // Bits of the device-side error word (read and cleared by gdn2_check_device_error).
 enum : unsigned int {
     kErrTimeout = 1u,  // a bounded wait gave up
-    kErrRange = 2u,    // a chunk's cumulative decay left the factored range
 };
 
-// Largest |Gamma_t - Gamma_ref| (natural log units) for which the split
-// factors exp(+x) and exp(-x) both stay normal fp32 numbers with margin.
-constexpr float kMaxHalfChunkLogDecay = 80.0f;
+// The chunk kernels fold the decay into split factors e^{+x} and e^{-x},
+// x = Gamma_t - Gamma_r, around a reference Gamma_r inside the chunk.  They
+// use that fast form while every |x| of the chunk stays within this range, in
+// which both factors are normal fp32 (and bf16) numbers with margin; a chunk
+// whose decay is stronger takes a bounded form whose factors are all decays
+// (<= 1).  The fp32 path uses a tighter range: the rounding of x (about
+// |x| * 2^-24 per cumulated term) must stay far below its 1e-4 tolerance.
+constexpr float kMidpointLogDecayRange = 80.0f;
+constexpr float kMidpointLogDecayRangeF32 = 24.0f;
 
 constexpr int kChunk = 64;  // tokens per chunk
 

@@ -12,6 +12,10 @@
 //   A = strict_lower(Ehat Khat^T), P = lower(Qhat Khat^T), Sref = e^{Gamma_r} S,
 //   (I + A) U = Z - Ehat Sref,     O = Qhat Sref + P U,
 //   S <- e^{Gamma_C} S + Ktil^T U.
+// A chunk whose decay is too strong for the midpoint split (some
+// |Gamma_t - Gamma_r| above kMidpointLogDecayRangeF32) uses the reference 0
+// instead (Qbar = e^{Gamma} q, Ebar = e^{Gamma} b k, Sref = S) and forms A and P
+// from running products of alpha, so that every factor is a decay (<= 1).
 // One CTA owns one (batch, head, 32-column value tile); value columns of the
 // state are independent because the erase and the decay act on key rows.
 #include "common.cuh"
@@ -96,53 +100,130 @@ fwd_simt_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__res
         __syncthreads();
 
         // ---- Gamma: inclusive cumulative log-decay per key channel, fp32 ----
+        // The midpoint form is used while every |Gamma_t - Gamma_r| of the chunk
+        // stays within kMidpointLogDecayRangeF32; otherwise (strong decay, or
+        // log_alpha = -inf) the chunk takes the bounded form below.
         const int rmid = min(C / 2, Lc);  // reference token count (midpoint)
+        bool far = false;
         for (int i = tid; i < DK; i += kSimtThreads) {
             float g = 0.f, gr = 0.f;
             for (int t = 0; t < C; ++t) {
                 g += sG[t * LDK + i];
-                sG[t * LDK + i] = g;
                 if (t == rmid - 1) gr = g;
+            }
+            float h = 0.f;
+            for (int t = 0; t < C; ++t) {
+                h += sG[t * LDK + i];
+                far |= !(fabsf(h - gr) <= kMidpointLogDecayRangeF32);
             }
             sGr[i] = gr;
             sGc[i] = g;
         }
-        __syncthreads();
+        const bool exact = __syncthreads_or(far) != 0;
 
-        // ---- decay-absorbed factors; Sref = e^{Gamma_r} S ----
-        unsigned int bad = 0;
-        for (int idx = tid; idx < C * DK; idx += kSimtThreads) {
-            const int t = idx / DK, i = idx % DK;
-            const float g = sG[t * LDK + i];
-            const float x = g - sGr[i];
-            bad |= (fabsf(x) > kMaxHalfChunkLogDecay);
-            const float up = expf(x), dn = expf(-x), tl = expf(sGc[i] - g);
-            const float kv = sK[t * LDK + i];
-            sQ[t * LDK + i] *= up;
-            sE[t * LDK + i] *= up * kv;
-            sK[t * LDK + i] = dn * kv;
-            sG[t * LDK + i] = tl * kv;
-        }
-        if (bad) atomicOr(err, kErrRange);
-        for (int idx = tid; idx < DK * DVT; idx += kSimtThreads)
-            sR[idx] = expf(sGr[idx / DVT]) * sS[idx];
-        __syncthreads();
-
-        // ---- A = strict_lower(Ehat Khat^T), P = lower(Qhat Khat^T) ----
-        for (int idx = tid; idx < C * C; idx += kSimtThreads) {
-            const int t = idx / C, s = idx % C;
-            float a = 0.f, p = 0.f;
-            if (s <= t) {
-                const float *e = sE + t * LDK, *qq = sQ + t * LDK, *kk = sK + s * LDK;
-#pragma unroll 8
-                for (int i = 0; i < DK; ++i) {
-                    a += e[i] * kk[i];
-                    p += qq[i] * kk[i];
+        if (!exact) {
+            for (int i = tid; i < DK; i += kSimtThreads) {
+                float g = 0.f;
+                for (int t = 0; t < C; ++t) {
+                    g += sG[t * LDK + i];
+                    sG[t * LDK + i] = g;
                 }
             }
-            sA[t * LDC + s] = (s < t) ? a : 0.f;
-            sP[t * LDC + s] = p;
+            __syncthreads();
+            // ---- decay-absorbed factors; Sref = e^{Gamma_r} S ----
+            for (int idx = tid; idx < C * DK; idx += kSimtThreads) {
+                const int t = idx / DK, i = idx % DK;
+                const float g = sG[t * LDK + i];
+                const float x = g - sGr[i];
+                const float up = expf(x), dn = expf(-x), tl = expf(sGc[i] - g);
+                const float kv = sK[t * LDK + i];
+                sQ[t * LDK + i] *= up;
+                sE[t * LDK + i] *= up * kv;
+                sK[t * LDK + i] = dn * kv;
+                sG[t * LDK + i] = tl * kv;
+            }
+            for (int idx = tid; idx < DK * DVT; idx += kSimtThreads)
+                sR[idx] = expf(sGr[idx / DVT]) * sS[idx];
+            __syncthreads();
+
+            // ---- A = strict_lower(Ehat Khat^T), P = lower(Qhat Khat^T) ----
+            for (int idx = tid; idx < C * C; idx += kSimtThreads) {
+                const int t = idx / C, s = idx % C;
+                float a = 0.f, p = 0.f;
+                if (s <= t) {
+                    const float *e = sE + t * LDK, *qq = sQ + t * LDK, *kk = sK + s * LDK;
+#pragma unroll 8
+                    for (int i = 0; i < DK; ++i) {
+                        a += e[i] * kk[i];
+                        p += qq[i] * kk[i];
+                    }
+                }
+                sA[t * LDC + s] = (s < t) ? a : 0.f;
+                sP[t * LDC + s] = p;
+            }
+        } else {
+            // ---- bounded form: every factor is a decay over a stretch of the chunk ----
+            //   A_ts = sum_i b_ti k_ti k_si f_tsi,  P_ts = sum_i q_ti k_si f_tsi,
+            //   f_tsi = e^{Gamma_ti - Gamma_si} = prod_{s < u <= t} alpha_ui (running products),
+            // then Qbar = e^{Gamma} q and Ebar = e^{Gamma} b k (decayed from the chunk
+            // start, Sref = S) and Ktil = e^{Gamma_C - Gamma} k from suffix sums.
+            for (int idx = tid; idx < DK * DVT; idx += kSimtThreads) sR[idx] = sS[idx];
+            {
+                constexpr int CPT = DK / 4;  // channels per thread; 4 lanes per token
+                const int t = tid >> 2, cq = tid & 3, i0 = cq * CPT;
+                const int tmax = (tid >> 5) * 8 + 7;  // the warp's largest token: every lane shuffles
+                float qv[CPT], ev[CPT], f[CPT];
+#pragma unroll
+                for (int j = 0; j < CPT; ++j) {
+                    qv[j] = sQ[t * LDK + i0 + j];
+                    ev[j] = sE[t * LDK + i0 + j] * sK[t * LDK + i0 + j];
+                    f[j] = 1.f;
+                }
+                for (int s = tmax; s >= 0; --s) {
+                    const bool on = s <= t;
+                    float pa = 0.f, aa = 0.f;
+                    if (on) {
+#pragma unroll
+                        for (int j = 0; j < CPT; ++j) {
+                            const float a = f[j] * sK[s * LDK + i0 + j];
+                            pa = fmaf(qv[j], a, pa);
+                            aa = fmaf(ev[j], a, aa);
+                            f[j] *= __expf(sG[s * LDK + i0 + j]);
+                        }
+                    }
+                    pa += __shfl_xor_sync(0xffffffffu, pa, 1);
+                    aa += __shfl_xor_sync(0xffffffffu, aa, 1);
+                    pa += __shfl_xor_sync(0xffffffffu, pa, 2);
+                    aa += __shfl_xor_sync(0xffffffffu, aa, 2);
+                    if (cq == 0) {
+                        sP[t * LDC + s] = on ? pa : 0.f;
+                        sA[t * LDC + s] = (s < t) ? aa : 0.f;
+                    }
+                }
+                if (cq == 0)
+                    for (int s = tmax + 1; s < C; ++s) {
+                        sP[t * LDC + s] = 0.f;
+                        sA[t * LDC + s] = 0.f;
+                    }
+            }
+            __syncthreads();
+            for (int i = tid; i < DK; i += kSimtThreads) {
+                float g = 0.f;
+                for (int t = 0; t < C; ++t) {
+                    g += sG[t * LDK + i];
+                    const float e = expf(g);
+                    sQ[t * LDK + i] *= e;
+                    sE[t * LDK + i] *= e * sK[t * LDK + i];
+                }
+                float suf = 0.f;
+                for (int t = C - 1; t >= 0; --t) {
+                    const float l = sG[t * LDK + i];
+                    sG[t * LDK + i] = expf(suf) * sK[t * LDK + i];
+                    suf += l;
+                }
+            }
         }
+        __syncthreads();
         // ---- right-hand side Z - Ehat Sref (in place in sU) ----
         for (int idx = tid; idx < C * DVT; idx += kSimtThreads) {
             const int t = idx / DVT, j = idx % DVT;

@@ -11,7 +11,7 @@
 
 namespace gdn2 {
 
-// Device-side error word: kernels OR bits into it (kErrTimeout, kErrRange);
+// Device-side error word: kernels OR bits into it (kErrTimeout);
 // gdn2_check_device_error() reads and clears it.  One per device (module global).
 __device__ unsigned int g_device_error = 0;
 
@@ -143,7 +143,6 @@ extern "C" gdn2_status gdn2_check_device_error(gdn2_stream_t stream)
         return GDN2_ERR_CUDA;
     if (word && cudaMemset(err, 0, sizeof(word)) != cudaSuccess) return GDN2_ERR_CUDA;
     if (word & kErrTimeout) return GDN2_ERR_DEVICE_TIMEOUT;
-    if (word & kErrRange) return GDN2_ERR_RANGE;
     return GDN2_OK;
 }
 
@@ -187,7 +186,7 @@ extern "C" const char *gdn2_status_string(gdn2_status status)
     case GDN2_ERR_UNSUPPORTED: return "GDN2_ERR_UNSUPPORTED: request outside the implemented set";
     case GDN2_ERR_CUDA: return "GDN2_ERR_CUDA: a CUDA runtime call or launch failed";
     case GDN2_ERR_DEVICE_TIMEOUT: return "GDN2_ERR_DEVICE_TIMEOUT: a device-side bounded wait gave up";
-    case GDN2_ERR_RANGE: return "GDN2_ERR_RANGE: a chunk's cumulative decay left the factored range";
+    case GDN2_ERR_RANGE: return "GDN2_ERR_RANGE: reserved (no longer reported)";
     case GDN2_ERR_SCRATCH_LIMIT: return "GDN2_ERR_SCRATCH_LIMIT: the problem needs more than the fixed scratch buffer";
     }
     return "GDN2 unknown status";

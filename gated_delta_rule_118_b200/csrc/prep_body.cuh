@@ -51,7 +51,8 @@ struct PrepLayout {
     static constexpr int LA = 65536;      // log_alpha -> fp32 A | fp32 T -> bf16 T over A
     static constexpr int PO = 98304;      // Gamma quarter totals -> P
     static constexpr int DEC = 106496;    // e^{Gamma_C-Gamma_r}[128], e^{Gamma_r}[128]
-    static constexpr int DATA = 107520;   // end of the buffers above
+    static constexpr int QP = 107520;     // bounded path: product of alpha per token quarter [4][128]
+    static constexpr int DATA = 109568;   // end of the buffers above
     static constexpr int BAR = DATA;      // the windowed kernel's mbarriers and TMEM slot
     static constexpr int SLOT = BAR + 16;
     static constexpr int BYTES = SLOT + 16 + 1024;
@@ -109,6 +110,7 @@ __device__ __forceinline__ bool prep_chunk(uint8_t *sm, uint32_t tmem, int tid, 
     float *Xs = reinterpret_cast<float *>(sm + L::XS);
     float *dec = reinterpret_cast<float *>(sm + L::DEC);
     float *tot = reinterpret_cast<float *>(sm + L::TOT);
+    float *qprod = reinterpret_cast<float *>(sm + L::QP);
     const uint32_t sbase = smem_u32(sm);
     const uint32_t lane_base = (uint32_t)(wq * 32) << 16;
     // v and w for Z = w v: plain vector loads, issued before anything waits
@@ -139,8 +141,25 @@ __device__ __forceinline__ bool prep_chunk(uint8_t *sm, uint32_t tmem, int tid, 
     };
     bool ok = named_bar_and(bar_id, kPrepThreads, (tid == 0) ? mbar_wait(bar_tma, tma_phase, err) : true) != 0;
 
+    // Z = w v, straight into the record (MN-major operand blocks of 64 value
+    // columns; each warp fills whole 128-byte rows)
+    auto write_z = [&]() {
+#pragma unroll
+        for (int m = 0; m < ZV; ++m) {
+            const int idx = tid + m * kPrepThreads;
+            const int t = idx / (DV / 8), j = (idx % (DV / 8)) * 8;
+            float fv[8], fw[8], fz[8];
+            unpack8(vv[m], fv);
+            unpack8(wv[m], fw);
+#pragma unroll
+            for (int u = 0; u < 8; ++u) fz[u] = fv[u] * fw[u];
+            *reinterpret_cast<uint4 *>(rec + R::Z + (j >> 6) * 8192 + swz_off(t, (j & 63) * 2, 128)) = pack8(fz);
+        }
+    };
+    bool exact = false;  // this chunk's decay is too strong for the midpoint reference
+
     if (ok) {
-        // ---------------------------------------------------------- Gamma and factors (in place)
+        // ---------------------------------------------------------- Gamma
         const int p = tid & 63, qr = tid >> 6;           // channel pair, token quarter
         float2 lv[16];
 #pragma unroll
@@ -163,85 +182,216 @@ __device__ __forceinline__ bool prep_chunk(uint8_t *sm, uint32_t tmem, int tid, 
         }
         // midpoint reference: Gamma after 32 tokens (tokens past T carry log_alpha = 0)
         const float gr0 = tot[2 * p] + tot[kDK + 2 * p], gr1 = tot[2 * p + 1] + tot[kDK + 2 * p + 1];
-        if (qr == 0) {
-            const float e0 = expf(gc0), e1 = expf(gc1);
-            dec[2 * p] = expf(gc0 - gr0);
-            dec[2 * p + 1] = expf(gc1 - gr1);
-            dec[kDK + 2 * p] = expf(gr0);
-            dec[kDK + 2 * p + 1] = expf(gr1);
-            *reinterpret_cast<float2 *>(rec + R::DEC + 8 * p) = make_float2(e0, e1);
-        }
-        // x = Gamma_t - Gamma_r of this thread's tokens and channels, over log_alpha
-        unsigned int bad = 0;
+        // x = Gamma_t - Gamma_r of this thread's tokens and channels.  The split
+        // factors e^{+x} and e^{-x} stay finite fp32/bf16 numbers for |x| <= 80;
+        // a chunk where some |x| is larger (or not a number: log_alpha = -inf)
+        // takes the bounded path below instead.
         const float sh0 = pre0 - gr0, sh1 = pre1 - gr1;
+        bool far = false;
 #pragma unroll
-        for (int u = 0; u < 16; ++u) {
-            const float x0 = lv[u].x + sh0, x1 = lv[u].y + sh1;
-            bad |= (fabsf(x0) > kMaxHalfChunkLogDecay) | (fabsf(x1) > kMaxHalfChunkLogDecay);
-            *reinterpret_cast<float2 *>(la + (qr * 16 + u) * kDK + 2 * p) = make_float2(x0, x1);
-        }
-        if (bad) atomicOr(err, kErrRange);
-        named_bar(bar_id, kPrepThreads);
-        // the factors in place, one 16-byte piece (8 channels of one token) of
-        // each swizzled tile per step: Ehat over b, Qhat over q, Khat over k
-#pragma unroll
-        for (int m = 0; m < 4; ++m) {
-            const int idx = tid + m * kPrepThreads;
-            const int t = idx >> 4, g = idx & 15, hb = g >> 3;  // token, channel group, 64-channel half tile
-            const uint32_t off = swz_off(t, (g & 7) * 16, 128);
-            uint8_t *ep = sm + L::EQ + hb * 16384 + off, *qp = ep + 8192, *kp = sm + L::KT + hb * 8192 + off;
-            const float4 xa = *reinterpret_cast<const float4 *>(la + t * kDK + 8 * g);
-            const float4 xb = *reinterpret_cast<const float4 *>(la + t * kDK + 8 * g + 4);
-            const float x[8] = {xa.x, xa.y, xa.z, xa.w, xb.x, xb.y, xb.z, xb.w};
-            float kv[8], bv[8], qv[8], fe[8], fq[8], fk[8];
-            unpack8(*reinterpret_cast<const uint4 *>(kp), kv);
-            unpack8(*reinterpret_cast<const uint4 *>(ep), bv);
-            unpack8(*reinterpret_cast<const uint4 *>(qp), qv);
-#pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                const float up = ex2_approx(x[u] * kLog2e), dn = ex2_approx(-x[u] * kLog2e);
-                fe[u] = up * bv[u] * kv[u];
-                fq[u] = up * qv[u];
-                fk[u] = dn * kv[u];
-            }
-            *reinterpret_cast<uint4 *>(ep) = pack8(fe);
-            *reinterpret_cast<uint4 *>(qp) = pack8(fq);
-            *reinterpret_cast<uint4 *>(kp) = pack8(fk);
-        }
-        fence_proxy_async_smem();
-        named_bar(bar_id, kPrepThreads);
+        for (int u = 0; u < 16; ++u)
+            far |= !(fabsf(lv[u].x + sh0) <= kMidpointLogDecayRange) | !(fabsf(lv[u].y + sh1) <= kMidpointLogDecayRange);
+        exact = !named_bar_and(bar_id, kPrepThreads, !far);
+        if (qr == 0)
+            *reinterpret_cast<float2 *>(rec + R::DEC + 8 * p) = make_float2(expf(gc0), expf(gc1));
 
-        // ---------------------------------------------------------- Gram: [Ehat;Qhat] Khat^T
-        if (tid == 0) {
-            tc_fence_after();
-            const uint32_t id = idesc_bf16(128, 64, 0, 0);
-#pragma unroll
-            for (int ks = 0; ks < kDK / 16; ++ks) {
-                const uint32_t kofs = (ks & 3) * 32;
-                umma_bf16(tmem + L::TM_G, smem_desc(sbase + L::EQ + (ks >> 2) * 16384 + kofs, 16, 1024, kSw128),
-                          smem_desc(sbase + L::KT + (ks >> 2) * 8192 + kofs, 16, 1024, kSw128), id, ks > 0);
+        if (!exact) {
+            // ------------------------------------------------------ midpoint factors (in place)
+            if (qr == 0) {
+                dec[2 * p] = expf(gc0 - gr0);
+                dec[2 * p + 1] = expf(gc1 - gr1);
+                dec[kDK + 2 * p] = expf(gr0);
+                dec[kDK + 2 * p + 1] = expf(gr1);
             }
-            umma_commit(bar_mma);
-        }
-        // Z = w v while the Gram runs, straight into the record (MN-major operand
-        // blocks of 64 value columns; each warp fills whole 128-byte rows)
 #pragma unroll
-        for (int m = 0; m < ZV; ++m) {
-            const int idx = tid + m * kPrepThreads;
-            const int t = idx / (DV / 8), j = (idx % (DV / 8)) * 8;
-            float fv[8], fw[8], fz[8];
-            unpack8(vv[m], fv);
-            unpack8(wv[m], fw);
+            for (int u = 0; u < 16; ++u)
+                *reinterpret_cast<float2 *>(la + (qr * 16 + u) * kDK + 2 * p) =
+                    make_float2(lv[u].x + sh0, lv[u].y + sh1);
+            named_bar(bar_id, kPrepThreads);
+            // one 16-byte piece (8 channels of one token) of each swizzled tile per
+            // step: Ehat over b, Qhat over q, Khat over k
 #pragma unroll
-            for (int u = 0; u < 8; ++u) fz[u] = fv[u] * fw[u];
-            *reinterpret_cast<uint4 *>(rec + R::Z + (j >> 6) * 8192 + swz_off(t, (j & 63) * 2, 128)) = pack8(fz);
+            for (int m = 0; m < 4; ++m) {
+                const int idx = tid + m * kPrepThreads;
+                const int t = idx >> 4, g = idx & 15, hb = g >> 3;  // token, channel group, 64-channel half tile
+                const uint32_t off = swz_off(t, (g & 7) * 16, 128);
+                uint8_t *ep = sm + L::EQ + hb * 16384 + off, *qp = ep + 8192, *kp = sm + L::KT + hb * 8192 + off;
+                const float4 xa = *reinterpret_cast<const float4 *>(la + t * kDK + 8 * g);
+                const float4 xb = *reinterpret_cast<const float4 *>(la + t * kDK + 8 * g + 4);
+                const float x[8] = {xa.x, xa.y, xa.z, xa.w, xb.x, xb.y, xb.z, xb.w};
+                float kv[8], bv[8], qv[8], fe[8], fq[8], fk[8];
+                unpack8(*reinterpret_cast<const uint4 *>(kp), kv);
+                unpack8(*reinterpret_cast<const uint4 *>(ep), bv);
+                unpack8(*reinterpret_cast<const uint4 *>(qp), qv);
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    const float up = ex2_approx(x[u] * kLog2e), dn = ex2_approx(-x[u] * kLog2e);
+                    fe[u] = up * bv[u] * kv[u];
+                    fq[u] = up * qv[u];
+                    fk[u] = dn * kv[u];
+                }
+                *reinterpret_cast<uint4 *>(ep) = pack8(fe);
+                *reinterpret_cast<uint4 *>(qp) = pack8(fq);
+                *reinterpret_cast<uint4 *>(kp) = pack8(fk);
+            }
+            fence_proxy_async_smem();
+            named_bar(bar_id, kPrepThreads);
+
+            // ------------------------------------------------------ Gram: [Ehat;Qhat] Khat^T
+            if (tid == 0) {
+                tc_fence_after();
+                const uint32_t id = idesc_bf16(128, 64, 0, 0);
+#pragma unroll
+                for (int ks = 0; ks < kDK / 16; ++ks) {
+                    const uint32_t kofs = (ks & 3) * 32;
+                    umma_bf16(tmem + L::TM_G, smem_desc(sbase + L::EQ + (ks >> 2) * 16384 + kofs, 16, 1024, kSw128),
+                              smem_desc(sbase + L::KT + (ks >> 2) * 8192 + kofs, 16, 1024, kSw128), id, ks > 0);
+                }
+                umma_commit(bar_mma);
+            }
+            write_z();  // while the Gram runs
+            ok = mma_done();
+        } else {
+            // ------------------------------------------------------ bounded path
+            // Every factor is a decay over a stretch of the chunk, never the
+            // inverse of one, so nothing can overflow and what underflows is
+            // negligible:
+            //   A_ts = sum_j b_tj k_tj k_sj f_tsj,  P_ts = sum_j q_tj k_sj f_tsj,
+            //   f_tsj = e^{Gamma_tj - Gamma_sj} = prod_{s < u <= t} alpha_uj (running products),
+            //   Ebar = e^{Gamma} b k, Qbar = e^{Gamma} q (decayed from the chunk start),
+            //   Ktil = e^{Gamma_C - Gamma} k (decayed to the chunk end),
+            // and the record's scalings by e^{Gamma_C - Gamma_r} and e^{Gamma_r} become 1.
+            float *Ak = reinterpret_cast<float *>(sm + L::KH);  // A, fp32 (the solve's scratch is free)
+            if (qr == 0) {
+                dec[2 * p] = 1.f;
+                dec[2 * p + 1] = 1.f;
+                dec[kDK + 2 * p] = 1.f;
+                dec[kDK + 2 * p + 1] = 1.f;
+            }
+            // alpha over log_alpha, and each quarter's product of alpha per channel
+            {
+                float q0 = 1.f, q1 = 1.f;
+#pragma unroll
+                for (int u = 0; u < 16; ++u) {
+                    float2 *lp = reinterpret_cast<float2 *>(la + (qr * 16 + u) * kDK + 2 * p);
+                    const float2 l = *lp;
+                    const float2 a = make_float2(ex2_approx(l.x * kLog2e), ex2_approx(l.y * kLog2e));
+                    *lp = a;
+                    q0 *= a.x; q1 *= a.y;
+                }
+                *reinterpret_cast<float2 *>(qprod + qr * kDK + 2 * p) = make_float2(q0, q1);
+            }
+#pragma unroll
+            for (int m = 0; m < 4; ++m) reinterpret_cast<float4 *>(Ak)[tid + m * kPrepThreads] = make_float4(0.f, 0.f, 0.f, 0.f);
+            reinterpret_cast<float4 *>(sm + L::PO)[tid] = make_float4(0.f, 0.f, 0.f, 0.f);
+            reinterpret_cast<float4 *>(sm + L::PO)[tid + kPrepThreads] = make_float4(0.f, 0.f, 0.f, 0.f);
+            write_z();
+            named_bar(bar_id, kPrepThreads);
+            {
+                // thread: token pair (pr, 63 - pr), 16 channels; the 8 lanes of a token reduce by shuffles
+                const int pr = tid >> 3, cg = tid & 7, hb = cg >> 2, cb = (cg & 3) * 32;
+                const uint8_t *bt = sm + L::EQ + hb * 16384, *qt = bt + 8192, *kt = sm + L::KT + hb * 8192;
+                const float *al = la + 16 * cg;
+#pragma unroll 1
+                for (int pass = 0; pass < 2; ++pass) {
+                    // the lanes of a warp hold 4 tokens; the loop runs to the warp's
+                    // largest token so that every lane takes part in the shuffles
+                    const int t = pass ? 63 - pr : pr, tmax = pass ? 63 - 4 * warp : 4 * warp + 3;
+                    float qv[16], ev[16], f[16];
+                    unpack8(*reinterpret_cast<const uint4 *>(qt + swz_off(t, cb, 128)), qv);
+                    unpack8(*reinterpret_cast<const uint4 *>(qt + swz_off(t, cb + 16, 128)), qv + 8);
+                    unpack8(*reinterpret_cast<const uint4 *>(bt + swz_off(t, cb, 128)), ev);
+                    unpack8(*reinterpret_cast<const uint4 *>(bt + swz_off(t, cb + 16, 128)), ev + 8);
+                    unpack8(*reinterpret_cast<const uint4 *>(kt + swz_off(t, cb, 128)), f);
+                    unpack8(*reinterpret_cast<const uint4 *>(kt + swz_off(t, cb + 16, 128)), f + 8);
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) {
+                        ev[j] *= f[j];
+                        f[j] = 1.f;
+                    }
+#pragma unroll 1
+                    for (int s = tmax; s >= 0; --s) {
+                        const bool on = s <= t;
+                        float pa = 0.f, aa = 0.f;
+                        if (on) {
+                            float kv[16];
+                            unpack8(*reinterpret_cast<const uint4 *>(kt + swz_off(s, cb, 128)), kv);
+                            unpack8(*reinterpret_cast<const uint4 *>(kt + swz_off(s, cb + 16, 128)), kv + 8);
+#pragma unroll
+                            for (int j = 0; j < 16; ++j) {
+                                const float a = f[j] * kv[j];
+                                pa = fmaf(qv[j], a, pa);
+                                aa = fmaf(ev[j], a, aa);
+                            }
+#pragma unroll
+                            for (int j = 0; j < 16; j += 4) {
+                                const float4 a4 = *reinterpret_cast<const float4 *>(al + s * kDK + j);
+                                f[j] *= a4.x; f[j + 1] *= a4.y; f[j + 2] *= a4.z; f[j + 3] *= a4.w;
+                            }
+                        }
+#pragma unroll
+                        for (int o = 1; o < 8; o <<= 1) {
+                            pa += __shfl_xor_sync(0xffffffffu, pa, o);
+                            aa += __shfl_xor_sync(0xffffffffu, aa, o);
+                        }
+                        if (cg == 0 && on) {
+                            *reinterpret_cast<bf16 *>(sm + L::PO + swz_off(t, 2 * s, 128)) = __float2bfloat16_rn(pa);
+                            if (s < t) Ak[af_off(t, s)] = aa;
+                        }
+                    }
+                }
+            }
+            named_bar(bar_id, kPrepThreads);
+            // the bounded factors over the raw tiles (two channels of 16 tokens per
+            // thread), from running products of alpha: e^{Gamma_t} = prod_{u <= t} alpha_u,
+            // e^{Gamma_C - Gamma_t} = prod_{u > t} alpha_u
+            {
+                float pre0 = 1.f, pre1 = 1.f, post0 = 1.f, post1 = 1.f;
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const float2 a = *reinterpret_cast<const float2 *>(qprod + q * kDK + 2 * p);
+                    if (q < qr) { pre0 *= a.x; pre1 *= a.y; }
+                    if (q > qr) { post0 *= a.x; post1 *= a.y; }
+                }
+                float2 sf[16];
+#pragma unroll
+                for (int u = 15; u >= 0; --u) {
+                    sf[u] = make_float2(post0, post1);
+                    const float2 a = *reinterpret_cast<const float2 *>(la + (qr * 16 + u) * kDK + 2 * p);
+                    post0 *= a.x; post1 *= a.y;
+                }
+                const int hb = p >> 5;
+                const int cbyte = (2 * p & 63) * 2;
+#pragma unroll
+                for (int u = 0; u < 16; ++u) {
+                    const int t = qr * 16 + u;
+                    const float2 a = *reinterpret_cast<const float2 *>(la + t * kDK + 2 * p);
+                    pre0 *= a.x; pre1 *= a.y;
+                    const uint32_t off = swz_off(t, cbyte, 128);
+                    __nv_bfloat162 *ep = reinterpret_cast<__nv_bfloat162 *>(sm + L::EQ + hb * 16384 + off);
+                    __nv_bfloat162 *qp = reinterpret_cast<__nv_bfloat162 *>(sm + L::EQ + hb * 16384 + 8192 + off);
+                    __nv_bfloat162 *kp = reinterpret_cast<__nv_bfloat162 *>(sm + L::KT + hb * 8192 + off);
+                    const float2 bv = __bfloat1622float2(*ep), qv = __bfloat1622float2(*qp), kv = __bfloat1622float2(*kp);
+                    *ep = __floats2bfloat162_rn(pre0 * bv.x * kv.x, pre1 * bv.y * kv.y);
+                    *qp = __floats2bfloat162_rn(pre0 * qv.x, pre1 * qv.y);
+                    *kp = __floats2bfloat162_rn(sf[u].x * kv.x, sf[u].y * kv.y);
+                }
+            }
+            named_bar(bar_id, kPrepThreads);  // every thread has read alpha
+            // A into the solve's place, T starts as zero
+#pragma unroll
+            for (int m = 0; m < 4; ++m) {
+                const int idx = tid + m * kPrepThreads;
+                reinterpret_cast<float4 *>(Af)[idx] = reinterpret_cast<const float4 *>(Ak)[idx];
+                reinterpret_cast<float4 *>(Tf)[idx] = make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+            named_bar(bar_id, kPrepThreads);
         }
-        ok = mma_done();
     }
 
     if (ok) {
-        // ---------------------------------------------------------- A (fp32) and P (bf16)
-        {
+        if (!exact) {
+            // ------------------------------------------------------ A (fp32) and P (bf16) from the Gram
             const int r = wq * 32 + lane;
             float v[32];
             tmem_ld32_wait(tmem + lane_base + L::TM_GRAM + wh * 32, v);
@@ -271,9 +421,9 @@ __device__ __forceinline__ bool prep_chunk(uint8_t *sm, uint32_t tmem, int tid, 
 #pragma unroll
             for (int m = 0; m < 4; ++m)
                 reinterpret_cast<float4 *>(Tf)[tid + m * kPrepThreads] = make_float4(0.f, 0.f, 0.f, 0.f);
+            tc_fence_before();
+            named_bar(bar_id, kPrepThreads);
         }
-        tc_fence_before();
-        named_bar(bar_id, kPrepThreads);
 
         // ---------------------------------------------------------- T = (I + A)^{-1}
         // (a) diagonal 16x16 blocks: one column per thread, rows of A read as float4

@@ -33,9 +33,9 @@
  *   - Every pointer must be 16-byte aligned.
  *   - Supported head sizes: dk and dv each 64 or 128.
  *   - The returned status covers argument checks and launch errors only.
- *     Conditions found while the kernels run (a bounded wait that gave up, a
- *     decay outside the supported range) are recorded in a device-side error
- *     word and reported by gdn2_check_device_error().
+ *     A condition found while the kernels run (a bounded wait that gave up) is
+ *     recorded in a device-side error word and reported by
+ *     gdn2_check_device_error().
  *   - Gates are used as given: values outside [0, 1] (the pages' ablation
  *     widens the erase range to [0, 2]) are not clamped.
  */
@@ -55,7 +55,7 @@ typedef enum gdn2_status {
     GDN2_ERR_UNSUPPORTED = 5,    /* valid request outside the implemented set         */
     GDN2_ERR_CUDA = 6,           /* a CUDA runtime call or launch failed              */
     GDN2_ERR_DEVICE_TIMEOUT = 7, /* a device-side bounded wait gave up                */
-    GDN2_ERR_RANGE = 8,          /* a chunk's cumulative decay left the factored range */
+    GDN2_ERR_RANGE = 8,          /* reserved: no longer reported (every decay is computed) */
     GDN2_ERR_SCRATCH_LIMIT = 9   /* needs more than gdn2_fwd_chunked_noalloc's fixed buffer */
 } gdn2_status;
 
@@ -88,10 +88,12 @@ typedef struct CUstream_st *gdn2_stream_t;
  *                                      May alias S0 (in-place advance).
  *   B, H >= 1; T >= 0 (T = 0 only copies S0, or zeros, into S_T).
  *
- * Range: inside each 64-token chunk the cumulative log-decay of every key
- * channel is split at the chunk midpoint and each half must stay above -80
- * (any log_alpha >= -2.5 satisfies this).  A chunk outside this range sets
- * GDN2_ERR_RANGE in the device error word and its results are not valid.
+ * Decay: any log_alpha <= 0 is accepted, -inf included (alpha = 0: the
+ * channel forgets everything before that token).  A chunk whose cumulative
+ * decay is mild splits it into growing and shrinking factors around the chunk
+ * midpoint; a chunk where that split would leave the fp32 range (strong
+ * decay, e.g. log_alpha below about -2.5 held for 32 tokens) is computed in a
+ * form whose factors are all decays, at a higher cost for that chunk.
  *
  * Execution (bf16, dk = 128): when the sequences' state chains take at most a
  * quarter of the SMs (see gdn2_fwd_chunked_launches) the call is one
@@ -128,9 +130,11 @@ gdn2_status gdn2_fwd_chunked(const void *q, const void *k, const void *v,
  *
  * The first call on a device looks the buffer's device address up
  * (cudaGetSymbolAddress) with that device current; make that first call
- * before any stream capture.  All calls share the one buffer: calls whose
- * work overlaps on the GPU (different streams, or devices sharing nothing but
- * this buffer's name) race and corrupt each other's results; serialize them.
+ * before any stream capture.  All calls on one device share that device's
+ * buffer: calls whose work overlaps on the GPU (for instance on two streams of
+ * the same device) race and corrupt each other's results, so serialize them.
+ * Each device has its own copy of the buffer; calls on different devices do
+ * not share it.
  * Every byte of the buffer that a call reads, that call writes first, so its
  * leftover contents from earlier calls do not matter.
  */
@@ -163,7 +167,7 @@ gdn2_status gdn2_decode_step(const void *q, const void *k, const void *v,
 /*
  * gdn2_check_device_error -- wait for `stream`, then read and clear the
  * device error word of the current device.  Returns GDN2_OK,
- * GDN2_ERR_DEVICE_TIMEOUT, GDN2_ERR_RANGE or GDN2_ERR_CUDA.
+ * GDN2_ERR_DEVICE_TIMEOUT or GDN2_ERR_CUDA.
  */
 gdn2_status gdn2_check_device_error(gdn2_stream_t stream);
 

@@ -138,3 +138,31 @@ def draw_fwd_device(B, T, H, dk, dv, *, seed, device, dtype=torch.bfloat16,
     out = {n: t.to(dtype).contiguous() for n, t in dict(q=q, k=k, v=v, b=b, w=w).items()}
     out["log_alpha"] = (-torch.exp(u)).contiguous()
     return out
+
+
+# Decay distributions beyond the workloads' own, for the edge of the method
+# where alpha approaches 0 (fast-forgetting channels):
+#   "wide":   log_alpha = -exp(U(-1, 3)), i.e. from about -0.37 down to about -20 per token;
+#   "all3":   every channel at -3 per token;
+#   "mixed":  per (head, channel) either -20 (forgets within a token) or -1e-4 (keeps);
+#   "zeros":  the workload distribution, with alpha = 0 exactly (log_alpha = -inf)
+#             at a random 2% of (token, channel) entries.
+DECAY_KINDS = ("wide", "all3", "mixed", "zeros")
+
+
+def draw_log_alpha(B, T, H, dk, kind, *, seed):
+    """log_alpha [B,T,H,dk] (fp32) of one of the DECAY_KINDS distributions."""
+    g = torch.Generator(device="cpu").manual_seed(int(seed))
+    if kind == "wide":
+        return (-torch.exp(torch.rand(B, T, H, dk, generator=g) * 4.0 - 1.0)).contiguous()
+    if kind == "all3":
+        return torch.full((B, T, H, dk), -3.0)
+    if kind == "mixed":
+        fast = torch.rand(1, 1, H, dk, generator=g) < 0.5
+        la = torch.where(fast, torch.tensor(-20.0), torch.tensor(-1e-4))
+        return la.expand(B, T, H, dk).contiguous()
+    if kind == "zeros":
+        la = -torch.exp(torch.rand(B, T, H, dk, generator=g) * 4.0 - 5.0)
+        la[torch.rand(B, T, H, dk, generator=g) < 0.02] = float("-inf")
+        return la.contiguous()
+    raise ValueError(kind)

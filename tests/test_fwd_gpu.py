@@ -72,23 +72,19 @@ def test_small_shapes_elementwise(B, T, H, dk, dv, dtype, s0):
     assert rel_err(st, s_ref) <= tol(dtype)
 
 
-FULL = [
-    (synth.LAYER_BF16, [(0, 0), (0, 7), (0, 15)]),
-    (synth.TRAIN_BF16, [(0, 0), (3, 5), (7, 15)]),
-    (synth.LONG_BF16, [(0, 0), (0, 9)]),
-]
+FULL = [synth.LAYER_BF16, synth.TRAIN_BF16, synth.LONG_BF16]
 
 
-@pytest.mark.parametrize("case,pairs", FULL, ids=[c.name for c, _ in FULL])
-def test_full_size_sampled_pairs(case, pairs):
-    """Full-size launch; sampled (batch, head) pairs against the oracle, all outputs finite."""
+@pytest.mark.parametrize("case", FULL, ids=[c.name for c in FULL])
+def test_full_size_every_element(case):
+    """The three bf16 workloads at full size, in the launch configuration the
+    benchmark times: every output and every final-state element against the
+    oracle (which runs all (batch, head) pairs on the host's cores)."""
     d = synth.draw_case(case)
     o, st = run_gpu(d)
-    assert torch.isfinite(o).all() and torch.isfinite(st).all()
-    for (bi, h), (o_ref, s_ref) in zip(pairs, oracle_ref(d, pairs)):
-        eo = rel_err(o[bi:bi + 1, :, h:h + 1], o_ref)
-        es = rel_err(st[bi:bi + 1, h:h + 1], s_ref)
-        assert eo <= TOL_BF16 and es <= TOL_BF16, (case.name, bi, h, eo, es)
+    o_ref, s_ref = oracle_ref(d)
+    eo, es = rel_err(o, o_ref), rel_err(st, s_ref)
+    assert eo <= TOL_BF16 and es <= TOL_BF16, (case.name, eo, es)
 
 
 # The bf16 forward has two schedules: one persistent launch whose chain CTAs
@@ -175,18 +171,6 @@ def test_results_are_deterministic():
     o1, s1 = g.gdn2_fwd_chunked(*(d[n] for n in names), S0=d["S0"])
     o2, s2 = g.gdn2_fwd_chunked(*(d[n] for n in names), S0=d["S0"])
     assert torch.equal(o1, o2) and torch.equal(s1, s2)
-
-
-@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
-def test_decay_outside_range_is_reported(dtype):
-    """A chunk whose half-chunk log-decay passes -80 sets GDN2_ERR_RANGE; the next call is clean."""
-    d = to_dev(synth.draw_fwd(1, 128, 2, 64, 64, seed=12, dtype=dtype))
-    names = ("q", "k", "v", "b", "w", "log_alpha")
-    la = torch.full_like(d["log_alpha"], -3.0)
-    g.gdn2_fwd_chunked(*(d[n] for n in names[:5]), la)
-    assert g.gdn2_check_device_error() == g.GDN2_ERR_RANGE
-    g.gdn2_fwd_chunked(*(d[n] for n in names))
-    assert g.gdn2_check_device_error() == g.GDN2_OK
 
 
 def test_bounded_wait_gives_up_and_reports():
