@@ -2,9 +2,12 @@
 """Benchmark of the Gated DeltaNet-2 operator on B200.
 
 One step = one gdn2_fwd_chunked call over the 1.3B-layer workload (B=1, H=16,
-T=4096, dk=dv=128, bf16 inputs, fp32 decay and state, chunk 64).  The same
-run also times gdn2_decode_step on the decode workload (B=256, H=16, d=128,
-fp32 state of 268 MB updated in place) and reports its HBM bandwidth.
+T=4096, dk=dv=128, bf16 inputs, fp32 decay and state, chunk 64).  `value` is in
+tokens/s, a token being one position of one sequence with all 16 heads
+(B*T tokens per call).  The same run also times the training-batch (B=8) and
+long-context (T=65536) forwards, each against its own HBM roofline, and
+gdn2_decode_step on the decode workload (B=256, H=16, d=128, fp32 state of
+268 MB updated in place) with its HBM bandwidth.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
@@ -36,12 +39,19 @@ CASE = synth.LAYER_BF16
 DEC = synth.DECODE_F32
 N_INPUT_SETS = 4  # rotating input sets: 4 x 136 MB > 126 MB of L2
 
-# dram__bytes_read.sum + dram__bytes_write.sum per launch from an ncu capture of
-# the current kernels (None once a kernel has changed since the capture).  The
-# layer-workload forward is one persistent launch
-# (profiles/persist_kernel_layer_bf16.md); decode:
-# profiles/decode_kernel_decode_b256.md.
-NCU_TRAFFIC_BYTES = {"fwd": 117.728e6 + 56.744192e6, "decode": 281.078016e6 + 213.638144e6}
+# dram__bytes_read.sum + dram__bytes_write.sum per call from an ncu capture of
+# the current kernels (None once a kernel has changed since the capture), summed
+# over the kernels of one call; the captures are summarised under profiles/.
+NCU_TRAFFIC_BYTES = {"fwd": None, "train": None, "long": None, "decode": 281.078016e6 + 213.638144e6}
+EXTRA_CASES = ((synth.TRAIN_BF16, "train", 3, 10), (synth.LONG_BF16, "long", 2, 5))
+
+
+def bench_config():
+    """The `config` of the JSON line (the same for both arms)."""
+    c = CASE
+    return {"workload": c.name, "B": c.B, "T": c.T, "H": c.H, "dk": c.dk, "dv": c.dv, "chunk": 64,
+            "inputs": "bf16 q,k,v,b,w; fp32 log_alpha; fp32 state",
+            "l2": f"rotating {N_INPUT_SETS} device input sets (> 126 MB L2)"}
 
 
 def peaks():
@@ -52,10 +62,21 @@ def peaks():
     return FALLBACK_HBM_GBS, "fallback"
 
 
-def fwd_algorithmic_bytes(B, T, H, dk, dv, s_in, s_out, has_s0, has_st):
-    per_head_token = (3 * dk + 2 * dv) * s_in + 4 * dk + dv * s_out
+def fwd_algorithmic_bytes(B, T, H, dk, dv, s_in, s_out, has_s0, has_st, layout=0):
+    """Bytes a forward must move: inputs once, outputs once, states once.  With
+    a gate layout (bit 1 erase, 2 write, 4 decay) that gate is one value per
+    (token, head)."""
+    b_ch = 1 if layout & 1 else dk
+    w_ch = 1 if layout & 2 else dv
+    a_ch = 1 if layout & 4 else dk
+    per_head_token = (2 * dk + dv + b_ch + w_ch) * s_in + 4 * a_ch + dv * s_out
     state = B * H * dk * dv * 4
     return B * T * H * per_head_token + state * (int(has_s0) + int(has_st))
+
+
+def decode_tokens_algorithmic_bytes(B, T, H, dk, dv, s_in=4, s_out=4):
+    """T tokens on a resident state: the state read and written once, every token's inputs and outputs once."""
+    return B * H * (2 * dk * dv * 4 + T * ((3 * dk + 2 * dv) * s_in + 4 * dk + dv * s_out))
 
 
 def decode_algorithmic_bytes(B, H, dk, dv, s_in=4, s_out=4):
@@ -149,7 +170,7 @@ def cpu_oracle_tokens_per_s(sample_T: int, heads: int, nthreads: int = 0):
     t = time.perf_counter()
     orc.fwd(*args, S0=None, nthreads=nthreads)
     dt = time.perf_counter() - t
-    return sample_T * heads / dt, cores, dt
+    return sample_T / dt, cores, dt
 
 
 def run_reference(args, ws, rank):
@@ -159,7 +180,7 @@ def run_reference(args, ws, rank):
     heads = CASE.H
     rate, cores, _ = cpu_oracle_tokens_per_s(256, heads)          # calibration
     per_step_s = 120.0 / (args.steps + args.warmup)                # whole run ~2 min
-    T = int(max(64, min(CASE.T, per_step_s * rate / heads)))
+    T = int(max(64, min(CASE.T, per_step_s * rate)))
     vals = []
     for i in range(args.warmup + args.steps):
         v, cores, dt = cpu_oracle_tokens_per_s(T, heads)
@@ -170,10 +191,9 @@ def run_reference(args, ws, rank):
               f"OpenMP over heads")
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
             "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
-            "ms_per_step": CASE.B * CASE.T * CASE.H / value * 1e3, "higher_is_better": True,
+            "ms_per_step": CASE.B * CASE.T / value * 1e3, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": CASE.name, "B": 1, "T": CASE.T, "H": heads, "dk": 128,
-                       "dv": 128, "chunk": 64},
+            "config": bench_config(),
             "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
@@ -187,8 +207,8 @@ def run_profile_case(args):
     torch.cuda.set_device(0)
     dev = torch.device("cuda", 0)
     names = ("q", "k", "v", "b", "w", "log_alpha")
-    if args.profile in ("fwd", "fwd_train"):
-        c = CASE if args.profile == "fwd" else synth.TRAIN_BF16
+    if args.profile in ("fwd", "fwd_train", "fwd_long"):
+        c = {"fwd": CASE, "fwd_train": synth.TRAIN_BF16, "fwd_long": synth.LONG_BF16}[args.profile]
         d = synth.draw_fwd_device(c.B, c.T, c.H, c.dk, c.dv, seed=0, device=dev, dtype=c.dtype,
                                   log_alpha_range=c.log_alpha_range, gate_sigma=c.gate_sigma)
         for _ in range(args.warmup + args.steps):
@@ -213,7 +233,7 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--decode-steps", type=int, default=1000)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--profile", choices=["fwd", "fwd_train", "decode"], default=None,
+    ap.add_argument("--profile", choices=["fwd", "fwd_train", "fwd_long", "decode"], default=None,
                     help="run a few launches of one operator on the bench workload for an ncu "
                          "capture (no timing, no JSON line)")
     args = ap.parse_args()
@@ -285,7 +305,7 @@ def main():
     if g.gdn2_check_device_error() != g.GDN2_OK:
         raise RuntimeError("device error during the timed region")
 
-    tokens_per_step = c.B * c.T * c.H
+    tokens_per_step = c.B * c.T
     value = tokens_per_step * args.steps * ws / (total_ms / 1e3)
     alg_bytes = fwd_algorithmic_bytes(c.B, c.T, c.H, c.dk, c.dv, 2, 2, False, True)
     achieved = alg_bytes / (mean_launch_ms / 1e3) / 1e9
@@ -318,6 +338,75 @@ def main():
     e2e_value = tokens_per_step * e2e_steps * ws / (e2e_ms / 1e3)
     del sets, host, dev_in
 
+    # ---------------- the other bf16 workloads, each against its own roofline ----------------
+    extra = {}
+    for ce, key, warm, reps in EXTRA_CASES:
+        d = synth.draw_fwd_device(ce.B, ce.T, ce.H, ce.dk, ce.dv, seed=300 + rank, device=dev, dtype=ce.dtype,
+                                  log_alpha_range=ce.log_alpha_range, gate_sigma=ce.gate_sigma)
+        s0 = (ce.s0_sigma * torch.randn(ce.B, ce.H, ce.dk, ce.dv, device=dev)) if ce.s0_sigma > 0 else None
+        oe = torch.empty(ce.B, ce.T, ce.H, ce.dv, dtype=ce.dtype, device=dev)
+        se = torch.empty(ce.B, ce.H, ce.dk, ce.dv, dtype=torch.float32, device=dev)
+        for _ in range(warm):
+            g.gdn2_fwd_chunked(*(d[n] for n in names), S0=s0, o=oe, S_T=se, check=False)
+        torch.cuda.synchronize()
+        barrier(ws)
+        x0 = torch.cuda.Event(enable_timing=True); x1 = torch.cuda.Event(enable_timing=True)
+        x0.record(stream)
+        for _ in range(reps):
+            g.gdn2_fwd_chunked(*(d[n] for n in names), S0=s0, o=oe, S_T=se, check=False)
+        x1.record(stream)
+        torch.cuda.synchronize()
+        ms = max_over_ranks(x0.elapsed_time(x1), ws) / reps
+        eb = fwd_algorithmic_bytes(ce.B, ce.T, ce.H, ce.dk, ce.dv, 2, 2, s0 is not None, True)
+        gbs = eb / (ms / 1e3) / 1e9
+        extra[key] = {"workload": ce.name, "us_per_call": ms * 1e3, "tokens_per_s": ce.B * ce.T * ws / (ms / 1e3),
+                      "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm_peak, "unit": "GB/s",
+                                   "frac": gbs / hbm_peak, "traffic": NCU_TRAFFIC_BYTES[key],
+                                   "algorithmic_bytes_per_call": eb},
+                      "launches": g.gdn2_fwd_chunked_launches(ce.B, ce.T, ce.H, ce.dk, ce.dv, ce.dtype),
+                      "calls": reps, "l2": "inputs > 126 MB L2"}
+        del d, oe, se, s0
+    if g.gdn2_check_device_error() != g.GDN2_OK:
+        raise RuntimeError("device error while timing the other workloads")
+
+    # ---------------- gate-variant fast paths on the layer workload ----------------
+    layouts = {}
+    gen = torch.Generator(device=dev).manual_seed(401 + rank)
+    lsets = []
+    for i in range(N_INPUT_SETS):  # rotated, like the main measurement: more than L2 holds
+        d = synth.draw_fwd_device(c.B, c.T, c.H, c.dk, c.dv, seed=400 + 10 * rank + i, device=dev, dtype=c.dtype,
+                                  log_alpha_range=c.log_alpha_range, gate_sigma=c.gate_sigma)
+        d["beta"] = torch.sigmoid(torch.randn(c.B, c.T, c.H, generator=gen, device=dev)).to(c.dtype)
+        d["la_s"] = -torch.exp(torch.rand(c.B, c.T, c.H, generator=gen, device=dev) * 4.0 - 5.0)
+        del d["b"], d["w"]
+        lsets.append(d)
+    for lname, lay, la_key in (("kda", 3, "log_alpha"), ("gdn", 7, "la_s")):
+        def call(i):
+            d = lsets[i % N_INPUT_SETS]
+            g.gdn2_fwd_chunked(d["q"], d["k"], d["v"], d["beta"], d["beta"], d[la_key], S0=None, o=o, S_T=S_T,
+                               check=False)
+        for i in range(5):
+            call(i)
+        torch.cuda.synchronize()
+        barrier(ws)
+        x0 = torch.cuda.Event(enable_timing=True); x1 = torch.cuda.Event(enable_timing=True)
+        reps = 100
+        x0.record(stream)
+        for i in range(reps):
+            call(i)
+        x1.record(stream)
+        torch.cuda.synchronize()
+        ms = max_over_ranks(x0.elapsed_time(x1), ws) / reps
+        eb = fwd_algorithmic_bytes(c.B, c.T, c.H, c.dk, c.dv, 2, 2, False, True, layout=lay)
+        layouts[lname] = {"layout": lay, "us_per_call": ms * 1e3, "tokens_per_s": c.B * c.T * ws / (ms / 1e3),
+                          "roofline": {"bound": "hbm", "achieved": eb / (ms / 1e3) / 1e9, "peak": hbm_peak,
+                                       "unit": "GB/s", "frac": eb / (ms / 1e3) / 1e9 / hbm_peak,
+                                       "algorithmic_bytes_per_call": eb},
+                          "l2": f"rotating {N_INPUT_SETS} device input sets"}
+    del lsets
+    if g.gdn2_check_device_error() != g.GDN2_OK:
+        raise RuntimeError("device error while timing the gate layouts")
+
     # ---------------- decode: fp32 state resident in HBM, in place ----------------
     dc = DEC
     S = 0.05 * torch.randn(dc.B, dc.H, dc.dk, dc.dv, device=dev)
@@ -345,13 +434,39 @@ def main():
     if g.gdn2_check_device_error() != g.GDN2_OK:
         raise RuntimeError("device error during decode timing")
 
+    # ---------------- multi-token decode: T tokens per call on the resident state ----------------
+    tok_calls = {}
+    for Tn in (4, 16):
+        dd = synth.draw_fwd_device(dc.B, Tn, dc.H, dc.dk, dc.dv, seed=7100 + Tn, device=dev, dtype=torch.float32)
+        ot = torch.empty(dc.B, Tn, dc.H, dc.dv, device=dev)
+        for _ in range(3):
+            g.gdn2_decode_tokens(*(dd[n] for n in names), S, o=ot, check=False)
+        torch.cuda.synchronize()
+        barrier(ws)
+        x0 = torch.cuda.Event(enable_timing=True); x1 = torch.cuda.Event(enable_timing=True)
+        reps = 50
+        x0.record(stream)
+        for _ in range(reps):
+            g.gdn2_decode_tokens(*(dd[n] for n in names), S, o=ot, check=False)
+        x1.record(stream)
+        torch.cuda.synchronize()
+        ms = max_over_ranks(x0.elapsed_time(x1), ws) / reps
+        tb = decode_tokens_algorithmic_bytes(dc.B, Tn, dc.H, dc.dk, dc.dv)
+        tok_calls[f"T{Tn}"] = {"T": Tn, "us_per_call": ms * 1e3, "tokens_per_s": dc.B * Tn * ws / (ms / 1e3),
+                               "hbm_gbs": tb / (ms / 1e3) / 1e9, "frac": tb / (ms / 1e3) / 1e9 / hbm_peak,
+                               "algorithmic_bytes_per_call": tb,
+                               "vs_decode_steps": (Tn * dec_ms) / ms}
+        del dd, ot
+    if g.gdn2_check_device_error() != g.GDN2_OK:
+        raise RuntimeError("device error during multi-token decode timing")
+
     # ---------------- CPU baseline (oracle) on rank 0, N = 1 ----------------
     cpu = None
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
         v, cores, dt = cpu_oracle_tokens_per_s(c.T, c.H)
         v1, _, dt1 = cpu_oracle_tokens_per_s(1024, c.H, nthreads=1)
         cpu = {"value": v, "unit": "tokens/s", "cores": cores, "kind": "oracle",
-               "sample": f"the whole workload (B=1 H=16 T=4096 d=128, 65,536 head-tokens), fp64, "
+               "sample": f"the whole workload (B=1 H=16 T=4096 d=128, 4,096 tokens of 16 heads), fp64, "
                          f"{dt:.1f} s",
                "single_core": {"value": v1, "unit": "tokens/s",
                                "sample": f"the first 1024 tokens of the workload, 16 heads, one thread, "
@@ -363,11 +478,8 @@ def main():
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_ms / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic",
-            "config": {"workload": c.name, "B": c.B, "T": c.T, "H": c.H, "dk": c.dk, "dv": c.dv,
-                       "chunk": 64, "inputs": "bf16 q,k,v,b,w; fp32 log_alpha; fp32 state",
-                       "l2": f"rotating {N_INPUT_SETS} device input sets "
-                             f"({N_INPUT_SETS * alg_bytes / 1e6:.0f} MB > 126 MB L2)",
-                       "replicas": ws},
+            "config": bench_config(),
+            "head_tokens_per_s": value * c.H,
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
                          "frac": achieved / hbm_peak, "traffic": NCU_TRAFFIC_BYTES["fwd"],
                          "peak_kind": peak_kind, "algorithmic_bytes_per_launch": alg_bytes,
@@ -377,7 +489,13 @@ def main():
                        "frac": dec_gbs / hbm_peak, "peak": hbm_peak,
                        "algorithmic_bytes_per_step": dec_bytes, "steps": args.decode_steps,
                        "traffic": NCU_TRAFFIC_BYTES["decode"],
-                       "l2": "state 268 MB > 126 MB L2, streamed every step"},
+                       "dram_gbs": NCU_TRAFFIC_BYTES["decode"] / (dec_ms / 1e3) / 1e9,
+                       "l2": "state 268 MB > 126 MB L2, streamed every step (part of it stays in L2 "
+                             "between steps: DRAM bytes per step below the algorithmic bytes)"},
+            "workloads": extra,
+            "gate_layouts": layouts,
+            "decode_tokens": {"workload": "decode state B=256 H=16 d=128 fp32, T tokens per call",
+                              "calls": tok_calls},
             "cpu_baseline": cpu,
             "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "steps": e2e_steps},

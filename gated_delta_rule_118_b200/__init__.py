@@ -29,10 +29,16 @@ GDN2_ERR_SCRATCH_LIMIT = 9
 GDN2_F32 = 0
 GDN2_BF16 = 1
 
+# gdn2_gate_layout bits: which gates hold one value per (token, head)
+GDN2_GATES_PER_CHANNEL = 0
+GDN2_ERASE_SCALAR = 1
+GDN2_WRITE_SCALAR = 2
+GDN2_DECAY_SCALAR = 4
+
 # Every symbol include/gdn2.h declares.
-EXPORTED = ("gdn2_fwd_chunked", "gdn2_fwd_chunked_noalloc", "gdn2_decode_step",
-            "gdn2_check_device_error", "gdn2_selftest_bounded_wait", "gdn2_fwd_chunked_launches",
-            "gdn2_status_string")
+EXPORTED = ("gdn2_fwd_chunked", "gdn2_fwd_chunked_gates", "gdn2_fwd_chunked_noalloc",
+            "gdn2_decode_step", "gdn2_decode_tokens", "gdn2_check_device_error",
+            "gdn2_selftest_bounded_wait", "gdn2_fwd_chunked_launches", "gdn2_status_string")
 
 _lib = None
 
@@ -54,6 +60,10 @@ def lib() -> ctypes.CDLL:
         vp, fp, ci = ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int
         L.gdn2_fwd_chunked.argtypes = [vp] * 5 + [fp, fp, vp, fp] + [ci] * 6 + [vp]
         L.gdn2_fwd_chunked.restype = ci
+        L.gdn2_fwd_chunked_gates.argtypes = [vp] * 5 + [fp, fp, vp, fp] + [ci] * 6 + [ctypes.c_uint, vp]
+        L.gdn2_fwd_chunked_gates.restype = ci
+        L.gdn2_decode_tokens.argtypes = [vp] * 5 + [fp, fp, vp] + [ci] * 6 + [ctypes.c_uint, vp]
+        L.gdn2_decode_tokens.restype = ci
         L.gdn2_fwd_chunked_noalloc.argtypes = [vp] * 5 + [fp, fp, vp, fp] + [ci] * 6 + [vp]
         L.gdn2_fwd_chunked_noalloc.restype = ci
         L.gdn2_decode_step.argtypes = [vp] * 5 + [fp, fp, vp] + [ci] * 5 + [vp]
@@ -91,12 +101,22 @@ def _stream(stream):
     return ctypes.c_void_p(s.cuda_stream)
 
 
+def _gate_layout(q, b, w, log_alpha):
+    """gdn2_gate_layout bits from the shapes: a gate of shape q.shape[:-1] is per (token, head)."""
+    tok = tuple(q.shape[:-1])
+    return ((GDN2_ERASE_SCALAR if tuple(b.shape) == tok else 0)
+            | (GDN2_WRITE_SCALAR if tuple(w.shape) == tok else 0)
+            | (GDN2_DECAY_SCALAR if tuple(log_alpha.shape) == tok else 0))
+
+
 def gdn2_fwd_chunked(q, k, v, b, w, log_alpha, S0=None, o=None, S_T=None, *,
                      stream=None, want_state=True, check=True):
     """Chunked forward.  Tensors are CUDA, contiguous, [B,T,H,d]; returns (o, S_T).
 
     ``o`` and ``S_T`` are allocated with torch when not given (S_T only when
-    ``want_state``).  Raises Gdn2Error on a non-OK status.
+    ``want_state``).  b, w or log_alpha of shape [B,T,H] (one value per token and
+    head) select the matching gate layout (gdn2_fwd_chunked_gates).  Raises
+    Gdn2Error on a non-OK status.
     """
     B, T, H, dk = q.shape
     dv = v.shape[-1]
@@ -110,11 +130,17 @@ def gdn2_fwd_chunked(q, k, v, b, w, log_alpha, S0=None, o=None, S_T=None, *,
             raise ValueError(f"{name} must be a contiguous CUDA tensor")
     if log_alpha.dtype != torch.float32 or (S0 is not None and S0.dtype != torch.float32):
         raise TypeError("log_alpha and S0 must be float32")
-    st = lib().gdn2_fwd_chunked(_ptr(q), _ptr(k), _ptr(v), _ptr(b), _ptr(w), _ptr(log_alpha),
-                                _ptr(S0), _ptr(o), _ptr(S_T), B, T, H, dk, dv, _dtype_code(q),
-                                _stream(stream))
+    layout = _gate_layout(q, b, w, log_alpha)
+    if layout:
+        st = lib().gdn2_fwd_chunked_gates(_ptr(q), _ptr(k), _ptr(v), _ptr(b), _ptr(w), _ptr(log_alpha),
+                                          _ptr(S0), _ptr(o), _ptr(S_T), B, T, H, dk, dv, _dtype_code(q),
+                                          layout, _stream(stream))
+    else:
+        st = lib().gdn2_fwd_chunked(_ptr(q), _ptr(k), _ptr(v), _ptr(b), _ptr(w), _ptr(log_alpha),
+                                    _ptr(S0), _ptr(o), _ptr(S_T), B, T, H, dk, dv, _dtype_code(q),
+                                    _stream(stream))
     if check and st != GDN2_OK:
-        raise Gdn2Error(st, "gdn2_fwd_chunked")
+        raise Gdn2Error(st, "gdn2_fwd_chunked_gates" if layout else "gdn2_fwd_chunked")
     return o, S_T
 
 
@@ -151,6 +177,26 @@ def gdn2_decode_step(q, k, v, b, w, log_alpha, S, o=None, *, stream=None, check=
                                 _ptr(S), _ptr(o), B, H, dk, dv, _dtype_code(q), _stream(stream))
     if check and st != GDN2_OK:
         raise Gdn2Error(st, "gdn2_decode_step")
+    return o
+
+
+def gdn2_decode_tokens(q, k, v, b, w, log_alpha, S, o=None, *, stream=None, check=True):
+    """T recurrent tokens on a resident state: [B,T,H,d] inputs (b, w, log_alpha may be
+    [B,T,H]: one value per token and head), S [B,H,dk,dv] fp32 updated in place;
+    returns o [B,T,H,dv]."""
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    if o is None:
+        o = torch.empty((B, T, H, dv), dtype=q.dtype, device=q.device)
+    for name, t in (("q", q), ("k", k), ("v", v), ("b", b), ("w", w), ("log_alpha", log_alpha),
+                    ("S", S), ("o", o)):
+        if not (t.is_cuda and t.is_contiguous()):
+            raise ValueError(f"{name} must be a contiguous CUDA tensor")
+    st = lib().gdn2_decode_tokens(_ptr(q), _ptr(k), _ptr(v), _ptr(b), _ptr(w), _ptr(log_alpha),
+                                  _ptr(S), _ptr(o), B, T, H, dk, dv, _dtype_code(q),
+                                  _gate_layout(q, b, w, log_alpha), _stream(stream))
+    if check and st != GDN2_OK:
+        raise Gdn2Error(st, "gdn2_decode_tokens")
     return o
 
 

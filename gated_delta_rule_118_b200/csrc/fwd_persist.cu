@@ -160,7 +160,8 @@ template <int DV, int DVT>
 __global__ void __launch_bounds__(kPersistThreads, 1)
 persist_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ CUtensorMap tm_la,
-               const bf16 *__restrict__ vg, const bf16 *__restrict__ wg, bf16 *__restrict__ o, const float *S0,
+               const bf16 *__restrict__ vg, const bf16 *__restrict__ wg, const prep::GateSrc gs,
+               bf16 *__restrict__ o, const float *S0,
                float *S_T, uint8_t *__restrict__ recs, uint8_t *__restrict__ sxs, uint32_t *flags, int B, int T,
                int H, int nchain, unsigned int *err)
 {
@@ -237,7 +238,8 @@ persist_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                     fence_proxy_async_global();
                     if (ok) {
                         if (it.kind == 0)
-                            prep::prep_issue_loads(hs, hb, &tm_q, &tm_k, &tm_b, &tm_la, c * kChunk, r % H, r / H);
+                            prep::prep_issue_loads(hs, hb, &tm_q, &tm_k, &tm_b, &tm_la, c * kChunk, r % H, r / H,
+                                                 gs.layout);
                         else
                             outp::out_issue_loads<DV>(hs, hb + 2, recs + ((long)r * kRing + slot) * Record<DV>::BYTES,
                                                       sxs + ((long)r * kRing + slot) * SxSlot<DV>::BYTES);
@@ -252,8 +254,8 @@ persist_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             uint64_t *ld_bar = it.kind == 0 ? hb : hb + 2;
             const uint32_t ld_phase = it.kind == 0 ? tma_phase : out_phase;
             if (it.kind == 0) {
-                ok = prep::prep_chunk<DV>(hs, ht, lt, bar_id, hb, tma_phase, hb + 1, mma_phase, vg, wg, rec, T, H,
-                                          c * kChunk, h, bi, err);
+                ok = prep::prep_chunk<DV>(hs, ht, lt, bar_id, hb, tma_phase, hb + 1, mma_phase, vg, wg, gs, rec, T,
+                                          H, c * kChunk, h, bi, err);
                 tma_phase ^= 1;
             } else {
                 const int t0 = c * kChunk;
@@ -340,8 +342,9 @@ cudaError_t launch_persist(const FwdArgs &a, const CUtensorMap *maps, uint8_t *w
     attr[0].val.cooperative = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
+    const prep::GateSrc gs{(const bf16 *)a.b, a.log_alpha, a.layout};
     return cudaLaunchKernelEx(&cfg, kern, maps[0], maps[1], maps[2], maps[3], (const bf16 *)a.v, (const bf16 *)a.w,
-                              (bf16 *)a.o, a.S0, a.S_T, recs, sxs, flags, a.B, a.T, a.H, p.nchain, a.err);
+                              gs, (bf16 *)a.o, a.S0, a.S_T, recs, sxs, flags, a.B, a.T, a.H, p.nchain, a.err);
 }
 
 }  // namespace gdn2

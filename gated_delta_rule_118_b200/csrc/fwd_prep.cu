@@ -16,8 +16,8 @@ template <int DV>
 __global__ void __launch_bounds__(kPrepThreads, 2)
 prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
             const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ CUtensorMap tm_la,
-            const bf16 *__restrict__ vg, const bf16 *__restrict__ wg, uint8_t *__restrict__ ws, int Tlen, int H,
-            int c0, int WC, unsigned int *err)
+            const bf16 *__restrict__ vg, const bf16 *__restrict__ wg, const GateSrc gs, uint8_t *__restrict__ ws,
+            int Tlen, int H, int c0, int WC, unsigned int *err)
 {
     using L = PrepLayout;
     using R = Record<DV>;
@@ -35,7 +35,7 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         mbar_init(bar_tma, 1);
         mbar_init(bar_mma, 1);
         fence_mbar_init();
-        prep_issue_loads(sm, bar_tma, &tm_q, &tm_k, &tm_b, &tm_la, t0, h, bi);
+        prep_issue_loads(sm, bar_tma, &tm_q, &tm_k, &tm_b, &tm_la, t0, h, bi, gs.layout);
     }
     if (warp == 0) {
         tmem_alloc(slot, L::TMEM_COLS);
@@ -48,7 +48,7 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     tc_fence_after();
     const uint32_t tmem = *slot;
     uint32_t mma_phase = 0;
-    prep_chunk<DV>(sm, tmem, tid, 0, bar_tma, 0, bar_mma, mma_phase, vg, wg, rec, Tlen, H, t0, h, bi, err);
+    prep_chunk<DV>(sm, tmem, tid, 0, bar_tma, 0, bar_mma, mma_phase, vg, wg, gs, rec, Tlen, H, t0, h, bi, err);
     tc_fence_before();
     __syncthreads();
     if (warp == 0) {
@@ -72,8 +72,9 @@ cudaError_t launch_prep_impl(const FwdArgs &a, const CUtensorMap *maps, uint8_t 
     cudaError_t e = ensure_smem_limit(kern, L::BYTES, smem_set);
     if (e != cudaSuccess) return e;
     LaunchCfg lc(dim3(ncw, a.H, a.B), dim3(kPrepThreads), L::BYTES, a.stream, overlap);
+    const GateSrc gs{(const bf16 *)a.b, a.log_alpha, a.layout};
     return cudaLaunchKernelEx(&lc.cfg, kern, maps[0], maps[1], maps[2], maps[3], (const bf16 *)a.v,
-                              (const bf16 *)a.w, ws, a.T, a.H, c0, WC, a.err);
+                              (const bf16 *)a.w, gs, ws, a.T, a.H, c0, WC, a.err);
 }
 
 cudaError_t launch_prep(const FwdArgs &a, const CUtensorMap *maps, uint8_t *ws, int c0, int ncw, int WC, bool overlap)

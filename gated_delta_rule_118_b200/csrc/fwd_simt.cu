@@ -19,6 +19,7 @@
 // One CTA owns one (batch, head, 32-column value tile); value columns of the
 // state are independent because the erase and the decay act on key rows.
 #include "common.cuh"
+#include "gdn2.h"
 #include "launch.h"
 
 namespace gdn2 {
@@ -44,7 +45,7 @@ __global__ void __launch_bounds__(kSimtThreads)
 fwd_simt_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__ v,
                 const T *__restrict__ b, const T *__restrict__ w,
                 const float *__restrict__ log_alpha, const float *S0, T *__restrict__ o,
-                float *S_T, int Tlen, int H, int DV, unsigned int *err)
+                float *S_T, int Tlen, int H, int DV, unsigned layout)
 {
     using L = SimtSmem<DK, DVT>;
     constexpr int C = kChunk, LDK = L::LDK, LDC = L::LDC;
@@ -66,6 +67,9 @@ fwd_simt_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__res
     const int h = blockIdx.y;
     const long bi = blockIdx.z;
     const long pair = bi * H + h;
+    // gate layouts: b, w or log_alpha may hold one value per (token, head)
+    const bool b_scalar = layout & GDN2_ERASE_SCALAR, w_scalar = layout & GDN2_WRITE_SCALAR,
+               a_scalar = layout & GDN2_DECAY_SCALAR;
 
     for (int idx = tid; idx < DK * DVT; idx += kSimtThreads) {
         const int i = idx / DVT, j = idx % DVT;
@@ -83,8 +87,10 @@ fwd_simt_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__res
             const int t = idx / DK, i = idx % DK;
             float qv = 0.f, kv = 0.f, bv = 0.f, la = 0.f;
             if (t < Lc) {
-                const long off = ((bi * Tlen + t0 + t) * H + h) * (long)DK + i;
-                qv = to_f32(q[off]); kv = to_f32(k[off]); bv = to_f32(b[off]); la = log_alpha[off];
+                const long tok = (bi * Tlen + t0 + t) * H + h, off = tok * DK + i;
+                qv = to_f32(q[off]); kv = to_f32(k[off]);
+                bv = to_f32(b[b_scalar ? tok : off]);
+                la = log_alpha[a_scalar ? tok : off];
             }
             sQ[t * LDK + i] = qv; sK[t * LDK + i] = kv; sE[t * LDK + i] = bv; sG[t * LDK + i] = la;
         }
@@ -92,8 +98,8 @@ fwd_simt_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__res
             const int t = idx / DVT, j = idx % DVT;
             float z = 0.f;
             if (t < Lc) {
-                const long off = ((bi * Tlen + t0 + t) * H + h) * (long)DV + j0 + j;
-                z = to_f32(w[off]) * to_f32(v[off]);
+                const long tok = (bi * Tlen + t0 + t) * H + h, off = tok * DV + j0 + j;
+                z = to_f32(w[w_scalar ? tok : off]) * to_f32(v[off]);
             }
             sU[idx] = z;
         }
@@ -282,7 +288,7 @@ cudaError_t launch(const FwdArgs &a)
     dim3 grid(a.dv / DVT, a.H, a.B);
     kern<<<grid, kSimtThreads, smem, a.stream>>>(
         (const T *)a.q, (const T *)a.k, (const T *)a.v, (const T *)a.b, (const T *)a.w,
-        a.log_alpha, a.S0, (T *)a.o, a.S_T, a.T, a.H, a.dv, a.err);
+        a.log_alpha, a.S0, (T *)a.o, a.S_T, a.T, a.H, a.dv, a.layout);
     return cudaGetLastError();
 }
 

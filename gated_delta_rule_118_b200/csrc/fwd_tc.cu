@@ -14,6 +14,7 @@
 
 #include <mutex>
 
+#include "gdn2.h"
 #include "launch.h"
 #include "tc_common.cuh"
 
@@ -69,6 +70,28 @@ cudaMemPool_t workspace_pool(int dev)
     return pools[dev];
 }
 
+// Tensor maps of the TMA-loaded inputs: q, k, b, log_alpha, and v, w when
+// `n` is 6.  A gate given as one value per (token, head) is loaded without TMA;
+// its slot holds q's map, which the kernels do not use for it.
+bool make_input_maps(const FwdArgs &a, CUtensorMap *maps, int n)
+{
+    const auto BF = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+    if (!make_map(&maps[0], a.q, BF, 2, 128, a.H, a.T, a.B, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map(&maps[1], a.k, BF, 2, 128, a.H, a.T, a.B, 64, CU_TENSOR_MAP_SWIZZLE_128B))
+        return false;
+    maps[2] = maps[0];
+    maps[3] = maps[0];
+    if (!(a.layout & GDN2_ERASE_SCALAR) &&
+        !make_map(&maps[2], a.b, BF, 2, 128, a.H, a.T, a.B, 64, CU_TENSOR_MAP_SWIZZLE_128B))
+        return false;
+    if (!(a.layout & GDN2_DECAY_SCALAR) &&
+        !make_map(&maps[3], a.log_alpha, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, 128, a.H, a.T, a.B, 128,
+                  CU_TENSOR_MAP_SWIZZLE_NONE))
+        return false;
+    return n < 6 || (make_map(&maps[4], a.v, BF, 2, a.dv, a.H, a.T, a.B, a.dv, CU_TENSOR_MAP_SWIZZLE_NONE) &&
+                     make_map(&maps[5], a.w, BF, 2, a.dv, a.H, a.T, a.B, a.dv, CU_TENSOR_MAP_SWIZZLE_NONE));
+}
+
 }  // namespace
 
 FwdTcPlan plan_fwd_tc(int B, int T, int H, int dv, size_t budget, int num_sms)
@@ -110,15 +133,7 @@ FwdTcPlan plan_fwd_tc(int B, int T, int H, int dv, size_t budget, int num_sms)
 cudaError_t run_fwd_tc(const FwdArgs &a, const FwdTcPlan &p, uint8_t *ws)
 {
     CUtensorMap maps[6];
-    const auto BF = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
-    if (!make_map(&maps[0], a.q, BF, 2, 128, a.H, a.T, a.B, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !make_map(&maps[1], a.k, BF, 2, 128, a.H, a.T, a.B, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !make_map(&maps[2], a.b, BF, 2, 128, a.H, a.T, a.B, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !make_map(&maps[3], a.log_alpha, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, 128, a.H, a.T, a.B, 128,
-                  CU_TENSOR_MAP_SWIZZLE_NONE) ||
-        !make_map(&maps[4], a.v, BF, 2, a.dv, a.H, a.T, a.B, a.dv, CU_TENSOR_MAP_SWIZZLE_NONE) ||
-        !make_map(&maps[5], a.w, BF, 2, a.dv, a.H, a.T, a.B, a.dv, CU_TENSOR_MAP_SWIZZLE_NONE))
-        return cudaErrorInvalidValue;
+    if (!make_input_maps(a, maps, 6)) return cudaErrorInvalidValue;
     uint8_t *recs = ws, *sxs = ws + p.rec_total;
     float *carry = p.carry_bytes ? reinterpret_cast<float *>(ws + p.rec_total + p.sx_total) : nullptr;
     for (int w = 0; w < p.nwindows; ++w) {
@@ -183,15 +198,7 @@ StreamSet *stream_set(int dev)
 cudaError_t run_fwd_tc_overlapped(const FwdArgs &a, const FwdTcPlan &p, uint8_t *ws, StreamSet &ss)
 {
     CUtensorMap maps[6];
-    const auto BF = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
-    if (!make_map(&maps[0], a.q, BF, 2, 128, a.H, a.T, a.B, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !make_map(&maps[1], a.k, BF, 2, 128, a.H, a.T, a.B, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !make_map(&maps[2], a.b, BF, 2, 128, a.H, a.T, a.B, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !make_map(&maps[3], a.log_alpha, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, 128, a.H, a.T, a.B, 128,
-                  CU_TENSOR_MAP_SWIZZLE_NONE) ||
-        !make_map(&maps[4], a.v, BF, 2, a.dv, a.H, a.T, a.B, a.dv, CU_TENSOR_MAP_SWIZZLE_NONE) ||
-        !make_map(&maps[5], a.w, BF, 2, a.dv, a.H, a.T, a.B, a.dv, CU_TENSOR_MAP_SWIZZLE_NONE))
-        return cudaErrorInvalidValue;
+    if (!make_input_maps(a, maps, 6)) return cudaErrorInvalidValue;
     const int nslots = p.slots;
     const size_t slot_bytes = p.rec_total + p.sx_total;
     float *carry = p.carry_bytes ? reinterpret_cast<float *>(ws + nslots * slot_bytes) : nullptr;
@@ -245,12 +252,7 @@ bool try_fwd_persist(const FwdArgs &a, cudaMemPool_t pool, cudaError_t *status)
     const PersistPlan p = plan_fwd_persist(a.B, a.T, a.H, a.dv, a.num_sms);
     if (!p.use) return false;
     CUtensorMap maps[4];
-    const auto BF = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
-    if (!make_map(&maps[0], a.q, BF, 2, 128, a.H, a.T, a.B, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !make_map(&maps[1], a.k, BF, 2, 128, a.H, a.T, a.B, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !make_map(&maps[2], a.b, BF, 2, 128, a.H, a.T, a.B, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !make_map(&maps[3], a.log_alpha, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, 128, a.H, a.T, a.B, 128,
-                  CU_TENSOR_MAP_SWIZZLE_NONE)) {
+    if (!make_input_maps(a, maps, 4)) {
         *status = cudaErrorInvalidValue;
         return true;
     }

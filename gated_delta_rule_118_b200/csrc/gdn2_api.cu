@@ -65,14 +65,17 @@ bool device_error_word(unsigned int **err)
 
 using namespace gdn2;
 
-extern "C" gdn2_status gdn2_fwd_chunked(const void *q, const void *k, const void *v,
-                                        const void *b, const void *w, const float *log_alpha,
-                                        const float *S0, void *o, float *S_T,
-                                        int B, int T, int H, int dk, int dv,
-                                        gdn2_dtype dtype, gdn2_stream_t stream)
+namespace {
+
+constexpr unsigned kLayoutBits = GDN2_ERASE_SCALAR | GDN2_WRITE_SCALAR | GDN2_DECAY_SCALAR;
+
+gdn2_status fwd_chunked(const void *q, const void *k, const void *v, const void *b, const void *w,
+                        const float *log_alpha, const float *S0, void *o, float *S_T, int B, int T, int H, int dk,
+                        int dv, gdn2_dtype dtype, unsigned layout, gdn2_stream_t stream)
 {
     if (dtype != GDN2_F32 && dtype != GDN2_BF16) return GDN2_ERR_DTYPE;
     if (B <= 0 || H <= 0 || T < 0) return GDN2_ERR_SHAPE;
+    if (layout & ~kLayoutBits) return GDN2_ERR_UNSUPPORTED;
     gdn2_status st = check_dims(dk, dv);
     if (st != GDN2_OK) return st;
     if (B > 65535 || H > 65535) return GDN2_ERR_UNSUPPORTED;  // grid y/z limits
@@ -99,6 +102,7 @@ extern "C" gdn2_status gdn2_fwd_chunked(const void *q, const void *k, const void
     a.S0 = S0; a.o = o; a.S_T = S_T;
     a.B = B; a.T = T; a.H = H; a.dk = dk; a.dv = dv;
     a.bf16 = (dtype == GDN2_BF16);
+    a.layout = layout;
     a.stream = s;
     st = device_context(&a.err, &a.num_sms);
     if (st != GDN2_OK) return st;
@@ -108,13 +112,13 @@ extern "C" gdn2_status gdn2_fwd_chunked(const void *q, const void *k, const void
     return e == cudaSuccess ? GDN2_OK : GDN2_ERR_CUDA;
 }
 
-extern "C" gdn2_status gdn2_decode_step(const void *q, const void *k, const void *v,
-                                        const void *b, const void *w, const float *log_alpha,
-                                        float *S, void *o, int B, int H, int dk, int dv,
-                                        gdn2_dtype dtype, gdn2_stream_t stream)
+gdn2_status decode(const void *q, const void *k, const void *v, const void *b, const void *w,
+                   const float *log_alpha, float *S, void *o, int B, int T, int H, int dk, int dv,
+                   gdn2_dtype dtype, unsigned layout, gdn2_stream_t stream)
 {
     if (dtype != GDN2_F32 && dtype != GDN2_BF16) return GDN2_ERR_DTYPE;
-    if (B <= 0 || H <= 0) return GDN2_ERR_SHAPE;
+    if (B <= 0 || H <= 0 || T <= 0) return GDN2_ERR_SHAPE;
+    if (layout & ~kLayoutBits) return GDN2_ERR_UNSUPPORTED;
     gdn2_status st = check_dims(dk, dv);
     if (st != GDN2_OK) return st;
     if ((long long)B * H > 0x7fffffffLL) return GDN2_ERR_UNSUPPORTED;  // grid x limit
@@ -125,10 +129,47 @@ extern "C" gdn2_status gdn2_decode_step(const void *q, const void *k, const void
     }
     DecodeArgs a{};
     a.q = q; a.k = k; a.v = v; a.b = b; a.w = w; a.log_alpha = log_alpha;
-    a.S = S; a.o = o; a.B = B; a.H = H; a.dk = dk; a.dv = dv;
+    a.S = S; a.o = o; a.B = B; a.T = T; a.H = H; a.dk = dk; a.dv = dv;
     a.bf16 = (dtype == GDN2_BF16);
+    a.layout = layout;
     a.stream = reinterpret_cast<cudaStream_t>(stream);
     return launch_decode(a) == cudaSuccess ? GDN2_OK : GDN2_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" gdn2_status gdn2_fwd_chunked(const void *q, const void *k, const void *v,
+                                        const void *b, const void *w, const float *log_alpha,
+                                        const float *S0, void *o, float *S_T,
+                                        int B, int T, int H, int dk, int dv,
+                                        gdn2_dtype dtype, gdn2_stream_t stream)
+{
+    return fwd_chunked(q, k, v, b, w, log_alpha, S0, o, S_T, B, T, H, dk, dv, dtype, 0u, stream);
+}
+
+extern "C" gdn2_status gdn2_fwd_chunked_gates(const void *q, const void *k, const void *v,
+                                              const void *b, const void *w, const float *log_alpha,
+                                              const float *S0, void *o, float *S_T,
+                                              int B, int T, int H, int dk, int dv,
+                                              gdn2_dtype dtype, unsigned int layout, gdn2_stream_t stream)
+{
+    return fwd_chunked(q, k, v, b, w, log_alpha, S0, o, S_T, B, T, H, dk, dv, dtype, layout, stream);
+}
+
+extern "C" gdn2_status gdn2_decode_step(const void *q, const void *k, const void *v,
+                                        const void *b, const void *w, const float *log_alpha,
+                                        float *S, void *o, int B, int H, int dk, int dv,
+                                        gdn2_dtype dtype, gdn2_stream_t stream)
+{
+    return decode(q, k, v, b, w, log_alpha, S, o, B, 1, H, dk, dv, dtype, 0u, stream);
+}
+
+extern "C" gdn2_status gdn2_decode_tokens(const void *q, const void *k, const void *v,
+                                          const void *b, const void *w, const float *log_alpha,
+                                          float *S, void *o, int B, int T, int H, int dk, int dv,
+                                          gdn2_dtype dtype, unsigned int layout, gdn2_stream_t stream)
+{
+    return decode(q, k, v, b, w, log_alpha, S, o, B, T, H, dk, dv, dtype, layout, stream);
 }
 
 extern "C" gdn2_status gdn2_check_device_error(gdn2_stream_t stream)

@@ -16,8 +16,9 @@ struct DecodeArgs {
     const float *log_alpha;
     float *S;
     void *o;
-    int B, H, dk, dv;
+    int B, T, H, dk, dv;  // T tokens per call (1 for a decode step)
     bool bf16;
+    unsigned layout;      // gdn2_gate_layout bits
     cudaStream_t stream;
 };
 
@@ -29,6 +30,7 @@ struct FwdArgs {
     float *S_T;       // may be null (not written); may alias S0
     int B, T, H, dk, dv;
     bool bf16;
+    unsigned layout;    // gdn2_gate_layout bits
     cudaStream_t stream;
     unsigned int *err;  // device error word
     int num_sms;

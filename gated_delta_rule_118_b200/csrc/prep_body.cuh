@@ -63,6 +63,17 @@ struct PrepLayout {
 };
 static_assert(PrepLayout::BYTES * 2 + 2048 <= 233472, "two CTAs per SM");
 
+// Gate inputs that hold one value per (token, head) (gdn2_gate_layout bits in
+// `layout`); per-channel ones arrive by TMA.  Scalar b and log_alpha are
+// broadcast over the channels of their rows in shared memory, so everything
+// after the loads is the same for every layout.
+struct GateSrc {
+    const bf16 *b;     // [B][T][H] with GDN2_ERASE_SCALAR
+    const float *la;   // [B][T][H] with GDN2_DECAY_SCALAR
+    unsigned layout;
+};
+constexpr unsigned kEraseScalar = 1u, kWriteScalar = 2u, kDecayScalar = 4u;  // gdn2_gate_layout bits
+
 __device__ __forceinline__ void tmem_ld32_wait(uint32_t taddr, float (&r)[32])
 {
     tmem_ld32(taddr, r);
@@ -71,18 +82,20 @@ __device__ __forceinline__ void tmem_ld32_wait(uint32_t taddr, float (&r)[32])
 
 // The TMA loads of one chunk's q, b, k and log_alpha into a prep region,
 // completing on `bar_tma` (issued by one thread).
+// (b and log_alpha only where they are per channel).
 __device__ __forceinline__ void prep_issue_loads(uint8_t *sm, uint64_t *bar_tma, const CUtensorMap *tm_q,
                                                  const CUtensorMap *tm_k, const CUtensorMap *tm_b,
-                                                 const CUtensorMap *tm_la, int t0, int h, int bi)
+                                                 const CUtensorMap *tm_la, int t0, int h, int bi, unsigned layout)
 {
     using L = PrepLayout;
-    mbar_arrive_expect_tx(bar_tma, (uint32_t)L::TX);
+    const bool b_tma = !(layout & kEraseScalar), la_tma = !(layout & kDecayScalar);
+    mbar_arrive_expect_tx(bar_tma, (uint32_t)(L::TX - (b_tma ? 0 : 16384) - (la_tma ? 0 : 32768)));
     for (int kb = 0; kb < 2; ++kb) {
         tma_load_4d(sm + L::EQ + kb * 16384 + 8192, tm_q, bar_tma, kb * 64, h, t0, bi);
-        tma_load_4d(sm + L::EQ + kb * 16384, tm_b, bar_tma, kb * 64, h, t0, bi);
+        if (b_tma) tma_load_4d(sm + L::EQ + kb * 16384, tm_b, bar_tma, kb * 64, h, t0, bi);
         tma_load_4d(sm + L::KT + kb * 8192, tm_k, bar_tma, kb * 64, h, t0, bi);
     }
-    tma_load_4d(sm + L::LA, tm_la, bar_tma, 0, h, t0, bi);
+    if (la_tma) tma_load_4d(sm + L::LA, tm_la, bar_tma, 0, h, t0, bi);
 }
 
 // The prep of one chunk (tokens [t0, t0 + 64) of head h, batch bi) by the
@@ -96,8 +109,8 @@ template <int DV>
 __device__ __forceinline__ bool prep_chunk(uint8_t *sm, uint32_t tmem, int tid, int bar_id, uint64_t *bar_tma,
                                            uint32_t tma_phase, uint64_t *bar_mma, uint32_t &mma_phase,
                                            const bf16 *__restrict__ vg, const bf16 *__restrict__ wg,
-                                           uint8_t *__restrict__ rec, int Tlen, int H, int t0, int h, int bi,
-                                           unsigned int *err)
+                                           const GateSrc &gs, uint8_t *__restrict__ rec, int Tlen, int H, int t0,
+                                           int h, int bi, unsigned int *err)
 {
     using L = PrepLayout;
     using R = Record<DV>;
@@ -124,9 +137,36 @@ __device__ __forceinline__ bool prep_chunk(uint8_t *sm, uint32_t tmem, int tid, 
         vv[m] = make_uint4(0, 0, 0, 0);
         wv[m] = make_uint4(0, 0, 0, 0);
         if (t < Lc) {
-            const long off = (((long)bi * Tlen + t0 + t) * H + h) * DV + j;
+            const long tok = ((long)bi * Tlen + t0 + t) * H + h, off = tok * DV + j;
             vv[m] = __ldg(reinterpret_cast<const uint4 *>(vg + off));
-            wv[m] = __ldg(reinterpret_cast<const uint4 *>(wg + off));
+            if (gs.layout & kWriteScalar) {
+                const uint32_t two = (uint32_t)__bfloat16_as_ushort(wg[tok]) * 0x10001u;
+                wv[m] = make_uint4(two, two, two, two);
+            } else {
+                wv[m] = __ldg(reinterpret_cast<const uint4 *>(wg + off));
+            }
+        }
+    }
+    // scalar b / log_alpha: row t of the b tile (both 64-channel halves) and of
+    // log_alpha filled with the token's value (zero past the sequence end), into
+    // buffers the TMA leaves alone in these layouts
+    if (gs.layout & (kEraseScalar | kDecayScalar)) {
+        const int t = tid >> 2, part = tid & 3;
+        const long tok = ((long)bi * Tlen + t0 + t) * H + h;
+        if (gs.layout & kEraseScalar) {
+            const uint32_t two = t < Lc ? (uint32_t)__bfloat16_as_ushort(gs.b[tok]) * 0x10001u : 0u;
+#pragma unroll
+            for (int m = 0; m < 4; ++m) {
+                const int c = part * 4 + m;  // 16-byte piece of the token's 256 bytes
+                *reinterpret_cast<uint4 *>(sm + L::EQ + (c >> 3) * 16384 + t * 128 + (c & 7) * 16) =
+                    make_uint4(two, two, two, two);
+            }
+        }
+        if (gs.layout & kDecayScalar) {
+            const float lt = t < Lc ? gs.la[tok] : 0.f;
+#pragma unroll
+            for (int m = 0; m < 8; ++m)
+                *reinterpret_cast<float4 *>(sm + L::LA + t * 512 + part * 128 + m * 16) = make_float4(lt, lt, lt, lt);
         }
     }
     // One thread polls each mbarrier; the others park on the group's barrier,

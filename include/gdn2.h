@@ -64,6 +64,30 @@ typedef enum gdn2_dtype {
     GDN2_BF16 = 1
 } gdn2_dtype;
 
+/*
+ * Gate layouts: which of b, w and log_alpha hold one value per (token, head)
+ * instead of one per channel.  Bits of the `layout` argument of
+ * gdn2_fwd_chunked_gates and gdn2_decode_tokens; 0 is the per-channel layout of
+ * every other entry point.
+ *
+ * The pages derive the special cases of the operator from these shapes
+ * (iplexlaw.co.kr, section "Decisiones independientes en dos ejes"; gist.science,
+ * section 1): b = w = beta with beta a scalar per token gives Kimi Delta
+ * Attention (pass the same pointer for b and w with GDN2_ERASE_SCALAR |
+ * GDN2_WRITE_SCALAR); a scalar decay as well gives Gated DeltaNet (add
+ * GDN2_DECAY_SCALAR).  A channel-averaged erase or write gate alone is
+ * GDN2_ERASE_SCALAR or GDN2_WRITE_SCALAR.  A scalar tensor is [B][T][H]
+ * ([B][H] for gdn2_decode_step's T-less layout), same dtype as the per-channel
+ * one; it reads fewer bytes, which is what the bandwidth-bound kernels spend
+ * their time on.
+ */
+typedef enum gdn2_gate_layout {
+    GDN2_GATES_PER_CHANNEL = 0,  /* b [..][dk], w [..][dv], log_alpha [..][dk]     */
+    GDN2_ERASE_SCALAR = 1,       /* b is [B][T][H]: one erase gate per token, head  */
+    GDN2_WRITE_SCALAR = 2,       /* w is [B][T][H]: one write gate per token, head  */
+    GDN2_DECAY_SCALAR = 4        /* log_alpha is [B][T][H]: one decay per token, head */
+} gdn2_gate_layout;
+
 /* Same type as cudaStream_t; declared here so this header needs no CUDA header. */
 typedef struct CUstream_st *gdn2_stream_t;
 
@@ -163,6 +187,40 @@ gdn2_status gdn2_decode_step(const void *q, const void *k, const void *v,
                              const void *b, const void *w, const float *log_alpha,
                              float *S, void *o, int B, int H, int dk, int dv,
                              gdn2_dtype dtype, gdn2_stream_t stream);
+
+/*
+ * gdn2_decode_tokens -- T consecutive tokens of the recurrence on a state
+ * resident in device memory (multi-token decode, or a short prefill into a
+ * cached state: the recurrent form with a fixed-size state of gist.science,
+ * "Problem Statement").  Equivalent to T calls of gdn2_decode_step, but each
+ * state is read and written once per call instead of once per token; meant for
+ * T up to a few dozen (longer sequences: gdn2_fwd_chunked).
+ *
+ *   q, k        [B][T][H][dk]  dtype
+ *   v           [B][T][H][dv]  dtype
+ *   b           [B][T][H][dk], or [B][T][H] with GDN2_ERASE_SCALAR   dtype
+ *   w           [B][T][H][dv], or [B][T][H] with GDN2_WRITE_SCALAR   dtype
+ *   log_alpha   [B][T][H][dk], or [B][T][H] with GDN2_DECAY_SCALAR   fp32
+ *   S           [B][H][dk][dv] fp32   read and updated in place
+ *   o           [B][T][H][dv]  dtype  written
+ *   B, H, T >= 1; layout: a combination of gdn2_gate_layout bits.
+ */
+gdn2_status gdn2_decode_tokens(const void *q, const void *k, const void *v,
+                               const void *b, const void *w, const float *log_alpha,
+                               float *S, void *o, int B, int T, int H, int dk, int dv,
+                               gdn2_dtype dtype, unsigned int layout, gdn2_stream_t stream);
+
+/*
+ * gdn2_fwd_chunked_gates -- gdn2_fwd_chunked with a gate layout: b, w and/or
+ * log_alpha may be one value per (token, head) ([B][T][H]) as `layout` says.
+ * Everything else (arguments, results, execution) is as for gdn2_fwd_chunked,
+ * which is this function with layout 0.
+ */
+gdn2_status gdn2_fwd_chunked_gates(const void *q, const void *k, const void *v,
+                                   const void *b, const void *w, const float *log_alpha,
+                                   const float *S0, void *o, float *S_T,
+                                   int B, int T, int H, int dk, int dv,
+                                   gdn2_dtype dtype, unsigned int layout, gdn2_stream_t stream);
 
 /*
  * gdn2_check_device_error -- wait for `stream`, then read and clear the

@@ -166,3 +166,23 @@ def draw_log_alpha(B, T, H, dk, kind, *, seed):
         la[torch.rand(B, T, H, dk, generator=g) < 0.02] = float("-inf")
         return la.contiguous()
     raise ValueError(kind)
+
+
+def scalar_gates(d, layout, *, seed, gate_sigma=1.0):
+    """Replace b, w and/or log_alpha of a forward batch by one value per (token,
+    head) ([B,T,H]), as the gdn2_gate_layout bits in `layout` say: bit 1 erase
+    gate b, bit 2 write gate w (bits 1 and 2 together: one beta for both, the
+    same tensor), bit 4 the decay.  Drawn like the per-channel values."""
+    B, T, H, _ = d["q"].shape
+    g = torch.Generator(device="cpu").manual_seed(int(seed))
+    out = dict(d)
+    dtype = d["q"].dtype
+    beta = torch.sigmoid(gate_sigma * torch.randn(B, T, H, generator=g)).to(dtype).contiguous()
+    if layout & 1:
+        out["b"] = beta
+    if layout & 2:
+        out["w"] = beta if layout & 1 else \
+            torch.sigmoid(gate_sigma * torch.randn(B, T, H, generator=g)).to(dtype).contiguous()
+    if layout & 4:
+        out["log_alpha"] = (-torch.exp(torch.rand(B, T, H, generator=g) * 4.0 - 5.0)).contiguous()
+    return out

@@ -105,3 +105,48 @@ def test_noalloc_rejects_pairs_beyond_its_scratch(lib):
     for B, H in ((1, 178), (2, 89), (178, 1)):
         st = lib.gdn2_fwd_chunked_noalloc(P, P, P, P, P, P, None, P, None, B, 64, H, 128, 128, 1, None)
         assert st == g.GDN2_ERR_SCRATCH_LIMIT, (B, H)
+
+
+def fwd_gates(lib, *, layout=0, B=1, T=8, H=2, dk=64, dv=64, dtype=1, b=P):
+    return lib.gdn2_fwd_chunked_gates(P, P, P, b, P, P, None, P, None, B, T, H, dk, dv, dtype, layout, None)
+
+
+def dec_tokens(lib, *, layout=0, B=1, T=4, H=2, dk=64, dv=64, dtype=0, o=P):
+    return lib.gdn2_decode_tokens(P, P, P, P, P, P, P, o, B, T, H, dk, dv, dtype, layout, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(layout=8), g.GDN2_ERR_UNSUPPORTED),
+    (dict(layout=0xFFFF), g.GDN2_ERR_UNSUPPORTED),
+    (dict(dtype=7), g.GDN2_ERR_DTYPE),
+    (dict(B=0), g.GDN2_ERR_SHAPE),
+    (dict(dk=48), g.GDN2_ERR_UNSUPPORTED),
+    (dict(b=None), g.GDN2_ERR_NULL),
+    (dict(b=MIS, layout=1), g.GDN2_ERR_ALIGN),
+])
+def test_fwd_gates_rejects_bad_arguments(lib, kw, code):
+    assert fwd_gates(lib, **kw) == code
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(T=0), g.GDN2_ERR_SHAPE),
+    (dict(T=-1), g.GDN2_ERR_SHAPE),
+    (dict(layout=16), g.GDN2_ERR_UNSUPPORTED),
+    (dict(dtype=3), g.GDN2_ERR_DTYPE),
+    (dict(dv=32), g.GDN2_ERR_UNSUPPORTED),
+    (dict(o=None), g.GDN2_ERR_NULL),
+    (dict(o=MIS), g.GDN2_ERR_ALIGN),
+])
+def test_decode_tokens_rejects_bad_arguments(lib, kw, code):
+    assert dec_tokens(lib, **kw) == code
+
+
+def test_gate_layout_from_shapes():
+    import torch
+    q = torch.empty(2, 5, 3, 8)
+    per_ch = torch.empty(2, 5, 3, 8)
+    tok = torch.empty(2, 5, 3)
+    assert g._gate_layout(q, per_ch, per_ch, per_ch) == g.GDN2_GATES_PER_CHANNEL
+    assert g._gate_layout(q, tok, tok, per_ch) == g.GDN2_ERASE_SCALAR | g.GDN2_WRITE_SCALAR
+    assert g._gate_layout(q, tok, tok, tok) == 7
+    assert g._gate_layout(q, per_ch, tok, per_ch) == g.GDN2_WRITE_SCALAR
