@@ -79,6 +79,13 @@ def decode_tokens_algorithmic_bytes(B, T, H, dk, dv, s_in=4, s_out=4):
     return B * H * (2 * dk * dv * 4 + T * ((3 * dk + 2 * dv) * s_in + 4 * dk + dv * s_out))
 
 
+def layer_algorithmic_bytes(B, T, H, dk, dv, s_in=2, s_out=2):
+    """The fused layer: q, k, v, the erase/write/output-gate logits in the input dtype,
+    the decay logits in fp32, y out, the final state."""
+    per_head_token = (3 * dk + 3 * dv) * s_in + 4 * dk + dv * s_out
+    return B * T * H * per_head_token + B * H * dk * dv * 4
+
+
 def decode_algorithmic_bytes(B, H, dk, dv, s_in=4, s_out=4):
     # state read + written once, q,k,b (dk) and v,w (dv) in the input dtype,
     # log_alpha fp32, o in the input dtype
@@ -407,6 +414,34 @@ def main():
     if g.gdn2_check_device_error() != g.GDN2_OK:
         raise RuntimeError("device error while timing the gate layouts")
 
+    # ---------------- the fused layer entry point on the layer workload ----------------
+    lsets = [synth.draw_layer(c.B, c.T, c.H, c.dk, c.dv, seed=500 + 10 * rank + i, dtype=c.dtype)
+             for i in range(N_INPUT_SETS)]
+    lnames = ("q", "k", "v", "b_logit", "w_logit", "decay_logit", "g_logit", "norm_weight")
+    lsets = [{n: d[n].to(dev) for n in lnames} for d in lsets]
+    for i in range(5):
+        g.gdn2_layer_fwd(*(lsets[i % N_INPUT_SETS][n] for n in lnames), 1e-6, y=o, S_T=S_T, check=False)
+    torch.cuda.synchronize()
+    barrier(ws)
+    x0 = torch.cuda.Event(enable_timing=True); x1 = torch.cuda.Event(enable_timing=True)
+    reps = 100
+    x0.record(stream)
+    for i in range(reps):
+        g.gdn2_layer_fwd(*(lsets[i % N_INPUT_SETS][n] for n in lnames), 1e-6, y=o, S_T=S_T, check=False)
+    x1.record(stream)
+    torch.cuda.synchronize()
+    ms = max_over_ranks(x0.elapsed_time(x1), ws) / reps
+    lb = layer_algorithmic_bytes(c.B, c.T, c.H, c.dk, c.dv)
+    layer_line = {"workload": c.name + " (raw q, k and gate logits; RMS norm and output gate fused)",
+                  "us_per_call": ms * 1e3, "tokens_per_s": c.B * c.T * ws / (ms / 1e3),
+                  "roofline": {"bound": "hbm", "achieved": lb / (ms / 1e3) / 1e9, "peak": hbm_peak, "unit": "GB/s",
+                               "frac": lb / (ms / 1e3) / 1e9 / hbm_peak, "algorithmic_bytes_per_call": lb},
+                  "vs_unfused": (mean_launch_ms * 1e3 + 0.0) / (ms * 1e3),
+                  "l2": f"rotating {N_INPUT_SETS} device input sets"}
+    del lsets
+    if g.gdn2_check_device_error() != g.GDN2_OK:
+        raise RuntimeError("device error while timing the fused layer")
+
     # ---------------- decode: fp32 state resident in HBM, in place ----------------
     dc = DEC
     S = 0.05 * torch.randn(dc.B, dc.H, dc.dk, dc.dv, device=dev)
@@ -494,6 +529,7 @@ def main():
                              "between steps: DRAM bytes per step below the algorithmic bytes)"},
             "workloads": extra,
             "gate_layouts": layouts,
+            "layer_fused": layer_line,
             "decode_tokens": {"workload": "decode state B=256 H=16 d=128 fp32, T tokens per call",
                               "calls": tok_calls},
             "cpu_baseline": cpu,

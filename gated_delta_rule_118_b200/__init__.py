@@ -37,7 +37,7 @@ GDN2_DECAY_SCALAR = 4
 
 # Every symbol include/gdn2.h declares.
 EXPORTED = ("gdn2_fwd_chunked", "gdn2_fwd_chunked_gates", "gdn2_fwd_chunked_noalloc",
-            "gdn2_decode_step", "gdn2_decode_tokens", "gdn2_check_device_error",
+            "gdn2_layer_fwd", "gdn2_decode_step", "gdn2_decode_tokens", "gdn2_check_device_error",
             "gdn2_selftest_bounded_wait", "gdn2_fwd_chunked_launches", "gdn2_status_string")
 
 _lib = None
@@ -64,6 +64,8 @@ def lib() -> ctypes.CDLL:
         L.gdn2_fwd_chunked_gates.restype = ci
         L.gdn2_decode_tokens.argtypes = [vp] * 5 + [fp, fp, vp] + [ci] * 6 + [ctypes.c_uint, vp]
         L.gdn2_decode_tokens.restype = ci
+        L.gdn2_layer_fwd.argtypes = [vp] * 5 + [fp, vp, fp, ctypes.c_float, fp, vp, fp] + [ci] * 6 + [vp]
+        L.gdn2_layer_fwd.restype = ci
         L.gdn2_fwd_chunked_noalloc.argtypes = [vp] * 5 + [fp, fp, vp, fp] + [ci] * 6 + [vp]
         L.gdn2_fwd_chunked_noalloc.restype = ci
         L.gdn2_decode_step.argtypes = [vp] * 5 + [fp, fp, vp] + [ci] * 5 + [vp]
@@ -178,6 +180,33 @@ def gdn2_decode_step(q, k, v, b, w, log_alpha, S, o=None, *, stream=None, check=
     if check and st != GDN2_OK:
         raise Gdn2Error(st, "gdn2_decode_step")
     return o
+
+
+def gdn2_layer_fwd(q, k, v, b_logit, w_logit, decay_logit, g_logit, norm_weight, eps=1e-6, S0=None,
+                   y=None, S_T=None, *, stream=None, want_state=True, check=True):
+    """The operator with the layer's processing fused around it: L2-normalised q and
+    k, sigmoid gates from logits, log_alpha = log sigmoid(decay_logit), and
+    y = RMSNorm(o) * norm_weight * sigmoid(g_logit).  Tensors are CUDA, contiguous,
+    [B,T,H,d] (norm_weight [dv] fp32, decay_logit fp32); returns (y, S_T)."""
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    if y is None:
+        y = torch.empty((B, T, H, dv), dtype=q.dtype, device=q.device)
+    if S_T is None and want_state:
+        S_T = torch.empty((B, H, dk, dv), dtype=torch.float32, device=q.device)
+    for name, t in (("q", q), ("k", k), ("v", v), ("b_logit", b_logit), ("w_logit", w_logit),
+                    ("decay_logit", decay_logit), ("g_logit", g_logit), ("norm_weight", norm_weight),
+                    ("y", y), ("S0", S0), ("S_T", S_T)):
+        if t is not None and not (t.is_cuda and t.is_contiguous()):
+            raise ValueError(f"{name} must be a contiguous CUDA tensor")
+    if decay_logit.dtype != torch.float32 or norm_weight.dtype != torch.float32:
+        raise TypeError("decay_logit and norm_weight must be float32")
+    st = lib().gdn2_layer_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(b_logit), _ptr(w_logit), _ptr(decay_logit),
+                              _ptr(g_logit), _ptr(norm_weight), ctypes.c_float(eps), _ptr(S0), _ptr(y),
+                              _ptr(S_T), B, T, H, dk, dv, _dtype_code(q), _stream(stream))
+    if check and st != GDN2_OK:
+        raise Gdn2Error(st, "gdn2_layer_fwd")
+    return y, S_T
 
 
 def gdn2_decode_tokens(q, k, v, b, w, log_alpha, S, o=None, *, stream=None, check=True):

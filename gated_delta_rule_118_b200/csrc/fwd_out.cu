@@ -21,8 +21,8 @@ struct OutKernelLayout {
 
 template <int DV>
 __global__ void __launch_bounds__(kOutThreads)
-out_kernel(const uint8_t *__restrict__ ws, const uint8_t *__restrict__ sx, bf16 *__restrict__ o, int Tlen,
-           int H, int c0, int WC, unsigned int *err)
+out_kernel(const __grid_constant__ CUtensorMap tm_g, const uint8_t *__restrict__ ws, const uint8_t *__restrict__ sx,
+           bf16 *__restrict__ o, const OutEpi epi, int Tlen, int H, int c0, int WC, unsigned int *err)
 {
     using K = OutKernelLayout<DV>;
     using R = Record<DV>;
@@ -38,7 +38,8 @@ out_kernel(const uint8_t *__restrict__ ws, const uint8_t *__restrict__ sx, bf16 
         mbar_init(bar, 1);
         mbar_init(bar + 1, 1);
         fence_mbar_init();
-        out_issue_loads<DV>(sm, bar, ws + idx * R::BYTES, sx + idx * SxSlot<DV>::BYTES);
+        out_issue_loads<DV>(sm, bar, ws + idx * R::BYTES, sx + idx * SxSlot<DV>::BYTES, epi.g ? &tm_g : nullptr,
+                            (c0 + cw) * kChunk, h, bi);
     }
     if (warp == 0) {
         tmem_alloc(slot, OutLayout<DV>::TMEM_COLS);
@@ -52,8 +53,8 @@ out_kernel(const uint8_t *__restrict__ ws, const uint8_t *__restrict__ sx, bf16 
     const uint32_t tmem = *slot;
     const int ct0 = (c0 + cw) * kChunk;
     uint32_t phase = 0;
-    out_chunk<DV, kOutThreads>(sm, tmem, tid, 0, bar, bar + 1, phase, o + (((long)bi * Tlen + ct0) * H + h) * (long)DV,
-                               Tlen - ct0, (long)H * DV, err);
+    const long row0 = (((long)bi * Tlen + ct0) * H + h) * (long)DV;
+    out_chunk<DV, kOutThreads>(sm, tmem, tid, 0, bar, bar + 1, phase, o + row0, Tlen - ct0, (long)H * DV, epi, err);
     tc_fence_before();
     __syncthreads();
     if (warp == 0) {
@@ -63,8 +64,8 @@ out_kernel(const uint8_t *__restrict__ ws, const uint8_t *__restrict__ sx, bf16 
 }
 
 template <int DV>
-cudaError_t launch_out_impl(const FwdArgs &a, const uint8_t *ws, const uint8_t *sx, int c0, int ncw, int WC,
-                            bool overlap)
+cudaError_t launch_out_impl(const FwdArgs &a, const CUtensorMap *tm_g, const uint8_t *ws, const uint8_t *sx, int c0,
+                            int ncw, int WC, bool overlap)
 {
     using L = OutKernelLayout<DV>;
     auto kern = out_kernel<DV>;
@@ -72,15 +73,17 @@ cudaError_t launch_out_impl(const FwdArgs &a, const uint8_t *ws, const uint8_t *
     cudaError_t e = ensure_smem_limit(kern, L::BYTES, smem_set);
     if (e != cudaSuccess) return e;
     LaunchCfg lc(dim3(ncw, a.H, a.B), dim3(kOutThreads), L::BYTES, a.stream, overlap);
-    return cudaLaunchKernelEx(&lc.cfg, kern, ws, sx, (bf16 *)a.o, a.T, a.H, c0, WC, a.err);
+    const OutEpi epi{a.g, a.norm_weight, a.eps};
+    return cudaLaunchKernelEx(&lc.cfg, kern, *tm_g, ws, sx, (bf16 *)a.o, epi, a.T, a.H, c0, WC, a.err);
 }
 
 }  // namespace
 
-cudaError_t launch_out(const FwdArgs &a, const uint8_t *ws, const uint8_t *sx, int c0, int ncw, int WC, bool overlap)
+cudaError_t launch_out(const FwdArgs &a, const CUtensorMap *tm_g, const uint8_t *ws, const uint8_t *sx, int c0,
+                       int ncw, int WC, bool overlap)
 {
-    return a.dv == 128 ? launch_out_impl<128>(a, ws, sx, c0, ncw, WC, overlap)
-                       : launch_out_impl<64>(a, ws, sx, c0, ncw, WC, overlap);
+    return a.dv == 128 ? launch_out_impl<128>(a, tm_g, ws, sx, c0, ncw, WC, overlap)
+                       : launch_out_impl<64>(a, tm_g, ws, sx, c0, ncw, WC, overlap);
 }
 
 }  // namespace gdn2

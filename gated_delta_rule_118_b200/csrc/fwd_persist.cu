@@ -160,8 +160,9 @@ template <int DV, int DVT>
 __global__ void __launch_bounds__(kPersistThreads, 1)
 persist_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ CUtensorMap tm_la,
+               const __grid_constant__ CUtensorMap tm_g,
                const bf16 *__restrict__ vg, const bf16 *__restrict__ wg, const prep::GateSrc gs,
-               bf16 *__restrict__ o, const float *S0,
+               const outp::OutEpi epi, bf16 *__restrict__ o, const float *S0,
                float *S_T, uint8_t *__restrict__ recs, uint8_t *__restrict__ sxs, uint32_t *flags, int B, int T,
                int H, int nchain, unsigned int *err)
 {
@@ -242,7 +243,8 @@ persist_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                                                  gs.layout);
                         else
                             outp::out_issue_loads<DV>(hs, hb + 2, recs + ((long)r * kRing + slot) * Record<DV>::BYTES,
-                                                      sxs + ((long)r * kRing + slot) * SxSlot<DV>::BYTES);
+                                                      sxs + ((long)r * kRing + slot) * SxSlot<DV>::BYTES,
+                                                      epi.g ? &tm_g : nullptr, c * kChunk, r % H, r / H);
                     }
                 }
             }
@@ -259,9 +261,9 @@ persist_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 tma_phase ^= 1;
             } else {
                 const int t0 = c * kChunk;
-                ok = outp::out_chunk<DV, 256>(hs, ht, lt, bar_id, hb + 2, hb + 3, out_phase,
-                                              o + (((long)bi * T + t0) * H + h) * (long)DV, T - t0, (long)H * DV,
-                                              err);
+                const long row0 = (((long)bi * T + t0) * H + h) * (long)DV;
+                ok = outp::out_chunk<DV, 256>(hs, ht, lt, bar_id, hb + 2, hb + 3, out_phase, o + row0, T - t0,
+                                              (long)H * DV, epi, err);
             }
             // publish: every thread's stores, then one release
             fence_proxy_async_global();
@@ -343,8 +345,10 @@ cudaError_t launch_persist(const FwdArgs &a, const CUtensorMap *maps, uint8_t *w
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     const prep::GateSrc gs{(const bf16 *)a.b, a.log_alpha, a.layout};
-    return cudaLaunchKernelEx(&cfg, kern, maps[0], maps[1], maps[2], maps[3], (const bf16 *)a.v, (const bf16 *)a.w,
-                              gs, (bf16 *)a.o, a.S0, a.S_T, recs, sxs, flags, a.B, a.T, a.H, p.nchain, a.err);
+    const outp::OutEpi epi{a.g, a.norm_weight, a.eps};
+    return cudaLaunchKernelEx(&cfg, kern, maps[0], maps[1], maps[2], maps[3], maps[4], (const bf16 *)a.v,
+                              (const bf16 *)a.w,
+                              gs, epi, (bf16 *)a.o, a.S0, a.S_T, recs, sxs, flags, a.B, a.T, a.H, p.nchain, a.err);
 }
 
 }  // namespace gdn2

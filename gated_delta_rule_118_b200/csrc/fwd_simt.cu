@@ -70,6 +70,8 @@ fwd_simt_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__res
     // gate layouts: b, w or log_alpha may hold one value per (token, head)
     const bool b_scalar = layout & GDN2_ERASE_SCALAR, w_scalar = layout & GDN2_WRITE_SCALAR,
                a_scalar = layout & GDN2_DECAY_SCALAR;
+    // the fused layer's raw inputs: q and k before their L2 norm, gate and decay logits
+    const bool logits = layout & kLayerInputsBit;
 
     for (int idx = tid; idx < DK * DVT; idx += kSimtThreads) {
         const int i = idx / DVT, j = idx % DVT;
@@ -91,6 +93,10 @@ fwd_simt_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__res
                 qv = to_f32(q[off]); kv = to_f32(k[off]);
                 bv = to_f32(b[b_scalar ? tok : off]);
                 la = log_alpha[a_scalar ? tok : off];
+                if (logits) {
+                    bv = 1.f / (1.f + expf(-bv));
+                    la = fminf(la, 0.f) - log1pf(expf(-fabsf(la)));  // log sigmoid
+                }
             }
             sQ[t * LDK + i] = qv; sK[t * LDK + i] = kv; sE[t * LDK + i] = bv; sG[t * LDK + i] = la;
         }
@@ -99,11 +105,22 @@ fwd_simt_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__res
             float z = 0.f;
             if (t < Lc) {
                 const long tok = (bi * Tlen + t0 + t) * H + h, off = tok * DV + j0 + j;
-                z = to_f32(w[w_scalar ? tok : off]) * to_f32(v[off]);
+                const float wv = to_f32(w[w_scalar ? tok : off]);
+                z = (logits ? 1.f / (1.f + expf(-wv)) : wv) * to_f32(v[off]);
             }
             sU[idx] = z;
         }
         __syncthreads();
+        if (logits) {  // L2 norm of each q and k row (rows past the sequence end stay zero)
+            for (int r = tid; r < 2 * C; r += kSimtThreads) {
+                float *row = (r < C ? sQ : sK) + (r % C) * LDK;
+                float ss = 0.f;
+                for (int i = 0; i < DK; ++i) ss = fmaf(row[i], row[i], ss);
+                const float inv = 1.f / sqrtf(ss + 1e-6f);
+                for (int i = 0; i < DK; ++i) row[i] *= inv;
+            }
+            __syncthreads();
+        }
 
         // ---- Gamma: inclusive cumulative log-decay per key channel, fp32 ----
         // The midpoint form is used while every |Gamma_t - Gamma_r| of the chunk
@@ -292,7 +309,55 @@ cudaError_t launch(const FwdArgs &a)
     return cudaGetLastError();
 }
 
+// The fused layer's output processing on the fp32-pipe path, whose CTAs each
+// hold a 32-column slice of the outputs: one warp per (batch, token, head) row,
+// in place: y = o / sqrt(mean(o^2) + eps) * weight * sigmoid(g)
+// ("Gated DeltaNet-2", iplexlaw.co.kr, section "Procesamiento del token y
+// entrenamiento paralelo": RMS normalisation and an output gate).
+template <typename T, int DV>
+__global__ void __launch_bounds__(256)
+layer_epilogue_kernel(T *__restrict__ y, const T *__restrict__ g, const float *__restrict__ weight, float eps,
+                      long rows)
+{
+    constexpr int PER = DV / 32;
+    const long row = (long)blockIdx.x * 8 + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (row >= rows) return;  // whole warps
+    T *yr = y + row * DV;
+    const T *gr = g + row * DV;
+    float x[PER];
+    float ss = 0.f;
+#pragma unroll
+    for (int u = 0; u < PER; ++u) {
+        x[u] = to_f32(yr[lane + 32 * u]);
+        ss = fmaf(x[u], x[u], ss);
+    }
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+    const float inv = rsqrtf(ss * (1.f / DV) + eps);
+#pragma unroll
+    for (int u = 0; u < PER; ++u) {
+        const int j = lane + 32 * u;
+        yr[j] = from_f32<T>(x[u] * inv * weight[j] / (1.f + expf(-to_f32(gr[j]))));
+    }
+}
+
+template <typename T, int DV>
+cudaError_t launch_epi(const FwdArgs &a)
+{
+    const long rows = (long)a.B * a.T * a.H;
+    layer_epilogue_kernel<T, DV><<<(unsigned)((rows + 7) / 8), 256, 0, a.stream>>>((T *)a.o, (const T *)a.g,
+                                                                                  a.norm_weight, a.eps, rows);
+    return cudaGetLastError();
+}
+
 }  // namespace
+
+cudaError_t launch_layer_epilogue_rows(const FwdArgs &a)
+{
+    if (a.bf16) return a.dv == 128 ? launch_epi<__nv_bfloat16, 128>(a) : launch_epi<__nv_bfloat16, 64>(a);
+    return a.dv == 128 ? launch_epi<float, 128>(a) : launch_epi<float, 64>(a);
+}
 
 cudaError_t launch_fwd_simt(const FwdArgs &a)
 {

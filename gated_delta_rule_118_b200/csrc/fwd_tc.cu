@@ -70,17 +70,17 @@ cudaMemPool_t workspace_pool(int dev)
     return pools[dev];
 }
 
-// Tensor maps of the TMA-loaded inputs: q, k, b, log_alpha, and v, w when
-// `n` is 6.  A gate given as one value per (token, head) is loaded without TMA;
-// its slot holds q's map, which the kernels do not use for it.
-bool make_input_maps(const FwdArgs &a, CUtensorMap *maps, int n)
+// Tensor maps of the TMA-loaded inputs: q, k, b, log_alpha and the output-gate
+// logits of the fused layer.  A gate given as one value per (token, head), and
+// an absent output gate, are not loaded by TMA; their slots hold q's map, which
+// the kernels do not use for them.
+bool make_input_maps(const FwdArgs &a, CUtensorMap *maps)
 {
     const auto BF = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
     if (!make_map(&maps[0], a.q, BF, 2, 128, a.H, a.T, a.B, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
         !make_map(&maps[1], a.k, BF, 2, 128, a.H, a.T, a.B, 64, CU_TENSOR_MAP_SWIZZLE_128B))
         return false;
-    maps[2] = maps[0];
-    maps[3] = maps[0];
+    maps[2] = maps[3] = maps[4] = maps[0];
     if (!(a.layout & GDN2_ERASE_SCALAR) &&
         !make_map(&maps[2], a.b, BF, 2, 128, a.H, a.T, a.B, 64, CU_TENSOR_MAP_SWIZZLE_128B))
         return false;
@@ -88,8 +88,7 @@ bool make_input_maps(const FwdArgs &a, CUtensorMap *maps, int n)
         !make_map(&maps[3], a.log_alpha, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, 128, a.H, a.T, a.B, 128,
                   CU_TENSOR_MAP_SWIZZLE_NONE))
         return false;
-    return n < 6 || (make_map(&maps[4], a.v, BF, 2, a.dv, a.H, a.T, a.B, a.dv, CU_TENSOR_MAP_SWIZZLE_NONE) &&
-                     make_map(&maps[5], a.w, BF, 2, a.dv, a.H, a.T, a.B, a.dv, CU_TENSOR_MAP_SWIZZLE_NONE));
+    return !a.g || make_map(&maps[4], a.g, BF, 2, a.dv, a.H, a.T, a.B, 64, CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
 }  // namespace
@@ -132,8 +131,8 @@ FwdTcPlan plan_fwd_tc(int B, int T, int H, int dv, size_t budget, int num_sms)
 
 cudaError_t run_fwd_tc(const FwdArgs &a, const FwdTcPlan &p, uint8_t *ws)
 {
-    CUtensorMap maps[6];
-    if (!make_input_maps(a, maps, 6)) return cudaErrorInvalidValue;
+    CUtensorMap maps[5];
+    if (!make_input_maps(a, maps)) return cudaErrorInvalidValue;
     uint8_t *recs = ws, *sxs = ws + p.rec_total;
     float *carry = p.carry_bytes ? reinterpret_cast<float *>(ws + p.rec_total + p.sx_total) : nullptr;
     for (int w = 0; w < p.nwindows; ++w) {
@@ -143,7 +142,7 @@ cudaError_t run_fwd_tc(const FwdArgs &a, const FwdTcPlan &p, uint8_t *ws)
         float *S_out = (w == p.nwindows - 1) ? a.S_T : carry;
         cudaError_t e = launch_prep(a, maps, recs, c0, ncw, p.wc, false);
         if (e == cudaSuccess) e = launch_chain(a, p.dvt, recs, sxs, S_in, S_out, ncw, p.wc, false);
-        if (e == cudaSuccess) e = launch_out(a, recs, sxs, c0, ncw, p.wc, false);
+        if (e == cudaSuccess) e = launch_out(a, &maps[4], recs, sxs, c0, ncw, p.wc, false);
         if (e != cudaSuccess) return e;
     }
     return cudaSuccess;
@@ -197,8 +196,8 @@ StreamSet *stream_set(int dev)
 // the caller's stream at the start and joins it at the end.
 cudaError_t run_fwd_tc_overlapped(const FwdArgs &a, const FwdTcPlan &p, uint8_t *ws, StreamSet &ss)
 {
-    CUtensorMap maps[6];
-    if (!make_input_maps(a, maps, 6)) return cudaErrorInvalidValue;
+    CUtensorMap maps[5];
+    if (!make_input_maps(a, maps)) return cudaErrorInvalidValue;
     const int nslots = p.slots;
     const size_t slot_bytes = p.rec_total + p.sx_total;
     float *carry = p.carry_bytes ? reinterpret_cast<float *>(ws + nslots * slot_bytes) : nullptr;
@@ -235,7 +234,7 @@ cudaError_t run_fwd_tc_overlapped(const FwdArgs &a, const FwdTcPlan &p, uint8_t 
         if (e == cudaSuccess) e = cudaEventRecord(ss.ev_c[slot], a.stream);
         if (e == cudaSuccess) e = cudaStreamWaitEvent(ss.out, ss.ev_c[slot], 0);
         // output launches of consecutive windows write disjoint rows
-        if (e == cudaSuccess) e = launch_out(ao, recs, sxs, c0, ncw, p.wc, true);
+        if (e == cudaSuccess) e = launch_out(ao, &maps[4], recs, sxs, c0, ncw, p.wc, true);
         if (e == cudaSuccess) e = cudaEventRecord(ss.ev_o[slot], ss.out);
     }
     // join: the caller's stream waits for the last output (the output stream runs
@@ -251,8 +250,8 @@ bool try_fwd_persist(const FwdArgs &a, cudaMemPool_t pool, cudaError_t *status)
 {
     const PersistPlan p = plan_fwd_persist(a.B, a.T, a.H, a.dv, a.num_sms);
     if (!p.use) return false;
-    CUtensorMap maps[4];
-    if (!make_input_maps(a, maps, 4)) {
+    CUtensorMap maps[5];
+    if (!make_input_maps(a, maps)) {
         *status = cudaErrorInvalidValue;
         return true;
     }

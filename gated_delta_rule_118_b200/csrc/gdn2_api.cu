@@ -69,9 +69,18 @@ namespace {
 
 constexpr unsigned kLayoutBits = GDN2_ERASE_SCALAR | GDN2_WRITE_SCALAR | GDN2_DECAY_SCALAR;
 
+// The chunked forward; with `epi` (gdn2_layer_fwd) the inputs are the layer's
+// raw ones and the outputs get the layer's RMS norm and output gate.
+struct LayerEpi {
+    const void *g;
+    const float *weight;
+    float eps;
+};
+
 gdn2_status fwd_chunked(const void *q, const void *k, const void *v, const void *b, const void *w,
                         const float *log_alpha, const float *S0, void *o, float *S_T, int B, int T, int H, int dk,
-                        int dv, gdn2_dtype dtype, unsigned layout, gdn2_stream_t stream)
+                        int dv, gdn2_dtype dtype, unsigned layout, gdn2_stream_t stream,
+                        const LayerEpi *epi = nullptr)
 {
     if (dtype != GDN2_F32 && dtype != GDN2_BF16) return GDN2_ERR_DTYPE;
     if (B <= 0 || H <= 0 || T < 0) return GDN2_ERR_SHAPE;
@@ -79,13 +88,14 @@ gdn2_status fwd_chunked(const void *q, const void *k, const void *v, const void 
     gdn2_status st = check_dims(dk, dv);
     if (st != GDN2_OK) return st;
     if (B > 65535 || H > 65535) return GDN2_ERR_UNSUPPORTED;  // grid y/z limits
-    const void *ins[] = {q, k, v, b, w, log_alpha, o};
+    const void *ins[] = {q, k, v, b, w, log_alpha, o, epi ? epi->g : q, epi ? epi->weight : q};
     if (T > 0)
         for (const void *p : ins)
             if (!p) return GDN2_ERR_NULL;
-    const void *all[] = {q, k, v, b, w, log_alpha, o, S0, S_T};
+    const void *all[] = {q, k, v, b, w, log_alpha, o, S0, S_T, epi ? epi->g : nullptr, epi ? epi->weight : nullptr};
     for (const void *p : all)
         if (p && !aligned16(p)) return GDN2_ERR_ALIGN;
+    if (epi && !(epi->eps >= 0.f)) return GDN2_ERR_SHAPE;
 
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     if (T == 0) {  // nothing to run: S_T = S0 (or zeros)
@@ -104,11 +114,24 @@ gdn2_status fwd_chunked(const void *q, const void *k, const void *v, const void 
     a.bf16 = (dtype == GDN2_BF16);
     a.layout = layout;
     a.stream = s;
+    if (epi) {
+        a.layout |= kLayerInputsBit;
+        a.g = epi->g;
+        a.norm_weight = epi->weight;
+        a.eps = epi->eps;
+    }
     st = device_context(&a.err, &a.num_sms);
     if (st != GDN2_OK) return st;
-    // bf16 inputs with dk = 128 run on the tensor cores; fp32 inputs (and dk = 64)
-    // run on the fp32 pipes, which meet the fp32 tolerance.
-    const cudaError_t e = (a.bf16 && dk == 128) ? launch_fwd_tc(a) : launch_fwd_simt(a);
+    // bf16 inputs with dk = 128 run on the tensor cores (the output processing
+    // inside the output work); fp32 inputs (and dk = 64) run on the fp32 pipes,
+    // which meet the fp32 tolerance, with the output processing as a row kernel.
+    cudaError_t e;
+    if (a.bf16 && dk == 128) {
+        e = launch_fwd_tc(a);
+    } else {
+        e = launch_fwd_simt(a);
+        if (e == cudaSuccess && epi) e = launch_layer_epilogue_rows(a);
+    }
     return e == cudaSuccess ? GDN2_OK : GDN2_ERR_CUDA;
 }
 
@@ -154,6 +177,17 @@ extern "C" gdn2_status gdn2_fwd_chunked_gates(const void *q, const void *k, cons
                                               gdn2_dtype dtype, unsigned int layout, gdn2_stream_t stream)
 {
     return fwd_chunked(q, k, v, b, w, log_alpha, S0, o, S_T, B, T, H, dk, dv, dtype, layout, stream);
+}
+
+extern "C" gdn2_status gdn2_layer_fwd(const void *q, const void *k, const void *v, const void *b_logit,
+                                      const void *w_logit, const float *decay_logit, const void *g_logit,
+                                      const float *norm_weight, float eps, const float *S0, void *y, float *S_T,
+                                      int B, int T, int H, int dk, int dv, gdn2_dtype dtype,
+                                      gdn2_stream_t stream)
+{
+    const LayerEpi epi{g_logit, norm_weight, eps};
+    return fwd_chunked(q, k, v, b_logit, w_logit, decay_logit, S0, y, S_T, B, T, H, dk, dv, dtype, 0u, stream,
+                       &epi);
 }
 
 extern "C" gdn2_status gdn2_decode_step(const void *q, const void *k, const void *v,

@@ -30,11 +30,18 @@ struct FwdArgs {
     float *S_T;       // may be null (not written); may alias S0
     int B, T, H, dk, dv;
     bool bf16;
-    unsigned layout;    // gdn2_gate_layout bits
+    unsigned layout;    // gdn2_gate_layout bits, and kLayerInputs for the fused layer
     cudaStream_t stream;
     unsigned int *err;  // device error word
     int num_sms;
+    // the fused layer's output processing (null g: the operator's plain outputs)
+    const void *g;             // [B][T][H][dv] output-gate logits
+    const float *norm_weight;  // [dv]
+    float eps;
 };
+// FwdArgs::layout bit: q, k and the gates are the layer's raw inputs (gdn2_layer_fwd)
+constexpr unsigned kLayerInputsBit = 8u;
+cudaError_t launch_layer_epilogue_rows(const FwdArgs &a);  // y = RMSNorm(o) * weight * sigmoid(g), in place
 
 bool device_error_word(unsigned int **err);
 cudaError_t launch_decode(const DecodeArgs &a);
@@ -74,8 +81,8 @@ cudaError_t launch_prep(const FwdArgs &a, const CUtensorMap *maps, uint8_t *ws, 
                         bool overlap);
 cudaError_t launch_chain(const FwdArgs &a, int dvt, const uint8_t *ws, uint8_t *sx, const float *S_in,
                          float *S_out, int ncw, int WC, bool overlap);
-cudaError_t launch_out(const FwdArgs &a, const uint8_t *ws, const uint8_t *sx, int c0, int ncw, int WC,
-                       bool overlap);
+cudaError_t launch_out(const FwdArgs &a, const CUtensorMap *tm_g, const uint8_t *ws, const uint8_t *sx, int c0,
+                       int ncw, int WC, bool overlap);
 // Persistent forward (fwd_persist.cu): prep, chain and output work in one
 // cooperative launch of one CTA per SM, records and state images in rings of
 // kRing chunks per (batch, head); the outputs of chunk c are handed out after

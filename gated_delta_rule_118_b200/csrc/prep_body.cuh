@@ -67,12 +67,41 @@ static_assert(PrepLayout::BYTES * 2 + 2048 <= 233472, "two CTAs per SM");
 // `layout`); per-channel ones arrive by TMA.  Scalar b and log_alpha are
 // broadcast over the channels of their rows in shared memory, so everything
 // after the loads is the same for every layout.
+//
+// With kLayerInputs (gdn2_layer_fwd) the loaded tiles are the layer's raw
+// inputs -- q and k before their L2 normalisation, and the logits of the erase
+// gate, the write gate and the decay -- and the prep turns them into the
+// operator's inputs in place ("Gated DeltaNet-2", iplexlaw.co.kr, section
+// "Procesamiento del token y entrenamiento paralelo": L2-normalised queries and
+// keys, sigmoid gates): q / sqrt(|q|^2 + 1e-6), k likewise, b = sigmoid(.),
+// w = sigmoid(.), log_alpha = log sigmoid(.).
 struct GateSrc {
     const bf16 *b;     // [B][T][H] with GDN2_ERASE_SCALAR
     const float *la;   // [B][T][H] with GDN2_DECAY_SCALAR
     unsigned layout;
 };
 constexpr unsigned kEraseScalar = 1u, kWriteScalar = 2u, kDecayScalar = 4u;  // gdn2_gate_layout bits
+constexpr unsigned kLayerInputs = 8u;  // raw q, k and gate logits (the fused layer entry point)
+constexpr float kL2Eps = 1e-6f;
+
+// sigmoid(x) = (1 + tanh(x / 2)) / 2, one MUFU operation (tanh.approx.f32,
+// relative error about 2^-11: below the bf16 rounding of the gates)
+__device__ __forceinline__ float sigmoid_f(float x)
+{
+    float t;
+    asm("tanh.approx.f32 %0, %1;" : "=f"(t) : "f"(0.5f * x));
+    return fmaf(0.5f, t, 0.5f);
+}
+// log(sigmoid(x)) = min(x, 0) - log(1 + y), y = e^{-|x|} in (0, 1], finite for
+// every finite x.  For y < 2^-10 the log is its series y - y^2/2 (the next term,
+// y^3/3, is below 4e-7 of the result): a decay near 1 keeps its small log,
+// which a rounded 1 + y would lose.
+__device__ __forceinline__ float log_sigmoid_f(float x)
+{
+    const float y = __expf(-fabsf(x));
+    const float l = y < 0.0009765625f ? y * (1.f - 0.5f * y) : __logf(1.f + y);
+    return fminf(x, 0.f) - l;
+}
 
 __device__ __forceinline__ void tmem_ld32_wait(uint32_t taddr, float (&r)[32])
 {
@@ -130,23 +159,33 @@ __device__ __forceinline__ bool prep_chunk(uint8_t *sm, uint32_t tmem, int tid, 
     // (tokens past the sequence end give zero rows of Z)
     constexpr int ZV = 64 * DV / 8 / kPrepThreads;  // 16-byte vectors per thread
     uint4 vv[ZV], wv[ZV];
+    auto load_vw = [&]() {
 #pragma unroll
-    for (int m = 0; m < ZV; ++m) {
-        const int idx = tid + m * kPrepThreads;
-        const int t = idx / (DV / 8), j = (idx % (DV / 8)) * 8;
-        vv[m] = make_uint4(0, 0, 0, 0);
-        wv[m] = make_uint4(0, 0, 0, 0);
-        if (t < Lc) {
-            const long tok = ((long)bi * Tlen + t0 + t) * H + h, off = tok * DV + j;
-            vv[m] = __ldg(reinterpret_cast<const uint4 *>(vg + off));
-            if (gs.layout & kWriteScalar) {
-                const uint32_t two = (uint32_t)__bfloat16_as_ushort(wg[tok]) * 0x10001u;
-                wv[m] = make_uint4(two, two, two, two);
-            } else {
-                wv[m] = __ldg(reinterpret_cast<const uint4 *>(wg + off));
+        for (int m = 0; m < ZV; ++m) {
+            const int idx = tid + m * kPrepThreads;
+            const int t = idx / (DV / 8), j = (idx % (DV / 8)) * 8;
+            vv[m] = make_uint4(0, 0, 0, 0);
+            wv[m] = make_uint4(0, 0, 0, 0);
+            if (t < Lc) {
+                const long tok = ((long)bi * Tlen + t0 + t) * H + h, off = tok * DV + j;
+                vv[m] = __ldg(reinterpret_cast<const uint4 *>(vg + off));
+                if (gs.layout & kWriteScalar) {  // (a logit, with kLayerInputs: turned into a gate below)
+                    const uint32_t two = (uint32_t)__bfloat16_as_ushort(wg[tok]) * 0x10001u;
+                    wv[m] = make_uint4(two, two, two, two);
+                } else {
+                    wv[m] = __ldg(reinterpret_cast<const uint4 *>(wg + off));
+                }
+                if (gs.layout & kLayerInputs) {  // write gate from its logits
+                    float f[8];
+                    unpack8(wv[m], f);
+#pragma unroll
+                    for (int u = 0; u < 8; ++u) f[u] = sigmoid_f(f[u]);
+                    wv[m] = pack8(f);
+                }
             }
         }
-    }
+    };
+    load_vw();
     // scalar b / log_alpha: row t of the b tile (both 64-channel halves) and of
     // log_alpha filled with the token's value (zero past the sequence end), into
     // buffers the TMA leaves alone in these layouts
@@ -154,19 +193,22 @@ __device__ __forceinline__ bool prep_chunk(uint8_t *sm, uint32_t tmem, int tid, 
         const int t = tid >> 2, part = tid & 3;
         const long tok = ((long)bi * Tlen + t0 + t) * H + h;
         if (gs.layout & kEraseScalar) {
-            const uint32_t two = t < Lc ? (uint32_t)__bfloat16_as_ushort(gs.b[tok]) * 0x10001u : 0u;
+            bf16 bt = t < Lc ? gs.b[tok] : __float2bfloat16_rn(0.f);
+            if (gs.layout & kLayerInputs) bt = __float2bfloat16_rn(sigmoid_f(__bfloat162float(bt)));
+            const uint32_t two = (uint32_t)__bfloat16_as_ushort(bt) * 0x10001u;
 #pragma unroll
             for (int m = 0; m < 4; ++m) {
-                const int c = part * 4 + m;  // 16-byte piece of the token's 256 bytes
+                const int c = part * 4 + ((m + t) & 3);  // 16-byte piece of the token's 256 bytes (rotated)
                 *reinterpret_cast<uint4 *>(sm + L::EQ + (c >> 3) * 16384 + t * 128 + (c & 7) * 16) =
                     make_uint4(two, two, two, two);
             }
         }
         if (gs.layout & kDecayScalar) {
-            const float lt = t < Lc ? gs.la[tok] : 0.f;
+            const float lt = t < Lc ? ((gs.layout & kLayerInputs) ? log_sigmoid_f(gs.la[tok]) : gs.la[tok]) : 0.f;
 #pragma unroll
             for (int m = 0; m < 8; ++m)
-                *reinterpret_cast<float4 *>(sm + L::LA + t * 512 + part * 128 + m * 16) = make_float4(lt, lt, lt, lt);
+                *reinterpret_cast<float4 *>(sm + L::LA + t * 512 + part * 128 + ((m + t) & 7) * 16) =
+                    make_float4(lt, lt, lt, lt);
         }
     }
     // One thread polls each mbarrier; the others park on the group's barrier,
@@ -180,6 +222,61 @@ __device__ __forceinline__ bool prep_chunk(uint8_t *sm, uint32_t tmem, int tid, 
         return all;
     };
     bool ok = named_bar_and(bar_id, kPrepThreads, (tid == 0) ? mbar_wait(bar_tma, tma_phase, err) : true) != 0;
+
+    if (ok && (gs.layout & kLayerInputs)) {
+        // ---------------------------------------------------------- the layer's input processing
+        {   // L2 norm of each q and k row: two threads per row, one 64-channel half each
+            const int r = tid >> 1, half = tid & 1, t = r & 63;
+            uint8_t *row = (r < 64) ? sm + L::EQ + half * 16384 + 8192 + t * 128 : sm + L::KT + half * 8192 + t * 128;
+            // the row's 16-byte pieces in an order rotated by the row, so that the
+            // lanes of a warp (16 rows) spread over the banks
+            float ss = 0.f;
+#pragma unroll 2
+            for (int c = 0; c < 8; ++c) {
+                float x[8];
+                unpack8(*reinterpret_cast<const uint4 *>(row + 16 * ((c + t) & 7)), x);
+#pragma unroll
+                for (int u = 0; u < 8; ++u) ss = fmaf(x[u], x[u], ss);
+            }
+            ss += __shfl_xor_sync(0xffffffffu, ss, 1);
+            const float inv = rsqrtf(ss + kL2Eps);
+#pragma unroll 2
+            for (int c = 0; c < 8; ++c) {
+                float x[8];
+                uint4 *pp = reinterpret_cast<uint4 *>(row + 16 * ((c + t) & 7));
+                unpack8(*pp, x);
+#pragma unroll
+                for (int u = 0; u < 8; ++u) x[u] *= inv;
+                *pp = pack8(x);
+            }
+        }
+        if (!(gs.layout & kEraseScalar) || !(gs.layout & kDecayScalar)) {
+            const int t = tid >> 2, part = tid & 3;  // token, quarter of its channels
+            if (!(gs.layout & kEraseScalar)) {   // erase gate from its logits (row t of both half tiles)
+#pragma unroll 1
+                for (int m = 0; m < 4; ++m) {
+                    const int c = part * 4 + ((m + t) & 3);  // rotated by the row: bank spread
+                    uint4 *pp = reinterpret_cast<uint4 *>(sm + L::EQ + (c >> 3) * 16384 + t * 128 + (c & 7) * 16);
+                    float f[8];
+                    unpack8(*pp, f);
+#pragma unroll
+                    for (int u = 0; u < 8; ++u) f[u] = sigmoid_f(f[u]);
+                    *pp = pack8(f);
+                }
+            }
+            if (!(gs.layout & kDecayScalar)) {   // log-decay from its logits; none past the sequence end
+#pragma unroll 2
+                for (int m = 0; m < 8; ++m) {
+                    float4 *pp = reinterpret_cast<float4 *>(sm + L::LA + t * 512 + part * 128 + ((m + t) & 7) * 16);
+                    const float4 x = *pp;
+                    *pp = t < Lc ? make_float4(log_sigmoid_f(x.x), log_sigmoid_f(x.y), log_sigmoid_f(x.z),
+                                               log_sigmoid_f(x.w))
+                                 : make_float4(0.f, 0.f, 0.f, 0.f);
+                }
+            }
+        }
+        named_bar(bar_id, kPrepThreads);
+    }
 
     // Z = w v, straight into the record (MN-major operand blocks of 64 value
     // columns; each warp fills whole 128-byte rows)

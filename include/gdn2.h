@@ -223,6 +223,43 @@ gdn2_status gdn2_fwd_chunked_gates(const void *q, const void *k, const void *v,
                                    gdn2_dtype dtype, unsigned int layout, gdn2_stream_t stream);
 
 /*
+ * gdn2_layer_fwd -- the chunked forward with the layer's processing around the
+ * operator fused into its kernels ("Gated DeltaNet-2", iplexlaw.co.kr, section
+ * "Procesamiento del token y entrenamiento paralelo": queries and keys are
+ * L2-normalised, the gates come through sigmoids, and the recurrent output
+ * receives RMS normalisation and an independent output gate before the output
+ * projection).  The projections, the short convolution and the SiLU stay with
+ * the caller.  Per (batch, token, head):
+ *
+ *     q_hat = q / sqrt(|q|^2 + 1e-6),  k_hat = k / sqrt(|k|^2 + 1e-6)
+ *     b = sigmoid(b_logit),  w = sigmoid(w_logit),  log_alpha = log sigmoid(decay_logit)
+ *     o, S_T = the operator of gdn2_fwd_chunked on (q_hat, k_hat, v, b, w, log_alpha, S0)
+ *     y = o / sqrt(mean_j o_j^2 + eps) * norm_weight * sigmoid(g_logit)
+ *
+ * The pages name neither the decay's activation nor the output gate's, nor the
+ * epsilons: this library reads both activations as the sigmoid the pages give
+ * for the erase and write gates.  o never reaches device memory: y is formed
+ * from the fp32 accumulators (bf16 inputs, dk = 128) or by a row kernel after
+ * the operator (other inputs).
+ *
+ *   q, k                 [B][T][H][dk]  dtype   before the L2 norm
+ *   v                    [B][T][H][dv]  dtype
+ *   b_logit              [B][T][H][dk]  dtype
+ *   w_logit, g_logit     [B][T][H][dv]  dtype
+ *   decay_logit          [B][T][H][dk]  fp32
+ *   norm_weight          [dv]           fp32   RMS-norm weight
+ *   eps                  >= 0                  RMS-norm epsilon
+ *   S0, S_T, B, T, H, dk, dv, dtype, stream    as for gdn2_fwd_chunked
+ *   y                    [B][T][H][dv]  dtype   written
+ */
+gdn2_status gdn2_layer_fwd(const void *q, const void *k, const void *v,
+                           const void *b_logit, const void *w_logit, const float *decay_logit,
+                           const void *g_logit, const float *norm_weight, float eps,
+                           const float *S0, void *y, float *S_T,
+                           int B, int T, int H, int dk, int dv,
+                           gdn2_dtype dtype, gdn2_stream_t stream);
+
+/*
  * gdn2_check_device_error -- wait for `stream`, then read and clear the
  * device error word of the current device.  Returns GDN2_OK,
  * GDN2_ERR_DEVICE_TIMEOUT or GDN2_ERR_CUDA.

@@ -186,3 +186,30 @@ def scalar_gates(d, layout, *, seed, gate_sigma=1.0):
     if layout & 4:
         out["log_alpha"] = (-torch.exp(torch.rand(B, T, H, generator=g) * 4.0 - 5.0)).contiguous()
     return out
+
+
+def draw_layer(B, T, H, dk, dv, *, seed, dtype=torch.float32, s0_sigma=0.0):
+    """Inputs of the fused layer entry point: q, k and v as they leave the
+    layer's convolution and SiLU (no L2 normalisation), pre-sigmoid logits for
+    the erase, write, decay and output gates, and the RMS-norm weight.  Logit
+    scales put the gates and alpha = sigmoid(decay_logit) across (0, 1), with
+    decays near 1 (as the workloads' log_alpha = -exp(U(-5, -1))) and a spread
+    of faster ones.  Returns a dict of CPU tensors (logits of the decay and the
+    weight in fp32, the rest in ``dtype``)."""
+    g = torch.Generator(device="cpu").manual_seed(int(seed))
+    silu = torch.nn.functional.silu
+    q = silu(torch.randn(B, T, H, dk, generator=g))
+    k = silu(torch.randn(B, T, H, dk, generator=g))
+    v = silu(torch.randn(B, T, H, dv, generator=g))
+    b_logit = torch.randn(B, T, H, dk, generator=g)
+    w_logit = torch.randn(B, T, H, dv, generator=g)
+    decay_logit = 2.0 + 2.5 * torch.randn(B, T, H, dk, generator=g)
+    g_logit = torch.randn(B, T, H, dv, generator=g)
+    norm_weight = 1.0 + 0.1 * torch.randn(dv, generator=g)
+    S0 = s0_sigma * torch.randn(B, H, dk, dv, generator=g) if s0_sigma > 0 else None
+    out = {n: t.to(dtype).contiguous() for n, t in
+           dict(q=q, k=k, v=v, b_logit=b_logit, w_logit=w_logit, g_logit=g_logit).items()}
+    out["decay_logit"] = decay_logit.contiguous()
+    out["norm_weight"] = norm_weight.contiguous()
+    out["S0"] = S0
+    return out

@@ -150,3 +150,14 @@ def test_gate_layout_from_shapes():
     assert g._gate_layout(q, tok, tok, per_ch) == g.GDN2_ERASE_SCALAR | g.GDN2_WRITE_SCALAR
     assert g._gate_layout(q, tok, tok, tok) == 7
     assert g._gate_layout(q, per_ch, tok, per_ch) == g.GDN2_WRITE_SCALAR
+
+
+def test_layer_fwd_rejects_bad_arguments(lib):
+    import ctypes as ct
+    f = lambda **kw: lib.gdn2_layer_fwd(P, P, P, P, P, P, kw.get("g", P), kw.get("nw", P),
+                                        ct.c_float(kw.get("eps", 1e-6)), None, P, None,
+                                        1, 8, 2, 64, 64, 1, None)
+    assert f(g=None) == g.GDN2_ERR_NULL
+    assert f(nw=None) == g.GDN2_ERR_NULL
+    assert f(g=MIS) == g.GDN2_ERR_ALIGN
+    assert f(eps=-1.0) == g.GDN2_ERR_SHAPE
