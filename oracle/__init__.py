@@ -46,6 +46,8 @@ class Oracle:
         dp = ctypes.POINTER(ctypes.c_double)
         self._lib.gdn2_oracle_fwd.argtypes = [dp] * 9 + [ctypes.c_int] * 6
         self._lib.gdn2_oracle_fwd.restype = ctypes.c_int
+        self._lib.gdn2_oracle_bwd.argtypes = [dp] * 16 + [ctypes.c_int] * 6
+        self._lib.gdn2_oracle_bwd.restype = ctypes.c_int
         self._lib.gdn2_oracle_max_threads.argtypes = []
         self._lib.gdn2_oracle_max_threads.restype = ctypes.c_int
 
@@ -92,6 +94,32 @@ class Oracle:
             raise RuntimeError(f"gdn2_oracle_fwd failed with code {rc}")
         return o, st
 
+    def bwd(self, q, k, v, b, w, log_alpha, S0, dO, dS_T=None, nthreads: int = 0):
+        """Gradients of sum(o * dO) + sum(S_T * dS_T) (backpropagation through
+        the recurrence, fp64): returns dict dq, dk, dv, db, dw, dlog_alpha, dS0."""
+        q, k, v, b, w, la, dO = (self._f64(a) for a in (q, k, v, b, w, log_alpha, dO))
+        B, T, H, dk = q.shape
+        dv = v.shape[-1]
+        if dO.shape != (B, T, H, dv):
+            raise ValueError(f"dO has shape {dO.shape}")
+        s0 = None if S0 is None else self._f64(S0)
+        dst = None if dS_T is None else self._f64(dS_T)
+        out = {n: np.zeros((B, T, H, dk)) for n in ("dq", "dk", "db", "dlog_alpha")}
+        out.update({n: np.zeros((B, T, H, dv)) for n in ("dv", "dw")})
+        out["dS0"] = np.zeros((B, H, dk, dv))
+        dp = ctypes.POINTER(ctypes.c_double)
+
+        def ptr(a):
+            return a.ctypes.data_as(dp) if a is not None else None
+
+        rc = self._lib.gdn2_oracle_bwd(ptr(q), ptr(k), ptr(v), ptr(b), ptr(w), ptr(la), ptr(s0), ptr(dO),
+                                       ptr(dst), ptr(out["dq"]), ptr(out["dk"]), ptr(out["dv"]), ptr(out["db"]),
+                                       ptr(out["dw"]), ptr(out["dlog_alpha"]), ptr(out["dS0"]),
+                                       B, T, H, dk, dv, int(nthreads))
+        if rc != 0:
+            raise RuntimeError(f"gdn2_oracle_bwd failed with code {rc}")
+        return out
+
     def decode_step(self, q, k, v, b, w, log_alpha, S, nthreads: int = 0):
         """One token of the recurrence: [B,H,d] inputs and state -> (o, S_new)."""
         ins = [self._f64(a)[:, None] for a in (q, k, v, b, w, log_alpha)]
@@ -120,6 +148,10 @@ def fwd(*args, **kwargs):
 
 def decode_step(*args, **kwargs):
     return load().decode_step(*args, **kwargs)
+
+
+def bwd(*args, **kwargs):
+    return load().bwd(*args, **kwargs)
 
 
 def host_cores() -> int:
