@@ -37,7 +37,7 @@ GDN2_DECAY_SCALAR = 4
 
 # Every symbol include/gdn2.h declares.
 EXPORTED = ("gdn2_fwd_chunked", "gdn2_fwd_chunked_gates", "gdn2_fwd_chunked_noalloc",
-            "gdn2_layer_fwd", "gdn2_decode_step", "gdn2_decode_tokens", "gdn2_check_device_error",
+            "gdn2_layer_fwd", "gdn2_bwd_chunked", "gdn2_decode_step", "gdn2_decode_tokens", "gdn2_check_device_error",
             "gdn2_selftest_bounded_wait", "gdn2_fwd_chunked_launches", "gdn2_status_string")
 
 _lib = None
@@ -66,6 +66,8 @@ def lib() -> ctypes.CDLL:
         L.gdn2_decode_tokens.restype = ci
         L.gdn2_layer_fwd.argtypes = [vp] * 5 + [fp, vp, fp, ctypes.c_float, fp, vp, fp] + [ci] * 6 + [vp]
         L.gdn2_layer_fwd.restype = ci
+        L.gdn2_bwd_chunked.argtypes = [vp] * 5 + [fp, fp, vp, fp] + [fp] * 7 + [ci] * 6 + [vp]
+        L.gdn2_bwd_chunked.restype = ci
         L.gdn2_fwd_chunked_noalloc.argtypes = [vp] * 5 + [fp, fp, vp, fp] + [ci] * 6 + [vp]
         L.gdn2_fwd_chunked_noalloc.restype = ci
         L.gdn2_decode_step.argtypes = [vp] * 5 + [fp, fp, vp] + [ci] * 5 + [vp]
@@ -207,6 +209,31 @@ def gdn2_layer_fwd(q, k, v, b_logit, w_logit, decay_logit, g_logit, norm_weight,
     if check and st != GDN2_OK:
         raise Gdn2Error(st, "gdn2_layer_fwd")
     return y, S_T
+
+
+def gdn2_bwd_chunked(q, k, v, b, w, log_alpha, S0, dO, dS_T=None, *, stream=None, check=True,
+                     want_dS0=True):
+    """Backward of the chunked forward: gradients of sum(o * dO) + sum(S_T * dS_T).
+    Inputs as for gdn2_fwd_chunked plus dO [B,T,H,dv] (input dtype) and dS_T
+    [B,H,dk,dv] fp32 or None; returns a dict of fp32 tensors dq, dk, dv, db, dw,
+    dlog_alpha and dS0 (None unless want_dS0)."""
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    f32 = dict(dtype=torch.float32, device=q.device)
+    g = {n: torch.empty((B, T, H, dk), **f32) for n in ("dq", "dk", "db", "dlog_alpha")}
+    g.update({n: torch.empty((B, T, H, dv), **f32) for n in ("dv", "dw")})
+    g["dS0"] = torch.empty((B, H, dk, dv), **f32) if want_dS0 else None
+    for name, t in (("q", q), ("k", k), ("v", v), ("b", b), ("w", w), ("log_alpha", log_alpha),
+                    ("S0", S0), ("dO", dO), ("dS_T", dS_T)):
+        if t is not None and not (t.is_cuda and t.is_contiguous()):
+            raise ValueError(f"{name} must be a contiguous CUDA tensor")
+    st = lib().gdn2_bwd_chunked(_ptr(q), _ptr(k), _ptr(v), _ptr(b), _ptr(w), _ptr(log_alpha), _ptr(S0),
+                                _ptr(dO), _ptr(dS_T), _ptr(g["dq"]), _ptr(g["dk"]), _ptr(g["dv"]),
+                                _ptr(g["db"]), _ptr(g["dw"]), _ptr(g["dlog_alpha"]), _ptr(g["dS0"]),
+                                B, T, H, dk, dv, _dtype_code(q), _stream(stream))
+    if check and st != GDN2_OK:
+        raise Gdn2Error(st, "gdn2_bwd_chunked")
+    return g
 
 
 def gdn2_decode_tokens(q, k, v, b, w, log_alpha, S, o=None, *, stream=None, check=True):

@@ -50,6 +50,8 @@ bool make_map(CUtensorMap *m, const void *base, CUtensorMapDataType dt, int esiz
 }
 
 // Stream-ordered pool for the workspace; it keeps freed blocks for reuse.
+}  // namespace
+
 cudaMemPool_t workspace_pool(int dev)
 {
     static std::mutex mu;
@@ -69,6 +71,8 @@ cudaMemPool_t workspace_pool(int dev)
     }
     return pools[dev];
 }
+
+namespace {
 
 // Tensor maps of the TMA-loaded inputs: q, k, b, log_alpha and the output-gate
 // logits of the fused layer.  A gate given as one value per (token, head), and

@@ -190,6 +190,63 @@ extern "C" gdn2_status gdn2_layer_fwd(const void *q, const void *k, const void *
                        &epi);
 }
 
+extern "C" gdn2_status gdn2_bwd_chunked(const void *q, const void *k, const void *v, const void *b, const void *w,
+                                        const float *log_alpha, const float *S0, const void *dO,
+                                        const float *dS_T, float *dq, float *dk_, float *dv_, float *db, float *dw,
+                                        float *dlog_alpha, float *dS0, int B, int T, int H, int dk, int dv,
+                                        gdn2_dtype dtype, gdn2_stream_t stream)
+{
+    if (dtype != GDN2_F32 && dtype != GDN2_BF16) return GDN2_ERR_DTYPE;
+    if (B <= 0 || H <= 0 || T < 0) return GDN2_ERR_SHAPE;
+    gdn2_status st = check_dims(dk, dv);
+    if (st != GDN2_OK) return st;
+    if (B > 65535 || H > 65535) return GDN2_ERR_UNSUPPORTED;
+    const void *req[] = {q, k, v, b, w, log_alpha, dO, dq, dk_, dv_, db, dw, dlog_alpha};
+    if (T > 0)
+        for (const void *p : req)
+            if (!p) return GDN2_ERR_NULL;
+    const void *all[] = {q, k, v, b, w, log_alpha, dO, dq, dk_, dv_, db, dw, dlog_alpha, S0, dS_T, dS0};
+    for (const void *p : all)
+        if (p && !aligned16(p)) return GDN2_ERR_ALIGN;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const size_t DD = sizeof(float) * (size_t)dk * dv;
+    if (T == 0) {  // o is empty and S_T = S0: dS0 = dS_T
+        if (!dS0) return GDN2_OK;
+        cudaError_t e = dS_T ? cudaMemcpyAsync(dS0, dS_T, DD * B * H, cudaMemcpyDeviceToDevice, s)
+                             : cudaMemsetAsync(dS0, 0, DD * B * H, s);
+        return e == cudaSuccess ? GDN2_OK : GDN2_ERR_CUDA;
+    }
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return GDN2_ERR_CUDA;
+    cudaMemPool_t pool = workspace_pool(dev);
+    if (!pool) return GDN2_ERR_CUDA;
+    // the forward's state entering every chunk (and S_T): the backward's checkpoints
+    const long nch = (T + kChunk - 1) / kChunk;
+    void *ckpt = nullptr;
+    cudaError_t e = cudaMallocFromPoolAsync(&ckpt, DD * B * H * (size_t)(nch + 1), pool, s);
+    if (e != cudaSuccess) return GDN2_ERR_CUDA;
+    const size_t nk = sizeof(float) * (size_t)B * T * H * dk;
+    for (float *p : {dq, dk_, db, dlog_alpha})
+        if (e == cudaSuccess) e = cudaMemsetAsync(p, 0, nk, s);
+    FwdArgs f{};
+    f.q = q; f.k = k; f.v = v; f.b = b; f.w = w; f.log_alpha = log_alpha;
+    f.S0 = S0; f.o = nullptr; f.S_T = nullptr;
+    f.B = B; f.T = T; f.H = H; f.dk = dk; f.dv = dv;
+    f.bf16 = (dtype == GDN2_BF16);
+    f.stream = s;
+    if (e == cudaSuccess) e = launch_fwd_simt_checkpoints(f, static_cast<float *>(ckpt));
+    BwdArgs a{};
+    a.q = q; a.k = k; a.v = v; a.b = b; a.w = w; a.log_alpha = log_alpha;
+    a.dO = dO; a.dS_T = dS_T; a.ckpt = static_cast<const float *>(ckpt);
+    a.gq = dq; a.gk = dk_; a.gv = dv_; a.gb = db; a.gw = dw; a.gla = dlog_alpha; a.dS0 = dS0;
+    a.B = B; a.T = T; a.H = H; a.dk = dk; a.dv = dv;
+    a.bf16 = f.bf16;
+    a.stream = s;
+    if (e == cudaSuccess) e = launch_bwd_simt(a);
+    const cudaError_t fe = cudaFreeAsync(ckpt, s);
+    return (e == cudaSuccess && fe == cudaSuccess) ? GDN2_OK : GDN2_ERR_CUDA;
+}
+
 extern "C" gdn2_status gdn2_decode_step(const void *q, const void *k, const void *v,
                                         const void *b, const void *w, const float *log_alpha,
                                         float *S, void *o, int B, int H, int dk, int dv,

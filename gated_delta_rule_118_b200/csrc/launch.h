@@ -43,6 +43,26 @@ struct FwdArgs {
 constexpr unsigned kLayerInputsBit = 8u;
 cudaError_t launch_layer_epilogue_rows(const FwdArgs &a);  // y = RMSNorm(o) * weight * sigmoid(g), in place
 
+// Chunkwise backward (bwd_simt.cu): gradients of sum(o * dO) + sum(S_T * dS_T).
+struct BwdArgs {
+    const void *q, *k, *v, *b, *w;
+    const float *log_alpha;
+    const void *dO;
+    const float *dS_T;   // may be null (zero)
+    const float *ckpt;   // [B][H][nchunks + 1][dk][dv] fp32: the state entering each chunk, and S_T
+    float *gq, *gk, *gv, *gb, *gw, *gla;   // fp32 gradients; gq, gk, gb, gla zeroed before the launch (atomics)
+    float *dS0;          // may be null (not written)
+    int B, T, H, dk, dv;
+    bool bf16;
+    cudaStream_t stream;
+};
+cudaError_t launch_bwd_simt(const BwdArgs &a);
+// The fp32-pipe forward writing the state entering every chunk (and the final
+// state) to `ckpt` ([B][H][nchunks + 1][dk][dv]); outputs are not written.
+cudaError_t launch_fwd_simt_checkpoints(const FwdArgs &a, float *ckpt);
+// The library's stream-ordered workspace pool of a device (keeps freed blocks).
+cudaMemPool_t workspace_pool(int dev);
+
 bool device_error_word(unsigned int **err);
 cudaError_t launch_decode(const DecodeArgs &a);
 cudaError_t launch_fwd_simt(const FwdArgs &a);

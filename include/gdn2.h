@@ -260,6 +260,36 @@ gdn2_status gdn2_layer_fwd(const void *q, const void *k, const void *v,
                            gdn2_dtype dtype, gdn2_stream_t stream);
 
 /*
+ * gdn2_bwd_chunked -- the backward of gdn2_fwd_chunked: gradients of
+ * L = sum(o * dO) + sum(S_T * dS_T) with respect to every input, chunkwise
+ * over 64-token chunks in reverse ("Gated DeltaNet-2", iplexlaw.co.kr, section
+ * "Procesamiento del token y entrenamiento paralelo": the WY form's backward
+ * must use the modulated keys and values, the per-channel gates staying inside
+ * the gradient aggregation).  b and w get gradients of their own, per channel.
+ * The forward is recomputed first (its chunk-entry states are the backward's
+ * checkpoints, held in a workspace from the library's pool); all arithmetic is
+ * fp32 on the CUDA cores, and every decay between two tokens is a running
+ * product of alpha, so any log_alpha <= 0 is handled.
+ *
+ *   q, k, v, b, w, log_alpha, S0, B, T, H, dk, dv, dtype   as for gdn2_fwd_chunked
+ *   dO          [B][T][H][dv]  dtype   incoming gradient of o
+ *   dS_T        [B][H][dk][dv] fp32    incoming gradient of S_T; NULL means zero
+ *   dq, dk, db, dlog_alpha  [B][T][H][dk]  fp32   written
+ *   dv, dw                  [B][T][H][dv]  fp32   written
+ *   dS0         [B][H][dk][dv] fp32    written; NULL means not wanted
+ *
+ * The key-axis gradients are sums over the value columns, added across column
+ * tiles with fp32 atomics: their last bits may differ from run to run.
+ */
+gdn2_status gdn2_bwd_chunked(const void *q, const void *k, const void *v,
+                             const void *b, const void *w, const float *log_alpha,
+                             const float *S0, const void *dO, const float *dS_T,
+                             float *dq, float *dk, float *dv, float *db, float *dw,
+                             float *dlog_alpha, float *dS0,
+                             int B, int T, int H, int dk_, int dv_,
+                             gdn2_dtype dtype, gdn2_stream_t stream);
+
+/*
  * gdn2_check_device_error -- wait for `stream`, then read and clear the
  * device error word of the current device.  Returns GDN2_OK,
  * GDN2_ERR_DEVICE_TIMEOUT or GDN2_ERR_CUDA.

@@ -161,3 +161,14 @@ def test_layer_fwd_rejects_bad_arguments(lib):
     assert f(nw=None) == g.GDN2_ERR_NULL
     assert f(g=MIS) == g.GDN2_ERR_ALIGN
     assert f(eps=-1.0) == g.GDN2_ERR_SHAPE
+
+
+def test_bwd_rejects_bad_arguments(lib):
+    f = lambda **kw: lib.gdn2_bwd_chunked(P, P, P, P, P, P, None, kw.get("dO", P), None, P, P, P, P, P,
+                                          kw.get("dla", P), None, kw.get("B", 1), 8, 2, kw.get("dk", 64), 64,
+                                          kw.get("dtype", 1), None)
+    assert f(dO=None) == g.GDN2_ERR_NULL
+    assert f(dla=MIS) == g.GDN2_ERR_ALIGN
+    assert f(B=0) == g.GDN2_ERR_SHAPE
+    assert f(dk=32) == g.GDN2_ERR_UNSUPPORTED
+    assert f(dtype=9) == g.GDN2_ERR_DTYPE
