@@ -45,7 +45,7 @@ __global__ void __launch_bounds__(kSimtThreads)
 fwd_simt_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__ v,
                 const T *__restrict__ b, const T *__restrict__ w,
                 const float *__restrict__ log_alpha, const float *S0, T *__restrict__ o,
-                float *S_T, int Tlen, int H, int DV, unsigned layout, float *__restrict__ ckpt)
+                float *S_T, int Tlen, int H, int DV, unsigned layout)
 {
     using L = SimtSmem<DK, DVT>;
     constexpr int C = kChunk, LDK = L::LDK, LDC = L::LDC;
@@ -83,11 +83,6 @@ fwd_simt_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__res
         const int t0 = c * C;
         const int Lc = min(C, Tlen - t0);
         __syncthreads();  // previous chunk done with every buffer
-        if (ckpt) {  // the state entering the chunk (for the backward)
-            float *dst = ckpt + (pair * (nchunks + 1) + c) * (long)DK * DV;
-            for (int idx = tid; idx < DK * DVT; idx += kSimtThreads)
-                dst[(long)(idx / DVT) * DV + j0 + idx % DVT] = sS[idx];
-        }
 
         // ---- load the chunk (rows past the sequence end are zero) ----
         for (int idx = tid; idx < C * DK; idx += kSimtThreads) {
@@ -280,7 +275,7 @@ fwd_simt_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__res
 #pragma unroll 8
             for (int i = 0; i < DK; ++i) acc += qq[i] * sR[i * DVT + j];
             for (int s = 0; s <= t; ++s) acc += pp[s] * sU[s * DVT + j];
-            if (o) o[((bi * Tlen + t0 + t) * H + h) * (long)DV + j0 + j] = from_f32<T>(acc);
+            o[((bi * Tlen + t0 + t) * H + h) * (long)DV + j0 + j] = from_f32<T>(acc);
         }
         // ---- S <- e^{Gamma_C} S + Ktil^T U ----
         for (int idx = tid; idx < DK * DVT; idx += kSimtThreads) {
@@ -291,11 +286,6 @@ fwd_simt_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__res
         }
     }
     __syncthreads();
-    if (ckpt) {
-        float *dst = ckpt + (pair * (nchunks + 1) + nchunks) * (long)DK * DV;
-        for (int idx = tid; idx < DK * DVT; idx += kSimtThreads)
-            dst[(long)(idx / DVT) * DV + j0 + idx % DVT] = sS[idx];
-    }
     if (S_T) {
         for (int idx = tid; idx < DK * DVT; idx += kSimtThreads) {
             const int i = idx / DVT, j = idx % DVT;
@@ -305,7 +295,7 @@ fwd_simt_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__res
 }
 
 template <typename T, int DK>
-cudaError_t launch(const FwdArgs &a, float *ckpt = nullptr)
+cudaError_t launch(const FwdArgs &a)
 {
     constexpr int DVT = kSimtDvTile;
     const size_t smem = SimtSmem<DK, DVT>::kBytes;
@@ -315,7 +305,7 @@ cudaError_t launch(const FwdArgs &a, float *ckpt = nullptr)
     dim3 grid(a.dv / DVT, a.H, a.B);
     kern<<<grid, kSimtThreads, smem, a.stream>>>(
         (const T *)a.q, (const T *)a.k, (const T *)a.v, (const T *)a.b, (const T *)a.w,
-        a.log_alpha, a.S0, (T *)a.o, a.S_T, a.T, a.H, a.dv, a.layout, ckpt);
+        a.log_alpha, a.S0, (T *)a.o, a.S_T, a.T, a.H, a.dv, a.layout);
     return cudaGetLastError();
 }
 
@@ -367,12 +357,6 @@ cudaError_t launch_layer_epilogue_rows(const FwdArgs &a)
 {
     if (a.bf16) return a.dv == 128 ? launch_epi<__nv_bfloat16, 128>(a) : launch_epi<__nv_bfloat16, 64>(a);
     return a.dv == 128 ? launch_epi<float, 128>(a) : launch_epi<float, 64>(a);
-}
-
-cudaError_t launch_fwd_simt_checkpoints(const FwdArgs &a, float *ckpt)
-{
-    if (a.bf16) return a.dk == 128 ? launch<__nv_bfloat16, 128>(a, ckpt) : launch<__nv_bfloat16, 64>(a, ckpt);
-    return a.dk == 128 ? launch<float, 128>(a, ckpt) : launch<float, 64>(a, ckpt);
 }
 
 cudaError_t launch_fwd_simt(const FwdArgs &a)

@@ -220,30 +220,19 @@ extern "C" gdn2_status gdn2_bwd_chunked(const void *q, const void *k, const void
     if (cudaGetDevice(&dev) != cudaSuccess) return GDN2_ERR_CUDA;
     cudaMemPool_t pool = workspace_pool(dev);
     if (!pool) return GDN2_ERR_CUDA;
-    // the forward's state entering every chunk (and S_T): the backward's checkpoints
-    const long nch = (T + kChunk - 1) / kChunk;
-    void *ckpt = nullptr;
-    cudaError_t e = cudaMallocFromPoolAsync(&ckpt, DD * B * H * (size_t)(nch + 1), pool, s);
+    // per chunk: T and P, the state entering it, U, dU and the adjoint at its end
+    void *ws = nullptr;
+    cudaError_t e = cudaMallocFromPoolAsync(&ws, sizeof(float) * bwd_workspace_floats(B, T, H, dk, dv), pool, s);
     if (e != cudaSuccess) return GDN2_ERR_CUDA;
-    const size_t nk = sizeof(float) * (size_t)B * T * H * dk;
-    for (float *p : {dq, dk_, db, dlog_alpha})
-        if (e == cudaSuccess) e = cudaMemsetAsync(p, 0, nk, s);
-    FwdArgs f{};
-    f.q = q; f.k = k; f.v = v; f.b = b; f.w = w; f.log_alpha = log_alpha;
-    f.S0 = S0; f.o = nullptr; f.S_T = nullptr;
-    f.B = B; f.T = T; f.H = H; f.dk = dk; f.dv = dv;
-    f.bf16 = (dtype == GDN2_BF16);
-    f.stream = s;
-    if (e == cudaSuccess) e = launch_fwd_simt_checkpoints(f, static_cast<float *>(ckpt));
     BwdArgs a{};
-    a.q = q; a.k = k; a.v = v; a.b = b; a.w = w; a.log_alpha = log_alpha;
-    a.dO = dO; a.dS_T = dS_T; a.ckpt = static_cast<const float *>(ckpt);
+    a.q = q; a.k = k; a.v = v; a.b = b; a.w = w; a.log_alpha = log_alpha; a.S0 = S0;
+    a.dO = dO; a.dS_T = dS_T; a.ws = static_cast<float *>(ws);
     a.gq = dq; a.gk = dk_; a.gv = dv_; a.gb = db; a.gw = dw; a.gla = dlog_alpha; a.dS0 = dS0;
     a.B = B; a.T = T; a.H = H; a.dk = dk; a.dv = dv;
-    a.bf16 = f.bf16;
+    a.bf16 = (dtype == GDN2_BF16);
     a.stream = s;
-    if (e == cudaSuccess) e = launch_bwd_simt(a);
-    const cudaError_t fe = cudaFreeAsync(ckpt, s);
+    e = launch_bwd_simt(a);
+    const cudaError_t fe = cudaFreeAsync(ws, s);
     return (e == cudaSuccess && fe == cudaSuccess) ? GDN2_OK : GDN2_ERR_CUDA;
 }
 

@@ -47,19 +47,18 @@ cudaError_t launch_layer_epilogue_rows(const FwdArgs &a);  // y = RMSNorm(o) * w
 struct BwdArgs {
     const void *q, *k, *v, *b, *w;
     const float *log_alpha;
+    const float *S0;     // may be null (zero)
     const void *dO;
     const float *dS_T;   // may be null (zero)
-    const float *ckpt;   // [B][H][nchunks + 1][dk][dv] fp32: the state entering each chunk, and S_T
-    float *gq, *gk, *gv, *gb, *gw, *gla;   // fp32 gradients; gq, gk, gb, gla zeroed before the launch (atomics)
+    float *ws;           // bwd_workspace_floats(...) fp32 of workspace
+    float *gq, *gk, *gv, *gb, *gw, *gla;   // fp32 gradients
     float *dS0;          // may be null (not written)
     int B, T, H, dk, dv;
     bool bf16;
     cudaStream_t stream;
 };
+size_t bwd_workspace_floats(int B, int T, int H, int dk, int dv);
 cudaError_t launch_bwd_simt(const BwdArgs &a);
-// The fp32-pipe forward writing the state entering every chunk (and the final
-// state) to `ckpt` ([B][H][nchunks + 1][dk][dv]); outputs are not written.
-cudaError_t launch_fwd_simt_checkpoints(const FwdArgs &a, float *ckpt);
 // The library's stream-ordered workspace pool of a device (keeps freed blocks).
 cudaMemPool_t workspace_pool(int dev);
 
