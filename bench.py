@@ -86,6 +86,13 @@ def layer_algorithmic_bytes(B, T, H, dk, dv, s_in=2, s_out=2):
     return B * T * H * per_head_token + B * H * dk * dv * 4
 
 
+def bwd_algorithmic_bytes(B, T, H, dk, dv, s_in=2):
+    """The backward: the forward's inputs and dO once (input dtype, log_alpha fp32),
+    the six gradients once (fp32), S0 / dS_T absent."""
+    per_head_token = (3 * dk + 2 * dv + dv) * s_in + 4 * dk + 4 * (4 * dk + 2 * dv)
+    return B * T * H * per_head_token
+
+
 def decode_algorithmic_bytes(B, H, dk, dv, s_in=4, s_out=4):
     # state read + written once, q,k,b (dk) and v,w (dv) in the input dtype,
     # log_alpha fp32, o in the input dtype
@@ -442,6 +449,33 @@ def main():
     if g.gdn2_check_device_error() != g.GDN2_OK:
         raise RuntimeError("device error while timing the fused layer")
 
+    # ---------------- backward on the layer workload ----------------
+    bsets = [synth.draw_fwd_device(c.B, c.T, c.H, c.dk, c.dv, seed=600 + 10 * rank + i, device=dev, dtype=c.dtype,
+                                   log_alpha_range=c.log_alpha_range, gate_sigma=c.gate_sigma) for i in range(2)]
+    for i, d in enumerate(bsets):
+        d["dO"] = torch.randn(c.B, c.T, c.H, c.dv, device=dev).to(c.dtype)
+    for i in range(2):
+        g.gdn2_bwd_chunked(*(bsets[i % 2][n] for n in names), None, bsets[i % 2]["dO"], check=False)
+    torch.cuda.synchronize()
+    barrier(ws)
+    x0 = torch.cuda.Event(enable_timing=True); x1 = torch.cuda.Event(enable_timing=True)
+    reps = 5
+    x0.record(stream)
+    for i in range(reps):
+        g.gdn2_bwd_chunked(*(bsets[i % 2][n] for n in names), None, bsets[i % 2]["dO"], check=False)
+    x1.record(stream)
+    torch.cuda.synchronize()
+    ms = max_over_ranks(x0.elapsed_time(x1), ws) / reps
+    bb = bwd_algorithmic_bytes(c.B, c.T, c.H, c.dk, c.dv)
+    bwd_line = {"workload": c.name + " (gradients of q, k, v, b, w, log_alpha; fp32 outputs)",
+                "us_per_call": ms * 1e3, "tokens_per_s": c.B * c.T * ws / (ms / 1e3),
+                "roofline": {"bound": "hbm", "achieved": bb / (ms / 1e3) / 1e9, "peak": hbm_peak, "unit": "GB/s",
+                             "frac": bb / (ms / 1e3) / 1e9 / hbm_peak, "algorithmic_bytes_per_call": bb},
+                "launches": 4, "l2": "two input sets (> 126 MB of L2 between calls)"}
+    del bsets
+    if g.gdn2_check_device_error() != g.GDN2_OK:
+        raise RuntimeError("device error while timing the backward")
+
     # ---------------- decode: fp32 state resident in HBM, in place ----------------
     dc = DEC
     S = 0.05 * torch.randn(dc.B, dc.H, dc.dk, dc.dv, device=dev)
@@ -530,6 +564,7 @@ def main():
             "workloads": extra,
             "gate_layouts": layouts,
             "layer_fused": layer_line,
+            "backward": bwd_line,
             "decode_tokens": {"workload": "decode state B=256 H=16 d=128 fp32, T tokens per call",
                               "calls": tok_calls},
             "cpu_baseline": cpu,

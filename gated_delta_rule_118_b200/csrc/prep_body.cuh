@@ -127,6 +127,216 @@ __device__ __forceinline__ void prep_issue_loads(uint8_t *sm, uint64_t *bar_tma,
     if (la_tma) tma_load_4d(sm + L::LA, tm_la, bar_tma, 0, h, t0, bi);
 }
 
+// The layer's input processing (gdn2_layer_fwd) on a chunk's loaded tiles, in
+// place: L2 norm of each q and k row, sigmoid of the erase-gate logits, log
+// sigmoid of the decay logits (zero past the sequence end).  Out of line: the
+// operator's own path compiles as without it.
+static __device__ __noinline__ void prep_layer_inputs(uint8_t *sm, int tid, int bar_id, int Lc, unsigned layout)
+{
+    using L = PrepLayout;
+    // ---------------------------------------------------------- the layer's input processing
+    {   // L2 norm of each q and k row: two threads per row, one 64-channel half each
+        const int r = tid >> 1, half = tid & 1, t = r & 63;
+        uint8_t *row = (r < 64) ? sm + L::EQ + half * 16384 + 8192 + t * 128 : sm + L::KT + half * 8192 + t * 128;
+        // the row's 16-byte pieces in an order rotated by the row, so that the
+        // lanes of a warp (16 rows) spread over the banks
+        float ss = 0.f;
+#pragma unroll 2
+        for (int c = 0; c < 8; ++c) {
+            float x[8];
+            unpack8(*reinterpret_cast<const uint4 *>(row + 16 * ((c + t) & 7)), x);
+#pragma unroll
+            for (int u = 0; u < 8; ++u) ss = fmaf(x[u], x[u], ss);
+        }
+        ss += __shfl_xor_sync(0xffffffffu, ss, 1);
+        const float inv = rsqrtf(ss + kL2Eps);
+#pragma unroll 2
+        for (int c = 0; c < 8; ++c) {
+            float x[8];
+            uint4 *pp = reinterpret_cast<uint4 *>(row + 16 * ((c + t) & 7));
+            unpack8(*pp, x);
+#pragma unroll
+            for (int u = 0; u < 8; ++u) x[u] *= inv;
+            *pp = pack8(x);
+        }
+    }
+    if (!(layout & kEraseScalar) || !(layout & kDecayScalar)) {
+        const int t = tid >> 2, part = tid & 3;  // token, quarter of its channels
+        if (!(layout & kEraseScalar)) {   // erase gate from its logits (row t of both half tiles)
+#pragma unroll 1
+            for (int m = 0; m < 4; ++m) {
+                const int c = part * 4 + ((m + t) & 3);  // rotated by the row: bank spread
+                uint4 *pp = reinterpret_cast<uint4 *>(sm + L::EQ + (c >> 3) * 16384 + t * 128 + (c & 7) * 16);
+                float f[8];
+                unpack8(*pp, f);
+#pragma unroll
+                for (int u = 0; u < 8; ++u) f[u] = sigmoid_f(f[u]);
+                *pp = pack8(f);
+            }
+        }
+        if (!(layout & kDecayScalar)) {   // log-decay from its logits; none past the sequence end
+#pragma unroll 2
+            for (int m = 0; m < 8; ++m) {
+                float4 *pp = reinterpret_cast<float4 *>(sm + L::LA + t * 512 + part * 128 + ((m + t) & 7) * 16);
+                const float4 x = *pp;
+                *pp = t < Lc ? make_float4(log_sigmoid_f(x.x), log_sigmoid_f(x.y), log_sigmoid_f(x.z),
+                                           log_sigmoid_f(x.w))
+                             : make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+        }
+    }
+    named_bar(bar_id, kPrepThreads);
+}
+
+// The bounded form of a chunk's Gram (its decay too strong for the midpoint
+// split), by the prep's threads once the chunk's inputs are in `sm` (raw b, q, k
+// tiles and log_alpha): every factor is a decay over a stretch of the chunk,
+// never the inverse of one, so nothing can overflow and what underflows is
+// negligible:
+//   A_ts = sum_j b_tj k_tj k_sj f_tsj,  P_ts = sum_j q_tj k_sj f_tsj,
+//   f_tsj = e^{Gamma_tj - Gamma_sj} = prod_{s < u <= t} alpha_uj (running products),
+//   Ebar = e^{Gamma} b k, Qbar = e^{Gamma} q (decayed from the chunk start),
+//   Ktil = e^{Gamma_C - Gamma} k (decayed to the chunk end),
+// and the record's scalings by e^{Gamma_C - Gamma_r} and e^{Gamma_r} become 1.
+// Leaves A and a zero T in their fp32 places and P in its bf16 tile, like the
+// midpoint form's Gram readout.  Out of line: the fast path's code stays as it is.
+static __device__ __noinline__ void prep_bounded(uint8_t *sm, int tid, int bar_id)
+{
+    using L = PrepLayout;
+    const int warp = tid >> 5;
+    const int p = tid & 63, qr = tid >> 6;
+    float *la = reinterpret_cast<float *>(sm + L::LA);
+    float *Af = reinterpret_cast<float *>(sm + L::AF);
+    float *Tf = reinterpret_cast<float *>(sm + L::TF);
+    float *dec = reinterpret_cast<float *>(sm + L::DEC);
+    float *qprod = reinterpret_cast<float *>(sm + L::QP);
+    // ------------------------------------------------------ bounded path
+    float *Ak = reinterpret_cast<float *>(sm + L::KH);  // A, fp32 (the solve's scratch is free)
+    if (qr == 0) {
+        dec[2 * p] = 1.f;
+        dec[2 * p + 1] = 1.f;
+        dec[kDK + 2 * p] = 1.f;
+        dec[kDK + 2 * p + 1] = 1.f;
+    }
+    // alpha over log_alpha, and each quarter's product of alpha per channel
+    {
+        float q0 = 1.f, q1 = 1.f;
+#pragma unroll
+        for (int u = 0; u < 16; ++u) {
+            float2 *lp = reinterpret_cast<float2 *>(la + (qr * 16 + u) * kDK + 2 * p);
+            const float2 l = *lp;
+            const float2 a = make_float2(ex2_approx(l.x * kLog2e), ex2_approx(l.y * kLog2e));
+            *lp = a;
+            q0 *= a.x; q1 *= a.y;
+        }
+        *reinterpret_cast<float2 *>(qprod + qr * kDK + 2 * p) = make_float2(q0, q1);
+    }
+#pragma unroll
+    for (int m = 0; m < 4; ++m) reinterpret_cast<float4 *>(Ak)[tid + m * kPrepThreads] = make_float4(0.f, 0.f, 0.f, 0.f);
+    reinterpret_cast<float4 *>(sm + L::PO)[tid] = make_float4(0.f, 0.f, 0.f, 0.f);
+    reinterpret_cast<float4 *>(sm + L::PO)[tid + kPrepThreads] = make_float4(0.f, 0.f, 0.f, 0.f);
+    named_bar(bar_id, kPrepThreads);
+    {
+        // thread: token pair (pr, 63 - pr), 16 channels; the 8 lanes of a token reduce by shuffles
+        const int pr = tid >> 3, cg = tid & 7, hb = cg >> 2, cb = (cg & 3) * 32;
+        const uint8_t *bt = sm + L::EQ + hb * 16384, *qt = bt + 8192, *kt = sm + L::KT + hb * 8192;
+        const float *al = la + 16 * cg;
+#pragma unroll 1
+        for (int pass = 0; pass < 2; ++pass) {
+            // the lanes of a warp hold 4 tokens; the loop runs to the warp's
+            // largest token so that every lane takes part in the shuffles
+            const int t = pass ? 63 - pr : pr, tmax = pass ? 63 - 4 * warp : 4 * warp + 3;
+            float qv[16], ev[16], f[16];
+            unpack8(*reinterpret_cast<const uint4 *>(qt + swz_off(t, cb, 128)), qv);
+            unpack8(*reinterpret_cast<const uint4 *>(qt + swz_off(t, cb + 16, 128)), qv + 8);
+            unpack8(*reinterpret_cast<const uint4 *>(bt + swz_off(t, cb, 128)), ev);
+            unpack8(*reinterpret_cast<const uint4 *>(bt + swz_off(t, cb + 16, 128)), ev + 8);
+            unpack8(*reinterpret_cast<const uint4 *>(kt + swz_off(t, cb, 128)), f);
+            unpack8(*reinterpret_cast<const uint4 *>(kt + swz_off(t, cb + 16, 128)), f + 8);
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+                ev[j] *= f[j];
+                f[j] = 1.f;
+            }
+#pragma unroll 1
+            for (int s = tmax; s >= 0; --s) {
+                const bool on = s <= t;
+                float pa = 0.f, aa = 0.f;
+                if (on) {
+                    float kv[16];
+                    unpack8(*reinterpret_cast<const uint4 *>(kt + swz_off(s, cb, 128)), kv);
+                    unpack8(*reinterpret_cast<const uint4 *>(kt + swz_off(s, cb + 16, 128)), kv + 8);
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) {
+                        const float a = f[j] * kv[j];
+                        pa = fmaf(qv[j], a, pa);
+                        aa = fmaf(ev[j], a, aa);
+                    }
+#pragma unroll
+                    for (int j = 0; j < 16; j += 4) {
+                        const float4 a4 = *reinterpret_cast<const float4 *>(al + s * kDK + j);
+                        f[j] *= a4.x; f[j + 1] *= a4.y; f[j + 2] *= a4.z; f[j + 3] *= a4.w;
+                    }
+                }
+#pragma unroll
+                for (int o = 1; o < 8; o <<= 1) {
+                    pa += __shfl_xor_sync(0xffffffffu, pa, o);
+                    aa += __shfl_xor_sync(0xffffffffu, aa, o);
+                }
+                if (cg == 0 && on) {
+                    *reinterpret_cast<bf16 *>(sm + L::PO + swz_off(t, 2 * s, 128)) = __float2bfloat16_rn(pa);
+                    if (s < t) Ak[af_off(t, s)] = aa;
+                }
+            }
+        }
+    }
+    named_bar(bar_id, kPrepThreads);
+    // the bounded factors over the raw tiles (two channels of 16 tokens per
+    // thread), from running products of alpha: e^{Gamma_t} = prod_{u <= t} alpha_u,
+    // e^{Gamma_C - Gamma_t} = prod_{u > t} alpha_u
+    {
+        float pre0 = 1.f, pre1 = 1.f, post0 = 1.f, post1 = 1.f;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const float2 a = *reinterpret_cast<const float2 *>(qprod + q * kDK + 2 * p);
+            if (q < qr) { pre0 *= a.x; pre1 *= a.y; }
+            if (q > qr) { post0 *= a.x; post1 *= a.y; }
+        }
+        float2 sf[16];
+#pragma unroll
+        for (int u = 15; u >= 0; --u) {
+            sf[u] = make_float2(post0, post1);
+            const float2 a = *reinterpret_cast<const float2 *>(la + (qr * 16 + u) * kDK + 2 * p);
+            post0 *= a.x; post1 *= a.y;
+        }
+        const int hb = p >> 5;
+        const int cbyte = (2 * p & 63) * 2;
+#pragma unroll
+        for (int u = 0; u < 16; ++u) {
+            const int t = qr * 16 + u;
+            const float2 a = *reinterpret_cast<const float2 *>(la + t * kDK + 2 * p);
+            pre0 *= a.x; pre1 *= a.y;
+            const uint32_t off = swz_off(t, cbyte, 128);
+            __nv_bfloat162 *ep = reinterpret_cast<__nv_bfloat162 *>(sm + L::EQ + hb * 16384 + off);
+            __nv_bfloat162 *qp = reinterpret_cast<__nv_bfloat162 *>(sm + L::EQ + hb * 16384 + 8192 + off);
+            __nv_bfloat162 *kp = reinterpret_cast<__nv_bfloat162 *>(sm + L::KT + hb * 8192 + off);
+            const float2 bv = __bfloat1622float2(*ep), qv = __bfloat1622float2(*qp), kv = __bfloat1622float2(*kp);
+            *ep = __floats2bfloat162_rn(pre0 * bv.x * kv.x, pre1 * bv.y * kv.y);
+            *qp = __floats2bfloat162_rn(pre0 * qv.x, pre1 * qv.y);
+            *kp = __floats2bfloat162_rn(sf[u].x * kv.x, sf[u].y * kv.y);
+        }
+    }
+    named_bar(bar_id, kPrepThreads);  // every thread has read alpha
+    // A into the solve's place, T starts as zero
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+        const int idx = tid + m * kPrepThreads;
+        reinterpret_cast<float4 *>(Af)[idx] = reinterpret_cast<const float4 *>(Ak)[idx];
+        reinterpret_cast<float4 *>(Tf)[idx] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    named_bar(bar_id, kPrepThreads);
+}
+
 // The prep of one chunk (tokens [t0, t0 + 64) of head h, batch bi) by the
 // kPrepThreads threads tid = 0.. that share named barrier `bar_id`, once
 // prep_issue_loads has been issued for it: `sm` is their PrepLayout region
@@ -223,60 +433,7 @@ __device__ __forceinline__ bool prep_chunk(uint8_t *sm, uint32_t tmem, int tid, 
     };
     bool ok = named_bar_and(bar_id, kPrepThreads, (tid == 0) ? mbar_wait(bar_tma, tma_phase, err) : true) != 0;
 
-    if (ok && (gs.layout & kLayerInputs)) {
-        // ---------------------------------------------------------- the layer's input processing
-        {   // L2 norm of each q and k row: two threads per row, one 64-channel half each
-            const int r = tid >> 1, half = tid & 1, t = r & 63;
-            uint8_t *row = (r < 64) ? sm + L::EQ + half * 16384 + 8192 + t * 128 : sm + L::KT + half * 8192 + t * 128;
-            // the row's 16-byte pieces in an order rotated by the row, so that the
-            // lanes of a warp (16 rows) spread over the banks
-            float ss = 0.f;
-#pragma unroll 2
-            for (int c = 0; c < 8; ++c) {
-                float x[8];
-                unpack8(*reinterpret_cast<const uint4 *>(row + 16 * ((c + t) & 7)), x);
-#pragma unroll
-                for (int u = 0; u < 8; ++u) ss = fmaf(x[u], x[u], ss);
-            }
-            ss += __shfl_xor_sync(0xffffffffu, ss, 1);
-            const float inv = rsqrtf(ss + kL2Eps);
-#pragma unroll 2
-            for (int c = 0; c < 8; ++c) {
-                float x[8];
-                uint4 *pp = reinterpret_cast<uint4 *>(row + 16 * ((c + t) & 7));
-                unpack8(*pp, x);
-#pragma unroll
-                for (int u = 0; u < 8; ++u) x[u] *= inv;
-                *pp = pack8(x);
-            }
-        }
-        if (!(gs.layout & kEraseScalar) || !(gs.layout & kDecayScalar)) {
-            const int t = tid >> 2, part = tid & 3;  // token, quarter of its channels
-            if (!(gs.layout & kEraseScalar)) {   // erase gate from its logits (row t of both half tiles)
-#pragma unroll 1
-                for (int m = 0; m < 4; ++m) {
-                    const int c = part * 4 + ((m + t) & 3);  // rotated by the row: bank spread
-                    uint4 *pp = reinterpret_cast<uint4 *>(sm + L::EQ + (c >> 3) * 16384 + t * 128 + (c & 7) * 16);
-                    float f[8];
-                    unpack8(*pp, f);
-#pragma unroll
-                    for (int u = 0; u < 8; ++u) f[u] = sigmoid_f(f[u]);
-                    *pp = pack8(f);
-                }
-            }
-            if (!(gs.layout & kDecayScalar)) {   // log-decay from its logits; none past the sequence end
-#pragma unroll 2
-                for (int m = 0; m < 8; ++m) {
-                    float4 *pp = reinterpret_cast<float4 *>(sm + L::LA + t * 512 + part * 128 + ((m + t) & 7) * 16);
-                    const float4 x = *pp;
-                    *pp = t < Lc ? make_float4(log_sigmoid_f(x.x), log_sigmoid_f(x.y), log_sigmoid_f(x.z),
-                                               log_sigmoid_f(x.w))
-                                 : make_float4(0.f, 0.f, 0.f, 0.f);
-                }
-            }
-        }
-        named_bar(bar_id, kPrepThreads);
-    }
+    if (ok && (gs.layout & kLayerInputs)) prep_layer_inputs(sm, tid, bar_id, Lc, gs.layout);
 
     // Z = w v, straight into the record (MN-major operand blocks of 64 value
     // columns; each warp fills whole 128-byte rows)
@@ -309,7 +466,13 @@ __device__ __forceinline__ bool prep_chunk(uint8_t *sm, uint32_t tmem, int tid, 
         }
         tot[qr * kDK + 2 * p] = g0;
         tot[qr * kDK + 2 * p + 1] = g1;
-        named_bar(bar_id, kPrepThreads);
+        // The split factors e^{+x} and e^{-x}, x = Gamma_t - Gamma_r around the
+        // chunk midpoint, stay finite fp32/bf16 numbers for |x| <= 80.  Gamma only
+        // decreases, so |x| is at most the decay of a half chunk, which is at most
+        // e^{-80} when each quarter's is at most e^{-40}: the midpoint form then.
+        // Otherwise (or not a number: log_alpha = -inf) the chunk takes the bounded form.
+        exact = !named_bar_and(bar_id, kPrepThreads, (g0 >= -0.5f * kMidpointLogDecayRange) &&
+                                                         (g1 >= -0.5f * kMidpointLogDecayRange));
         float pre0 = 0.f, pre1 = 0.f, gc0 = 0.f, gc1 = 0.f;
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
@@ -319,16 +482,7 @@ __device__ __forceinline__ bool prep_chunk(uint8_t *sm, uint32_t tmem, int tid, 
         }
         // midpoint reference: Gamma after 32 tokens (tokens past T carry log_alpha = 0)
         const float gr0 = tot[2 * p] + tot[kDK + 2 * p], gr1 = tot[2 * p + 1] + tot[kDK + 2 * p + 1];
-        // x = Gamma_t - Gamma_r of this thread's tokens and channels.  The split
-        // factors e^{+x} and e^{-x} stay finite fp32/bf16 numbers for |x| <= 80;
-        // a chunk where some |x| is larger (or not a number: log_alpha = -inf)
-        // takes the bounded path below instead.
-        const float sh0 = pre0 - gr0, sh1 = pre1 - gr1;
-        bool far = false;
-#pragma unroll
-        for (int u = 0; u < 16; ++u)
-            far |= !(fabsf(lv[u].x + sh0) <= kMidpointLogDecayRange) | !(fabsf(lv[u].y + sh1) <= kMidpointLogDecayRange);
-        exact = !named_bar_and(bar_id, kPrepThreads, !far);
+        const float sh0 = pre0 - gr0, sh1 = pre1 - gr1;  // x = lv + sh
         if (qr == 0)
             *reinterpret_cast<float2 *>(rec + R::DEC + 8 * p) = make_float2(expf(gc0), expf(gc1));
 
@@ -389,140 +543,9 @@ __device__ __forceinline__ bool prep_chunk(uint8_t *sm, uint32_t tmem, int tid, 
             write_z();  // while the Gram runs
             ok = mma_done();
         } else {
-            // ------------------------------------------------------ bounded path
-            // Every factor is a decay over a stretch of the chunk, never the
-            // inverse of one, so nothing can overflow and what underflows is
-            // negligible:
-            //   A_ts = sum_j b_tj k_tj k_sj f_tsj,  P_ts = sum_j q_tj k_sj f_tsj,
-            //   f_tsj = e^{Gamma_tj - Gamma_sj} = prod_{s < u <= t} alpha_uj (running products),
-            //   Ebar = e^{Gamma} b k, Qbar = e^{Gamma} q (decayed from the chunk start),
-            //   Ktil = e^{Gamma_C - Gamma} k (decayed to the chunk end),
-            // and the record's scalings by e^{Gamma_C - Gamma_r} and e^{Gamma_r} become 1.
-            float *Ak = reinterpret_cast<float *>(sm + L::KH);  // A, fp32 (the solve's scratch is free)
-            if (qr == 0) {
-                dec[2 * p] = 1.f;
-                dec[2 * p + 1] = 1.f;
-                dec[kDK + 2 * p] = 1.f;
-                dec[kDK + 2 * p + 1] = 1.f;
-            }
-            // alpha over log_alpha, and each quarter's product of alpha per channel
-            {
-                float q0 = 1.f, q1 = 1.f;
-#pragma unroll
-                for (int u = 0; u < 16; ++u) {
-                    float2 *lp = reinterpret_cast<float2 *>(la + (qr * 16 + u) * kDK + 2 * p);
-                    const float2 l = *lp;
-                    const float2 a = make_float2(ex2_approx(l.x * kLog2e), ex2_approx(l.y * kLog2e));
-                    *lp = a;
-                    q0 *= a.x; q1 *= a.y;
-                }
-                *reinterpret_cast<float2 *>(qprod + qr * kDK + 2 * p) = make_float2(q0, q1);
-            }
-#pragma unroll
-            for (int m = 0; m < 4; ++m) reinterpret_cast<float4 *>(Ak)[tid + m * kPrepThreads] = make_float4(0.f, 0.f, 0.f, 0.f);
-            reinterpret_cast<float4 *>(sm + L::PO)[tid] = make_float4(0.f, 0.f, 0.f, 0.f);
-            reinterpret_cast<float4 *>(sm + L::PO)[tid + kPrepThreads] = make_float4(0.f, 0.f, 0.f, 0.f);
+            // ------------------------------------------------------ bounded form
             write_z();
-            named_bar(bar_id, kPrepThreads);
-            {
-                // thread: token pair (pr, 63 - pr), 16 channels; the 8 lanes of a token reduce by shuffles
-                const int pr = tid >> 3, cg = tid & 7, hb = cg >> 2, cb = (cg & 3) * 32;
-                const uint8_t *bt = sm + L::EQ + hb * 16384, *qt = bt + 8192, *kt = sm + L::KT + hb * 8192;
-                const float *al = la + 16 * cg;
-#pragma unroll 1
-                for (int pass = 0; pass < 2; ++pass) {
-                    // the lanes of a warp hold 4 tokens; the loop runs to the warp's
-                    // largest token so that every lane takes part in the shuffles
-                    const int t = pass ? 63 - pr : pr, tmax = pass ? 63 - 4 * warp : 4 * warp + 3;
-                    float qv[16], ev[16], f[16];
-                    unpack8(*reinterpret_cast<const uint4 *>(qt + swz_off(t, cb, 128)), qv);
-                    unpack8(*reinterpret_cast<const uint4 *>(qt + swz_off(t, cb + 16, 128)), qv + 8);
-                    unpack8(*reinterpret_cast<const uint4 *>(bt + swz_off(t, cb, 128)), ev);
-                    unpack8(*reinterpret_cast<const uint4 *>(bt + swz_off(t, cb + 16, 128)), ev + 8);
-                    unpack8(*reinterpret_cast<const uint4 *>(kt + swz_off(t, cb, 128)), f);
-                    unpack8(*reinterpret_cast<const uint4 *>(kt + swz_off(t, cb + 16, 128)), f + 8);
-#pragma unroll
-                    for (int j = 0; j < 16; ++j) {
-                        ev[j] *= f[j];
-                        f[j] = 1.f;
-                    }
-#pragma unroll 1
-                    for (int s = tmax; s >= 0; --s) {
-                        const bool on = s <= t;
-                        float pa = 0.f, aa = 0.f;
-                        if (on) {
-                            float kv[16];
-                            unpack8(*reinterpret_cast<const uint4 *>(kt + swz_off(s, cb, 128)), kv);
-                            unpack8(*reinterpret_cast<const uint4 *>(kt + swz_off(s, cb + 16, 128)), kv + 8);
-#pragma unroll
-                            for (int j = 0; j < 16; ++j) {
-                                const float a = f[j] * kv[j];
-                                pa = fmaf(qv[j], a, pa);
-                                aa = fmaf(ev[j], a, aa);
-                            }
-#pragma unroll
-                            for (int j = 0; j < 16; j += 4) {
-                                const float4 a4 = *reinterpret_cast<const float4 *>(al + s * kDK + j);
-                                f[j] *= a4.x; f[j + 1] *= a4.y; f[j + 2] *= a4.z; f[j + 3] *= a4.w;
-                            }
-                        }
-#pragma unroll
-                        for (int o = 1; o < 8; o <<= 1) {
-                            pa += __shfl_xor_sync(0xffffffffu, pa, o);
-                            aa += __shfl_xor_sync(0xffffffffu, aa, o);
-                        }
-                        if (cg == 0 && on) {
-                            *reinterpret_cast<bf16 *>(sm + L::PO + swz_off(t, 2 * s, 128)) = __float2bfloat16_rn(pa);
-                            if (s < t) Ak[af_off(t, s)] = aa;
-                        }
-                    }
-                }
-            }
-            named_bar(bar_id, kPrepThreads);
-            // the bounded factors over the raw tiles (two channels of 16 tokens per
-            // thread), from running products of alpha: e^{Gamma_t} = prod_{u <= t} alpha_u,
-            // e^{Gamma_C - Gamma_t} = prod_{u > t} alpha_u
-            {
-                float pre0 = 1.f, pre1 = 1.f, post0 = 1.f, post1 = 1.f;
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const float2 a = *reinterpret_cast<const float2 *>(qprod + q * kDK + 2 * p);
-                    if (q < qr) { pre0 *= a.x; pre1 *= a.y; }
-                    if (q > qr) { post0 *= a.x; post1 *= a.y; }
-                }
-                float2 sf[16];
-#pragma unroll
-                for (int u = 15; u >= 0; --u) {
-                    sf[u] = make_float2(post0, post1);
-                    const float2 a = *reinterpret_cast<const float2 *>(la + (qr * 16 + u) * kDK + 2 * p);
-                    post0 *= a.x; post1 *= a.y;
-                }
-                const int hb = p >> 5;
-                const int cbyte = (2 * p & 63) * 2;
-#pragma unroll
-                for (int u = 0; u < 16; ++u) {
-                    const int t = qr * 16 + u;
-                    const float2 a = *reinterpret_cast<const float2 *>(la + t * kDK + 2 * p);
-                    pre0 *= a.x; pre1 *= a.y;
-                    const uint32_t off = swz_off(t, cbyte, 128);
-                    __nv_bfloat162 *ep = reinterpret_cast<__nv_bfloat162 *>(sm + L::EQ + hb * 16384 + off);
-                    __nv_bfloat162 *qp = reinterpret_cast<__nv_bfloat162 *>(sm + L::EQ + hb * 16384 + 8192 + off);
-                    __nv_bfloat162 *kp = reinterpret_cast<__nv_bfloat162 *>(sm + L::KT + hb * 8192 + off);
-                    const float2 bv = __bfloat1622float2(*ep), qv = __bfloat1622float2(*qp), kv = __bfloat1622float2(*kp);
-                    *ep = __floats2bfloat162_rn(pre0 * bv.x * kv.x, pre1 * bv.y * kv.y);
-                    *qp = __floats2bfloat162_rn(pre0 * qv.x, pre1 * qv.y);
-                    *kp = __floats2bfloat162_rn(sf[u].x * kv.x, sf[u].y * kv.y);
-                }
-            }
-            named_bar(bar_id, kPrepThreads);  // every thread has read alpha
-            // A into the solve's place, T starts as zero
-#pragma unroll
-            for (int m = 0; m < 4; ++m) {
-                const int idx = tid + m * kPrepThreads;
-                reinterpret_cast<float4 *>(Af)[idx] = reinterpret_cast<const float4 *>(Ak)[idx];
-                reinterpret_cast<float4 *>(Tf)[idx] = make_float4(0.f, 0.f, 0.f, 0.f);
-            }
-            named_bar(bar_id, kPrepThreads);
+            prep_bounded(sm, tid, bar_id);
         }
     }
 
