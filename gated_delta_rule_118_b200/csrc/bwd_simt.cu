@@ -25,8 +25,9 @@
 // so no factor can overflow and any log_alpha <= 0 (-inf included) is exact.
 //
 // Four kernels:
-//   gram   (per chunk and head, all in parallel)  A and P by running products; T
-//   fwd    (per head and 16-column value tile, chunks in order)  the state entering
+//   gram   (per chunk and head, all in parallel)  A and P by running products; T;
+//          the decayed factors Ebar, Qbar, Ktil and e^{Gamma_C}
+//   fwd    (per head and 8-column value tile, chunks in order)  the state entering
 //          each chunk (checkpoint) and U
 //   adj    (per head and value tile, chunks in reverse)  the adjoint at each chunk's
 //          end, dU, dv, dw, dS0
@@ -39,7 +40,7 @@ namespace gdn2 {
 namespace {
 
 constexpr int kBwdThreads = 256;
-constexpr int kBwdDvTile = 16;
+constexpr int kChainDvTile = 8;  // value columns of a chain CTA (fwd, adj)
 constexpr int C = kChunk;
 constexpr int LDC = kChunk + 1;
 
@@ -49,6 +50,9 @@ struct BwdWs {
     float *ck;      // [pair][nch + 1][dk][dv]: the state entering each chunk, and S_T
     float *U, *dU;  // [pair][nch][C][dv]
     float *dS;      // [pair][nch][dk][dv]: dL/dS at the end of each chunk
+    // decayed factors [pair][nch][C][dk]: Ebar = e^{Gamma} b k, Qbar = e^{Gamma} q,
+    // Ktil = e^{Gamma_C - Gamma} k; and e^{Gamma_C} [pair][nch][dk]
+    float *Eb, *Qb, *Kt, *gC;
 };
 
 // Chunk inputs into shared memory ([C][DK + 1] fp32; zero past the sequence end, alpha = 1 there).
@@ -100,14 +104,15 @@ bwd_gram_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__res
     // A_ts = sum_i E_ti k_si f_tsi (s < t), P_ts = sum_i q_ti k_si f_tsi (s <= t),
     // f_tsi = prod_{s<u<=t} alpha_ui: thread (token t, channel quarter), 4 lanes per token
     {
+        // (channel 4 j + cq for lane cq: the 4 lanes of a token hit 4 different banks)
         constexpr int CPT = DK / 4;
-        const int t = tid >> 2, cq = tid & 3, i0 = cq * CPT;
+        const int t = tid >> 2, cq = tid & 3;
         const int tmax = (tid >> 5) * 8 + 7;  // the warp's largest token: every lane shuffles
         float qv[CPT], ev[CPT], f[CPT];
 #pragma unroll
         for (int j = 0; j < CPT; ++j) {
-            qv[j] = sQ[t * LDK + i0 + j];
-            ev[j] = sB[t * LDK + i0 + j] * sK[t * LDK + i0 + j];
+            qv[j] = sQ[t * LDK + 4 * j + cq];
+            ev[j] = sB[t * LDK + 4 * j + cq] * sK[t * LDK + 4 * j + cq];
             f[j] = 1.f;
         }
         for (int s = tmax; s >= 0; --s) {
@@ -116,10 +121,10 @@ bwd_gram_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__res
             if (on) {
 #pragma unroll
                 for (int j = 0; j < CPT; ++j) {
-                    const float a = f[j] * sK[s * LDK + i0 + j];
+                    const float a = f[j] * sK[s * LDK + 4 * j + cq];
                     pa = fmaf(qv[j], a, pa);
                     aa = fmaf(ev[j], a, aa);
-                    f[j] *= sAl[s * LDK + i0 + j];
+                    f[j] *= sAl[s * LDK + 4 * j + cq];
                 }
             }
             pa += __shfl_xor_sync(0xffffffffu, pa, 1);
@@ -148,24 +153,47 @@ bwd_gram_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__res
         __syncthreads();
     }
     for (int idx = tid; idx < C * C; idx += kBwdThreads) Tg[idx] = sT[(idx / C) * LDC + idx % C];
+    // the decayed factors of the chain kernels (running products of alpha per channel)
+    const long fo = (pair * nch + c) * (long)C * DK;
+    if (tid < DK) {
+        const int i = tid;
+        float p = 1.f;
+        for (int t = 0; t < C; ++t) {
+            p *= sAl[t * LDK + i];
+            ws.Eb[fo + t * DK + i] = p * sB[t * LDK + i] * sK[t * LDK + i];
+            ws.Qb[fo + t * DK + i] = p * sQ[t * LDK + i];
+        }
+        ws.gC[(pair * nch + c) * DK + i] = p;
+    } else if (tid < 2 * DK) {
+        const int i = tid - DK;
+        float sf = 1.f;
+        for (int t = C - 1; t >= 0; --t) {
+            ws.Kt[fo + t * DK + i] = sf * sK[t * LDK + i];
+            sf *= sAl[t * LDK + i];
+        }
+    }
 }
+
+// Value-axis inputs of a chain kernel (zero past the sequence end).
+template <typename T>
+__device__ __forceinline__ float ld(const T *p, long off, bool on) { return on ? to_f32(p[off]) : 0.f; }
 
 // ------------------------------------------------------------------ fwd (checkpoints and U)
 template <int DK>
 struct FwdSmem {
-    static constexpr int LDK = DK + 1, DVT = kBwdDvTile;
-    static constexpr size_t kBytes = sizeof(float) * (4 * C * LDK + C * LDC + DK * DVT + 2 * C * DVT + DK);
+    static constexpr int LDK = DK + 1, DVT = kChainDvTile;
+    static constexpr size_t kBytes = sizeof(float) * (2 * C * LDK + C * LDC + DK * DVT + 2 * C * DVT + DK);
 };
 
 template <typename T, int DK>
-__global__ void __launch_bounds__(kBwdThreads, 1)
+__global__ void __launch_bounds__(kBwdThreads, 2)
 bwd_fwd_kernel(const T *__restrict__ k, const T *__restrict__ v, const T *__restrict__ b, const T *__restrict__ w,
                const float *__restrict__ log_alpha, const float *__restrict__ S0, BwdWs ws, int Tlen, int H, int DV)
 {
-    constexpr int LDK = DK + 1, DVT = kBwdDvTile;
+    constexpr int LDK = DK + 1, DVT = kChainDvTile;
     extern __shared__ float smem[];
-    float *sK = smem, *sB = sK + C * LDK, *sAl = sB + C * LDK, *sX = sAl + C * LDK;
-    float *sT = sX + C * LDK, *sS = sT + C * LDC, *sR = sS + DK * DVT, *sU = sR + C * DVT, *sG = sU + C * DVT;
+    float *sE = smem, *sKt = sE + C * LDK, *sT = sKt + C * LDK, *sS = sT + C * LDC, *sR = sS + DK * DVT;
+    float *sU = sR + C * DVT, *sG = sU + C * DVT;
     const int tid = threadIdx.x, j0 = blockIdx.x * DVT, h = blockIdx.y;
     const long bi = blockIdx.z, pair = bi * H + h;
     const int nch = (Tlen + C - 1) / C;
@@ -181,64 +209,72 @@ bwd_fwd_kernel(const T *__restrict__ k, const T *__restrict__ v, const T *__rest
         for (int idx = tid; idx < DK * DVT; idx += kBwdThreads) ck[(long)(idx / DVT) * DV + j0 + idx % DVT] = sS[idx];
         if (c == nch) break;
         const int t0 = c * C, Lc = min(C, Tlen - t0);
-        load_rows<T, DK>(sK, k, tid, bi, Tlen, H, h, t0, Lc);
-        load_rows<T, DK>(sB, b, tid, bi, Tlen, H, h, t0, Lc);
-        load_alpha<DK>(sAl, log_alpha, tid, bi, Tlen, H, h, t0, Lc);
         const float *Tg = ws.T + (pair * nch + c) * C * C;
         for (int idx = tid; idx < C * C; idx += kBwdThreads) sT[(idx / C) * LDC + idx % C] = Tg[idx];
         for (int idx = tid; idx < C * DVT; idx += kBwdThreads) {
             const int t = idx / DVT, j = idx % DVT;
-            float z = 0.f;
-            if (t < Lc) {
-                const long off = ((bi * Tlen + t0 + t) * H + h) * (long)DV + j0 + j;
-                z = to_f32(w[off]) * to_f32(v[off]);
+            const long off = ((bi * Tlen + t0 + t) * H + h) * (long)DV + j0 + j;
+            sR[idx] = ld(w, off, t < Lc) * ld(v, off, t < Lc);
+        }
+        // the chunk's decayed factors (from the gram kernel)
+        {
+            const long fo = (pair * nch + c) * (long)C * DK;
+            for (int idx = tid; idx < C * DK; idx += kBwdThreads) {
+                sE[(idx / DK) * LDK + idx % DK] = ws.Eb[fo + idx];
+                sKt[(idx / DK) * LDK + idx % DK] = ws.Kt[fo + idx];
             }
-            sR[idx] = z;
+            for (int i = tid; i < DK; i += kBwdThreads) sG[i] = ws.gC[(pair * nch + c) * DK + i];
         }
         __syncthreads();
-        // Ebar = e^{Gamma} (*) b (*) k (running products over the tokens); e^{Gamma_C}
-        for (int i = tid; i < DK; i += kBwdThreads) {
-            float p = 1.f;
-            for (int t = 0; t < C; ++t) {
-                p *= sAl[t * LDK + i];
-                sX[t * LDK + i] = p * sB[t * LDK + i] * sK[t * LDK + i];
-            }
-            sG[i] = p;
-        }
-        __syncthreads();
+        // the thread's outputs: column j of rows r0 + RS * m (independent sums, interleaved)
+        constexpr int RS = kBwdThreads / DVT;    // rows apart
+        constexpr int NO = C * DVT / kBwdThreads, NS = DK * DVT / kBwdThreads;
+        const int r0 = tid / DVT, j = tid % DVT;
         // RHS = Z - Ebar S
-        for (int idx = tid; idx < C * DVT; idx += kBwdThreads) {
-            const int t = idx / DVT, j = idx % DVT;
-            const float *e = sX + t * LDK;
-            float acc = 0.f;
-            for (int i = 0; i < DK; ++i) acc = fmaf(e[i], sS[i * DVT + j], acc);
-            sR[idx] -= acc;
+        {
+            float acc[NO];
+#pragma unroll
+            for (int m = 0; m < NO; ++m) acc[m] = 0.f;
+            for (int i = 0; i < DK; ++i) {
+                const float sv = sS[i * DVT + j];
+#pragma unroll
+                for (int m = 0; m < NO; ++m) acc[m] = fmaf(sE[(r0 + RS * m) * LDK + i], sv, acc[m]);
+            }
+#pragma unroll
+            for (int m = 0; m < NO; ++m) sR[(r0 + RS * m) * DVT + j] -= acc[m];
         }
         __syncthreads();
         // U = T RHS (T lower triangular)
-        float *Ug = ws.U + (pair * nch + c) * (long)C * DV;
-        for (int idx = tid; idx < C * DVT; idx += kBwdThreads) {
-            const int t = idx / DVT, j = idx % DVT;
-            float acc = 0.f;
-            for (int s = 0; s <= t; ++s) acc = fmaf(sT[t * LDC + s], sR[s * DVT + j], acc);
-            sU[idx] = acc;
-            Ug[(long)t * DV + j0 + j] = acc;
-        }
-        // Ktil = e^{Gamma_C - Gamma} (*) k (running products from the chunk end)
-        for (int i = tid; i < DK; i += kBwdThreads) {
-            float sf = 1.f;
-            for (int t = C - 1; t >= 0; --t) {
-                sX[t * LDK + i] = sf * sK[t * LDK + i];
-                sf *= sAl[t * LDK + i];
+        {
+            float *Ug = ws.U + (pair * nch + c) * (long)C * DV;
+            float acc[NO];
+#pragma unroll
+            for (int m = 0; m < NO; ++m) acc[m] = 0.f;
+            for (int s = 0; s < C; ++s) {
+                const float rv = sR[s * DVT + j];
+#pragma unroll
+                for (int m = 0; m < NO; ++m) acc[m] = fmaf(sT[(r0 + RS * m) * LDC + s], rv, acc[m]);
+            }
+#pragma unroll
+            for (int m = 0; m < NO; ++m) {
+                const int t = r0 + RS * m;
+                sU[t * DVT + j] = acc[m];
+                Ug[(long)t * DV + j0 + j] = acc[m];
             }
         }
         __syncthreads();
         // S <- e^{Gamma_C} S + Ktil^T U
-        for (int idx = tid; idx < DK * DVT; idx += kBwdThreads) {
-            const int i = idx / DVT, j = idx % DVT;
-            float acc = sG[i] * sS[idx];
-            for (int s = 0; s < C; ++s) acc = fmaf(sX[s * LDK + i], sU[s * DVT + j], acc);
-            sS[idx] = acc;
+        {
+            float acc[NS];
+#pragma unroll
+            for (int m = 0; m < NS; ++m) acc[m] = sG[r0 + RS * m] * sS[(r0 + RS * m) * DVT + j];
+            for (int s = 0; s < C; ++s) {
+                const float uv = sU[s * DVT + j];
+#pragma unroll
+                for (int m = 0; m < NS; ++m) acc[m] = fmaf(sKt[s * LDK + r0 + RS * m], uv, acc[m]);
+            }
+#pragma unroll
+            for (int m = 0; m < NS; ++m) sS[(r0 + RS * m) * DVT + j] = acc[m];
         }
     }
 }
@@ -246,21 +282,21 @@ bwd_fwd_kernel(const T *__restrict__ k, const T *__restrict__ v, const T *__rest
 // ------------------------------------------------------------------ adj (the adjoint chain)
 template <int DK>
 struct AdjSmem {
-    static constexpr int LDK = DK + 1, DVT = kBwdDvTile;
-    static constexpr size_t kBytes = sizeof(float) * (5 * C * LDK + 2 * C * LDC + DK * DVT + 2 * C * DVT);
+    static constexpr int LDK = DK + 1, DVT = kChainDvTile;
+    static constexpr size_t kBytes = sizeof(float) * (3 * C * LDK + 2 * C * LDC + DK * DVT + 3 * C * DVT + DK);
 };
 
 template <typename T, int DK>
-__global__ void __launch_bounds__(kBwdThreads, 1)
+__global__ void __launch_bounds__(kBwdThreads, 2)
 bwd_adj_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__ v, const T *__restrict__ b,
                const T *__restrict__ w, const float *__restrict__ log_alpha, const T *__restrict__ dO,
                const float *__restrict__ dS_T, BwdWs ws, float *__restrict__ gv, float *__restrict__ gw,
                float *__restrict__ dS0, int Tlen, int H, int DV)
 {
-    constexpr int LDK = DK + 1, DVT = kBwdDvTile;
+    constexpr int LDK = DK + 1, DVT = kChainDvTile;
     extern __shared__ float smem[];
-    float *sQ = smem, *sK = sQ + C * LDK, *sB = sK + C * LDK, *sAl = sB + C * LDK, *sX = sAl + C * LDK;
-    float *sT = sX + C * LDK, *sP = sT + C * LDC, *sD = sP + C * LDC, *sO = sD + DK * DVT, *sR = sO + C * DVT;
+    float *sKt = smem, *sQb = sKt + C * LDK, *sEb = sQb + C * LDK, *sT = sEb + C * LDK, *sP = sT + C * LDC;
+    float *sD = sP + C * LDC, *sO = sD + DK * DVT, *sR = sO + C * DVT, *sU = sR + C * DVT, *sG = sU + C * DVT;
     const int tid = threadIdx.x, j0 = blockIdx.x * DVT, h = blockIdx.y;
     const long bi = blockIdx.z, pair = bi * H + h;
     const int nch = (Tlen + C - 1) / C;
@@ -275,10 +311,6 @@ bwd_adj_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__rest
         __syncthreads();  // the later chunk is done with every buffer; dS' is final
         float *dsg = ws.dS + (pair * nch + c) * DD;
         for (int idx = tid; idx < DK * DVT; idx += kBwdThreads) dsg[(long)(idx / DVT) * DV + j0 + idx % DVT] = sD[idx];
-        load_rows<T, DK>(sQ, q, tid, bi, Tlen, H, h, t0, Lc);
-        load_rows<T, DK>(sK, k, tid, bi, Tlen, H, h, t0, Lc);
-        load_rows<T, DK>(sB, b, tid, bi, Tlen, H, h, t0, Lc);
-        load_alpha<DK>(sAl, log_alpha, tid, bi, Tlen, H, h, t0, Lc);
         const float *Tg = ws.T + (pair * nch + c) * C * C, *Pg = ws.P + (pair * nch + c) * C * C;
         for (int idx = tid; idx < C * C; idx += kBwdThreads) {
             sT[(idx / C) * LDC + idx % C] = Tg[idx];
@@ -286,40 +318,63 @@ bwd_adj_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__rest
         }
         for (int idx = tid; idx < C * DVT; idx += kBwdThreads) {
             const int t = idx / DVT, j = idx % DVT;
-            sO[idx] = (t < Lc) ? to_f32(dO[((bi * Tlen + t0 + t) * H + h) * (long)DV + j0 + j]) : 0.f;
+            sO[idx] = ld(dO, ((bi * Tlen + t0 + t) * H + h) * (long)DV + j0 + j, t < Lc);
         }
-        __syncthreads();
-        // Ktil = e^{Gamma_C - Gamma} (*) k
-        for (int i = tid; i < DK; i += kBwdThreads) {
-            float sf = 1.f;
-            for (int t = C - 1; t >= 0; --t) {
-                sX[t * LDK + i] = sf * sK[t * LDK + i];
-                sf *= sAl[t * LDK + i];
+        // the chunk's decayed factors (from the gram kernel)
+        {
+            const long fo = (pair * nch + c) * (long)C * DK;
+            for (int idx = tid; idx < C * DK; idx += kBwdThreads) {
+                const int r = (idx / DK) * LDK + idx % DK;
+                sKt[r] = ws.Kt[fo + idx];
+                sQb[r] = ws.Qb[fo + idx];
+                sEb[r] = ws.Eb[fo + idx];
             }
+            for (int i = tid; i < DK; i += kBwdThreads) sG[i] = ws.gC[(pair * nch + c) * DK + i];
         }
         __syncthreads();
-        // RHS2 = Ktil dS' + P^T dO
-        for (int idx = tid; idx < C * DVT; idx += kBwdThreads) {
-            const int s = idx / DVT, j = idx % DVT;
-            const float *kt = sX + s * LDK;
-            float acc = 0.f;
-            for (int i = 0; i < DK; ++i) acc = fmaf(kt[i], sD[i * DVT + j], acc);
-            for (int t = s; t < C; ++t) acc = fmaf(sP[t * LDC + s], sO[t * DVT + j], acc);
-            sR[idx] = acc;
+        // the thread's outputs: column j of rows r0 + RS * m (independent sums, interleaved)
+        constexpr int RS = kBwdThreads / DVT, NO = C * DVT / kBwdThreads;
+        const int r0 = tid / DVT, j = tid % DVT;
+        // RHS2 = Ktil dS' + P^T dO  (P lower: P_ts = 0 for t < s)
+        {
+            float acc[NO];
+#pragma unroll
+            for (int m = 0; m < NO; ++m) acc[m] = 0.f;
+            for (int i = 0; i < DK; ++i) {
+                const float dv = sD[i * DVT + j];
+#pragma unroll
+                for (int m = 0; m < NO; ++m) acc[m] = fmaf(sKt[(r0 + RS * m) * LDK + i], dv, acc[m]);
+            }
+            for (int t = 0; t < C; ++t) {
+                const float ov = sO[t * DVT + j];
+#pragma unroll
+                for (int m = 0; m < NO; ++m) acc[m] = fmaf(sP[t * LDC + r0 + RS * m], ov, acc[m]);
+            }
+#pragma unroll
+            for (int m = 0; m < NO; ++m) sR[(r0 + RS * m) * DVT + j] = acc[m];
         }
         __syncthreads();
-        // dU = T^T RHS2 (T^T upper triangular); dv = dU (*) w, dw = dU (*) v
-        float *dUg = ws.dU + (pair * nch + c) * (long)C * DV;
-        for (int idx = tid; idx < C * DVT; idx += kBwdThreads) {
-            const int s = idx / DVT, j = idx % DVT;
-            float acc = 0.f;
-            for (int t = s; t < C; ++t) acc = fmaf(sT[t * LDC + s], sR[t * DVT + j], acc);
-            sX[s * LDK + j] = acc;  // dU (Ktil's room: no longer needed)
-            dUg[(long)s * DV + j0 + j] = acc;
-            if (s < Lc) {
-                const long off = ((bi * Tlen + t0 + s) * H + h) * (long)DV + j0 + j;
-                gv[off] = acc * to_f32(w[off]);
-                gw[off] = acc * to_f32(v[off]);
+        // dU = T^T RHS2 (T lower: T_ts = 0 for t < s); dv = dU (*) w, dw = dU (*) v
+        {
+            float *dUg = ws.dU + (pair * nch + c) * (long)C * DV;
+            float acc[NO];
+#pragma unroll
+            for (int m = 0; m < NO; ++m) acc[m] = 0.f;
+            for (int t = 0; t < C; ++t) {
+                const float rv = sR[t * DVT + j];
+#pragma unroll
+                for (int m = 0; m < NO; ++m) acc[m] = fmaf(sT[t * LDC + r0 + RS * m], rv, acc[m]);
+            }
+#pragma unroll
+            for (int m = 0; m < NO; ++m) {
+                const int s = r0 + RS * m;
+                sU[s * DVT + j] = acc[m];
+                dUg[(long)s * DV + j0 + j] = acc[m];
+                if (s < Lc) {
+                    const long off = ((bi * Tlen + t0 + s) * H + h) * (long)DV + j0 + j;
+                    gv[off] = acc[m] * to_f32(w[off]);
+                    gw[off] = acc[m] * to_f32(v[off]);
+                }
             }
         }
         __syncthreads();
@@ -330,15 +385,14 @@ bwd_adj_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__rest
             float acc[JPT];
 #pragma unroll
             for (int j = 0; j < JPT; ++j) acc[j] = 0.f;
-            float p = 1.f;
             for (int t = 0; t < C; ++t) {
-                p *= sAl[t * LDK + i];
-                const float qp = p * sQ[t * LDK + i], ep = p * sB[t * LDK + i] * sK[t * LDK + i];
+                const float qp = sQb[t * LDK + i], ep = sEb[t * LDK + i];
 #pragma unroll
-                for (int j = 0; j < JPT; ++j) acc[j] += qp * sO[t * DVT + jb + j] - ep * sX[t * LDK + jb + j];
+                for (int j = 0; j < JPT; ++j) acc[j] += qp * sO[t * DVT + jb + j] - ep * sU[t * DVT + jb + j];
             }
+            const float g = sG[i];
 #pragma unroll
-            for (int j = 0; j < JPT; ++j) sD[i * DVT + jb + j] = p * sD[i * DVT + jb + j] + acc[j];
+            for (int j = 0; j < JPT; ++j) sD[i * DVT + jb + j] = g * sD[i * DVT + jb + j] + acc[j];
         }
     }
     __syncthreads();
@@ -348,12 +402,13 @@ bwd_adj_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__rest
 }
 
 // ------------------------------------------------------------------ grad (key-axis gradients)
-constexpr int kGradCols = 32;     // value columns staged at a time
+constexpr int kGradCols = 16;     // value columns staged at a time
 constexpr int kGradThreads = 512;  // 16 (token, channel) pairs per thread at dk = 128
 template <int DK>
 struct GradSmem {
     static constexpr int LDK = DK + 1;
-    static constexpr size_t kBytes = sizeof(float) * (4 * C * LDK + 2 * C * LDC + 3 * C * kGradCols + DK);
+    static constexpr size_t kBytes =
+        sizeof(float) * (4 * C * LDK + 2 * C * LDC + 3 * C * kGradCols + 3 * DK * (kGradCols + 1) + DK);
 };
 
 template <typename T, int DK>
@@ -368,7 +423,9 @@ bwd_grad_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__res
     extern __shared__ float smem[];
     float *sQ = smem, *sK = sQ + C * LDK, *sB = sK + C * LDK, *sAl = sB + C * LDK;
     float *sW1 = sAl + C * LDK, *sW2 = sW1 + C * LDC;  // W1[t][s] = dO_t . u_s, W2[t][s] = dU_t . u_s
-    float *sUc = sW2 + C * LDC, *sdUc = sUc + C * NC, *sOc = sdUc + C * NC, *sRow = sOc + C * NC;
+    float *sUc = sW2 + C * LDC, *sdUc = sUc + C * NC, *sOc = sdUc + C * NC;
+    // the block's columns of S (entering), dS' and S (leaving): rows padded to NC + 1
+    float *sSc = sOc + C * NC, *sDc = sSc + DK * (NC + 1), *sNc = sDc + DK * (NC + 1), *sRow = sNc + DK * (NC + 1);
     const int tid = threadIdx.x, c = blockIdx.x, h = blockIdx.y;
     const long bi = blockIdx.z, pair = bi * H + h;
     const int nch = gridDim.x, t0 = c * C, Lc = min(C, Tlen - t0);
@@ -399,6 +456,12 @@ bwd_grad_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__res
             sdUc[idx] = dUg[(long)t * DV + jc + j];
             sOc[idx] = (t < Lc) ? to_f32(dO[((bi * Tlen + t0 + t) * H + h) * (long)DV + jc + j]) : 0.f;
         }
+        for (int idx = tid; idx < DK * NC; idx += kGradThreads) {
+            const int r = idx / NC, j = idx % NC;
+            sSc[r * (NC + 1) + j] = Sc[(long)r * DV + jc + j];
+            sDc[r * (NC + 1) + j] = dSc[(long)r * DV + jc + j];
+            sNc[r * (NC + 1) + j] = Sn[(long)r * DV + jc + j];
+        }
         __syncthreads();
 #pragma unroll
         for (int m = 0; m < WPT; ++m) {
@@ -410,7 +473,7 @@ bwd_grad_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__res
             }
         }
         // (S dO_t)_i, (S dU_t)_i, (dS' u_t)_i and rowsum(dS' (*) S_next)_i over these columns
-        const float *si = Sc + (long)i * DV + jc, *di = dSc + (long)i * DV + jc, *ni = Sn + (long)i * DV + jc;
+        const float *si = sSc + i * (NC + 1), *di = sDc + i * (NC + 1), *ni = sNc + i * (NC + 1);
 #pragma unroll 4
         for (int j = 0; j < NC; ++j) {
             const float sij = si[j], dij = di[j];
@@ -498,8 +561,12 @@ cudaError_t launch(const BwdArgs &a)
     ws.ck = p; p += pairs * (nch + 1) * (long)a.dk * a.dv;
     ws.U = p; p += pairs * nch * (long)C * a.dv;
     ws.dU = p; p += pairs * nch * (long)C * a.dv;
-    ws.dS = p;
-    const dim3 chunks(nch, a.H, a.B), tiles(a.dv / kBwdDvTile, a.H, a.B);
+    ws.dS = p; p += pairs * nch * (long)a.dk * a.dv;
+    ws.Eb = p; p += pairs * nch * (long)C * a.dk;
+    ws.Qb = p; p += pairs * nch * (long)C * a.dk;
+    ws.Kt = p; p += pairs * nch * (long)C * a.dk;
+    ws.gC = p;
+    const dim3 chunks(nch, a.H, a.B), tiles(a.dv / kChainDvTile, a.H, a.B);
     kg<<<chunks, kBwdThreads, GramSmem<DK>::kBytes, a.stream>>>((const T *)a.q, (const T *)a.k, (const T *)a.b,
                                                                  a.log_alpha, ws, a.T, a.H);
     kf<<<tiles, kBwdThreads, FwdSmem<DK>::kBytes, a.stream>>>((const T *)a.k, (const T *)a.v, (const T *)a.b,
@@ -520,7 +587,7 @@ size_t bwd_workspace_floats(int B, int T, int H, int dk, int dv)
 {
     const long nch = (T + C - 1) / C, pairs = (long)B * H;
     return (size_t)pairs * (2 * nch * C * C + (nch + 1) * (long)dk * dv + 2 * nch * (long)C * dv +
-                            nch * (long)dk * dv);
+                            nch * (long)dk * dv + 3 * nch * (long)C * dk + nch * (long)dk);
 }
 
 cudaError_t launch_bwd_simt(const BwdArgs &a)
