@@ -42,8 +42,13 @@ N_INPUT_SETS = 4  # rotating input sets: 4 x 136 MB > 126 MB of L2
 # dram__bytes_read.sum + dram__bytes_write.sum per call from an ncu capture of
 # the current kernels (None once a kernel has changed since the capture), summed
 # over the kernels of one call; the captures are summarised under profiles/.
-NCU_TRAFFIC_BYTES = {"fwd": None, "train": None, "long": None, "decode": 281.078016e6 + 213.638144e6}
-EXTRA_CASES = ((synth.TRAIN_BF16, "train", 3, 10), (synth.LONG_BF16, "long", 2, 5))
+NCU_TRAFFIC_BYTES = {"fwd": 118119424 + 55336448, "train": 4 * (234994176 + 138480640 + 135311104 + 31001600
+                                                                   + 151028480 + 16768000),
+                     "long": 1888002048 + 1315758848, "decode": 281043456 + 212228864,
+                     "decode_tokens_T16": 469875456 + 245164288,
+                     "bwd": 83982080 + 79402496 + 118176256 + 64889344 + 195499776 + 135079168 + 303447808
+                            + 101542144}
+EXTRA_CASES = ((synth.TRAIN_BF16, "train", 3, 10), (synth.LONG_BF16, "long", 3, 10))
 
 
 def bench_config():
@@ -227,13 +232,25 @@ def run_profile_case(args):
                                   log_alpha_range=c.log_alpha_range, gate_sigma=c.gate_sigma)
         for _ in range(args.warmup + args.steps):
             g.gdn2_fwd_chunked(*(d[n] for n in names), S0=None)
+    elif args.profile == "bwd":
+        c = CASE
+        d = synth.draw_fwd_device(c.B, c.T, c.H, c.dk, c.dv, seed=0, device=dev, dtype=c.dtype,
+                                  log_alpha_range=c.log_alpha_range, gate_sigma=c.gate_sigma)
+        dO = torch.randn(c.B, c.T, c.H, c.dv, device=dev).to(c.dtype)
+        for _ in range(args.warmup + args.steps):
+            g.gdn2_bwd_chunked(*(d[n] for n in names), None, dO)
     else:
         dc = DEC
         S = 0.05 * torch.randn(dc.B, dc.H, dc.dk, dc.dv, device=dev)
-        dd = synth.draw_fwd_device(dc.B, 1, dc.H, dc.dk, dc.dv, seed=7000, device=dev, dtype=torch.float32)
-        x = {n: dd[n][:, 0].contiguous() for n in names}
-        for _ in range(args.warmup + args.steps):
-            g.gdn2_decode_step(*(x[n] for n in names), S)
+        Tn = 16 if args.profile == "decode_tokens" else 1
+        dd = synth.draw_fwd_device(dc.B, Tn, dc.H, dc.dk, dc.dv, seed=7000, device=dev, dtype=torch.float32)
+        if Tn == 1:
+            x = {n: dd[n][:, 0].contiguous() for n in names}
+            for _ in range(args.warmup + args.steps):
+                g.gdn2_decode_step(*(x[n] for n in names), S)
+        else:
+            for _ in range(args.warmup + args.steps):
+                g.gdn2_decode_tokens(*(dd[n] for n in names), S)
     torch.cuda.synchronize()
     if g.gdn2_check_device_error() != g.GDN2_OK:
         raise RuntimeError("device error")
@@ -247,7 +264,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--decode-steps", type=int, default=1000)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--profile", choices=["fwd", "fwd_train", "fwd_long", "decode"], default=None,
+    ap.add_argument("--profile", choices=["fwd", "fwd_train", "fwd_long", "decode", "decode_tokens", "bwd"],
+                    default=None,
                     help="run a few launches of one operator on the bench workload for an ncu "
                          "capture (no timing, no JSON line)")
     args = ap.parse_args()
@@ -470,7 +488,8 @@ def main():
     bwd_line = {"workload": c.name + " (gradients of q, k, v, b, w, log_alpha; fp32 outputs)",
                 "us_per_call": ms * 1e3, "tokens_per_s": c.B * c.T * ws / (ms / 1e3),
                 "roofline": {"bound": "hbm", "achieved": bb / (ms / 1e3) / 1e9, "peak": hbm_peak, "unit": "GB/s",
-                             "frac": bb / (ms / 1e3) / 1e9 / hbm_peak, "algorithmic_bytes_per_call": bb},
+                             "frac": bb / (ms / 1e3) / 1e9 / hbm_peak, "algorithmic_bytes_per_call": bb,
+                             "traffic": NCU_TRAFFIC_BYTES["bwd"]},
                 "launches": 4, "l2": "two input sets (> 126 MB of L2 between calls)"}
     del bsets
     if g.gdn2_check_device_error() != g.GDN2_OK:
@@ -524,6 +543,7 @@ def main():
         tok_calls[f"T{Tn}"] = {"T": Tn, "us_per_call": ms * 1e3, "tokens_per_s": dc.B * Tn * ws / (ms / 1e3),
                                "hbm_gbs": tb / (ms / 1e3) / 1e9, "frac": tb / (ms / 1e3) / 1e9 / hbm_peak,
                                "algorithmic_bytes_per_call": tb,
+                               "traffic": NCU_TRAFFIC_BYTES.get(f"decode_tokens_T{Tn}"),
                                "vs_decode_steps": (Tn * dec_ms) / ms}
         del dd, ot
     if g.gdn2_check_device_error() != g.GDN2_OK:
