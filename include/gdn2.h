@@ -278,8 +278,9 @@ gdn2_status gdn2_layer_fwd(const void *q, const void *k, const void *v,
  *   dv, dw                  [B][T][H][dv]  fp32   written
  *   dS0         [B][H][dk][dv] fp32    written; NULL means not wanted
  *
- * The key-axis gradients are sums over the value columns, added across column
- * tiles with fp32 atomics: their last bits may differ from run to run.
+ * The key-axis gradients are sums over the value columns; one CTA per chunk and
+ * head forms each of them in a fixed order, without atomics, so repeated calls
+ * give identical bits.
  */
 gdn2_status gdn2_bwd_chunked(const void *q, const void *k, const void *v,
                              const void *b, const void *w, const float *log_alpha,
