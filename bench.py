@@ -46,8 +46,7 @@ NCU_TRAFFIC_BYTES = {"fwd": 118119424 + 55336448, "train": 4 * (234994176 + 1384
                                                                    + 151028480 + 16768000),
                      "long": 1888002048 + 1315758848, "decode": 281043456 + 212228864,
                      "decode_tokens_T16": 469875456 + 245164288,
-                     "bwd": 83982080 + 79402496 + 118176256 + 64889344 + 195499776 + 135079168 + 303447808
-                            + 101542144}
+                     "bwd": None}
 EXTRA_CASES = ((synth.TRAIN_BF16, "train", 3, 10), (synth.LONG_BF16, "long", 3, 10))
 
 

@@ -42,6 +42,15 @@
 // business: a window of records that are all ready before the chain starts
 // (WindowFlow), or rings that the chain shares with concurrent prep and output
 // work, with flags in global memory (fwd_persist.cu).
+//
+// The adjoint chain of the backward (ADJ) walks the same records in reverse.
+// The gradient dS of the state entering a chunk follows from the gradient dS'
+// of the state leaving it and the chunk's output gradients dO by the transpose
+// of the chunk's map:
+//   dS = e^{Gamma_C} dS' + NG^T dS'x + QS^T dO,    dS'x = bf16(dS')
+// NG^T and QS^T are the record's NG and QS read as MN-major operands (the same
+// bytes), dO comes by TMA in Z's place, and the exported images are those of
+// dS' for every chunk.
 #pragma once
 
 #include "tc_common.cuh"
@@ -105,6 +114,27 @@ struct WindowFlow {
     __device__ void exported(int) const {}
 };
 
+// The adjoint walk: records and dS' image slots of chunks n-1, ..., 0, and the
+// output gradients dO of chunk c by TMA (`tm_do`: [B][T][H][DV] bf16, boxes of
+// 64 values x 64 tokens with the 128-byte swizzle).
+template <int DV>
+struct ReverseFlow {
+    static constexpr bool kPublishes = false;
+    const uint8_t *recs;
+    uint8_t *sxs;
+    const CUtensorMap *tm_do;
+    int n, h, bi;
+    __device__ const uint8_t *record(int cw) const { return recs + (long)(n - 1 - cw) * Record<DV>::BYTES; }
+    __device__ uint8_t *sx_slot(int cw) const { return sxs + (long)(n - 1 - cw) * SxSlot<DV>::BYTES; }
+    __device__ bool record_ready(int) const { return true; }
+    __device__ bool wait_count(const uint32_t *, uint32_t) const { return true; }
+    __device__ void exported(int) const {}
+    __device__ void load_do(uint8_t *dst, uint64_t *bar, int cw, int blk) const
+    {
+        tma_load_4d(dst, tm_do, bar, blk * 64, h, (n - 1 - cw) * kChunk, bi);
+    }
+};
+
 // One thread: the mbarriers of a chain CTA.
 template <int DV, int DVT>
 __device__ __forceinline__ void chain_init(uint8_t *sm)
@@ -129,7 +159,7 @@ __device__ __forceinline__ void chain_init(uint8_t *sm)
 // threads tid < kChainThreads of a CTA whose mbarriers chain_init has set up
 // and whose `tmem` holds TMEM_COLS columns.  S_in / S_out (either may be null)
 // are the [pairs][128][DV] fp32 states before the first and after the last chunk.
-template <int DV, int DVT, class Flow>
+template <int DV, int DVT, class Flow, bool ADJ = false>
 __device__ __forceinline__ void chain_run(uint8_t *sm, uint32_t tmem, int tid, const Flow &f, const float *S_in,
                                           float *S_out, long pair, int tile, int ncw, unsigned int *err)
 {
@@ -168,8 +198,13 @@ __device__ __forceinline__ void chain_run(uint8_t *sm, uint32_t tmem, int tid, c
                 const uint8_t *rec = f.record(cw);
                 mbar_arrive_expect_tx(full + s, (uint32_t)(L::STAGE + L::DEC_BYTES));
                 bulk_load(st + L::S_NG, rec + R::NG, 32768, full + s);
-                bulk_load(st + L::S_Y, rec + R::Y, 16384, full + s);
-                bulk_load(st + L::S_Z, rec + R::Z + tile * NB * 8192, NB * 8192, full + s);
+                if constexpr (ADJ) {
+                    bulk_load(st + L::S_Y, rec + R::QS, 16384, full + s);
+                    for (int b = 0; b < NB; ++b) f.load_do(st + L::S_Z + b * 8192, full + s, cw, tile * NB + b);
+                } else {
+                    bulk_load(st + L::S_Y, rec + R::Y, 16384, full + s);
+                    bulk_load(st + L::S_Z, rec + R::Z + tile * NB * 8192, NB * 8192, full + s);
+                }
                 bulk_load(sm + L::DECR + s * L::DEC_BYTES, rec + R::DEC, L::DEC_BYTES, full + s);
                 issued = cw + 1;
             }
@@ -179,8 +214,13 @@ __device__ __forceinline__ void chain_run(uint8_t *sm, uint32_t tmem, int tid, c
     } else if (warp == kYzWarp) {
         // ------------------------------------------------------------ Y Z issuer
         if (lane == 0) {
-            const uint32_t idd = idesc_bf16(128, DVT, 0, 1);
-            const uint64_t y0 = smem_desc(sbase + L::S_Y, 2048, 128, kSwNone);  // no-swizzle K chunks of 128 rows
+            // Y: K-major, no-swizzle K chunks of 128 rows (16 tokens a step = 4 KB);
+            // QS^T (ADJ): MN-major, 8-token K groups of 128 bytes, 8-key M chunks
+            // of 1 KB (16 tokens a step = 256 bytes)
+            const uint32_t idd = idesc_bf16(128, DVT, ADJ ? 1 : 0, 1);
+            const uint64_t y0 = ADJ ? smem_desc(sbase + L::S_Y, 128, 1024, kSwNone)
+                                    : smem_desc(sbase + L::S_Y, 2048, 128, kSwNone);
+            constexpr int kYStep = ADJ ? 256 : 4096;
             const uint64_t z0 = smem_desc(sbase + L::S_Z, 8192, 1024, kSw128);
             bool ok = true;
             for (int cw = 0; cw < ncw; ++cw) {
@@ -195,7 +235,7 @@ __device__ __forceinline__ void chain_run(uint8_t *sm, uint32_t tmem, int tid, c
                     const uint32_t d = tmem + (uint32_t)(b * DVT);
 #pragma unroll
                     for (int ks = 0; ks < 4; ++ks)
-                        umma_bf16(d, y0 + so + (uint64_t)((ks * 4096) >> 4), z0 + so + (uint64_t)((ks * 2048) >> 4),
+                        umma_bf16(d, y0 + so + (uint64_t)((ks * kYStep) >> 4), z0 + so + (uint64_t)((ks * 2048) >> 4),
                                   idd, ks > 0);
                 }
                 umma_commit(yz_done + b);
@@ -204,9 +244,14 @@ __device__ __forceinline__ void chain_run(uint8_t *sm, uint32_t tmem, int tid, c
     } else if (warp == kMmaWarp) {
         // ------------------------------------------------------------ NG Sx issuer
         if (lane == 0) {
-            const uint32_t idd = idesc_bf16(128, DVT, 0, 1);
+            // NG: K-major (16 key channels a step = 4 KB); NG^T (ADJ): MN-major, the
+            // same bytes with 8-row K groups of 128 bytes and 8-column M chunks of
+            // 2 KB (16 a step = 256 bytes)
+            const uint32_t idd = idesc_bf16(128, DVT, ADJ ? 1 : 0, 1);
             // descriptor start addresses are in 16-byte units: byte offsets >> 4 add directly
-            const uint64_t ng0 = smem_desc(sbase + L::S_NG, 2048, 128, kSwNone);
+            const uint64_t ng0 = ADJ ? smem_desc(sbase + L::S_NG, 128, 2048, kSwNone)
+                                     : smem_desc(sbase + L::S_NG, 2048, 128, kSwNone);
+            constexpr int kNgStep = ADJ ? 256 : 4096;
             const uint64_t sx0 = smem_desc(sbase + L::SR, 128, 2048, kSwNone);   // MN-major, 8-row K groups
             bool ok = true;
             for (int cw = 0; cw < ncw; ++cw) {
@@ -220,7 +265,7 @@ __device__ __forceinline__ void chain_run(uint8_t *sm, uint32_t tmem, int tid, c
                     const uint32_t d = tmem + (uint32_t)(b * DVT);
 #pragma unroll
                     for (int ks = 0; ks < kDK / 16; ++ks)
-                        umma_bf16(d, ng0 + so + (uint64_t)((ks * 4096) >> 4), sx0 + (uint64_t)((ks * 256) >> 4), idd, 1);
+                        umma_bf16(d, ng0 + so + (uint64_t)((ks * kNgStep) >> 4), sx0 + (uint64_t)((ks * 256) >> 4), idd, 1);
                 }
                 umma_commit(s_done);
                 if (cw + NS < ncw) umma_commit(empty + s);

@@ -72,7 +72,10 @@ cudaMemPool_t workspace_pool(int dev)
     return pools[dev];
 }
 
-namespace {
+bool make_token_map(CUtensorMap *m, const void *base, int d, int H, int T, int B)
+{
+    return make_map(m, base, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d, H, T, B, 64, CU_TENSOR_MAP_SWIZZLE_128B);
+}
 
 // Tensor maps of the TMA-loaded inputs: q, k, b, log_alpha and the output-gate
 // logits of the fused layer.  A gate given as one value per (token, head), and
@@ -94,8 +97,6 @@ bool make_input_maps(const FwdArgs &a, CUtensorMap *maps)
         return false;
     return !a.g || make_map(&maps[4], a.g, BF, 2, a.dv, a.H, a.T, a.B, 64, CU_TENSOR_MAP_SWIZZLE_128B);
 }
-
-}  // namespace
 
 FwdTcPlan plan_fwd_tc(int B, int T, int H, int dv, size_t budget, int num_sms)
 {

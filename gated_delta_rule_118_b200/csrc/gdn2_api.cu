@@ -220,18 +220,26 @@ extern "C" gdn2_status gdn2_bwd_chunked(const void *q, const void *k, const void
     if (cudaGetDevice(&dev) != cudaSuccess) return GDN2_ERR_CUDA;
     cudaMemPool_t pool = workspace_pool(dev);
     if (!pool) return GDN2_ERR_CUDA;
-    // per chunk: T and P, the state entering it, U, dU and the adjoint at its end
+    // bf16 inputs with dk = 128 run on the tensor cores (workspace: the prep
+    // records with T and P, and the state and dS' images of every chunk); fp32
+    // inputs and dk = 64 on the fp32 pipes (per chunk: T and P, the state
+    // entering it, U, dU and the adjoint at its end)
+    const bool tc = dtype == GDN2_BF16 && dk == 128;
+    unsigned int *err = nullptr;
+    int num_sms = 0;
+    if (tc && device_context(&err, &num_sms) != GDN2_OK) return GDN2_ERR_CUDA;
+    const size_t ws_bytes = tc ? bwd_tc_workspace_bytes(B, T, H, dv) : sizeof(float) * bwd_workspace_floats(B, T, H, dk, dv);
     void *ws = nullptr;
-    cudaError_t e = cudaMallocFromPoolAsync(&ws, sizeof(float) * bwd_workspace_floats(B, T, H, dk, dv), pool, s);
+    cudaError_t e = cudaMallocFromPoolAsync(&ws, ws_bytes, pool, s);
     if (e != cudaSuccess) return GDN2_ERR_CUDA;
     BwdArgs a{};
     a.q = q; a.k = k; a.v = v; a.b = b; a.w = w; a.log_alpha = log_alpha; a.S0 = S0;
-    a.dO = dO; a.dS_T = dS_T; a.ws = static_cast<float *>(ws);
+    a.dO = dO; a.dS_T = dS_T; a.ws = tc ? nullptr : static_cast<float *>(ws);
     a.gq = dq; a.gk = dk_; a.gv = dv_; a.gb = db; a.gw = dw; a.gla = dlog_alpha; a.dS0 = dS0;
     a.B = B; a.T = T; a.H = H; a.dk = dk; a.dv = dv;
     a.bf16 = (dtype == GDN2_BF16);
     a.stream = s;
-    e = launch_bwd_simt(a);
+    e = tc ? launch_bwd_tc(a, static_cast<uint8_t *>(ws), err, num_sms) : launch_bwd_simt(a);
     const cudaError_t fe = cudaFreeAsync(ws, s);
     return (e == cudaSuccess && fe == cudaSuccess) ? GDN2_OK : GDN2_ERR_CUDA;
 }

@@ -59,6 +59,12 @@ struct BwdArgs {
 };
 size_t bwd_workspace_floats(int B, int T, int H, int dk, int dv);
 cudaError_t launch_bwd_simt(const BwdArgs &a);
+// The bf16 tensor-core backward (bwd_tc.cu; dk = 128): prep records with T and
+// P for every chunk, the forward chain's state images, the adjoint chain's
+// images of dS', then the gradients of every chunk in parallel.  `ws` holds
+// bwd_tc_workspace_bytes(...) bytes.
+size_t bwd_tc_workspace_bytes(int B, int T, int H, int dv);
+cudaError_t launch_bwd_tc(const BwdArgs &a, uint8_t *ws, unsigned int *err, int num_sms);
 // The library's stream-ordered workspace pool of a device (keeps freed blocks).
 cudaMemPool_t workspace_pool(int dev);
 
@@ -92,12 +98,18 @@ constexpr int kWindowSlots = 4;
 // `budget` bytes (the no-allocation entry point).
 FwdTcPlan plan_fwd_tc(int B, int T, int H, int dv, size_t budget, int num_sms);
 cudaError_t run_fwd_tc(const FwdArgs &a, const FwdTcPlan &p, uint8_t *ws);
+// Tensor maps of the forward's TMA-loaded inputs (q, k, b, log_alpha, output-gate
+// logits), and of a bf16 [B][T][H][d] tensor in boxes of 64 channels x 64
+// tokens with the 128-byte swizzle.
+bool make_input_maps(const FwdArgs &a, CUtensorMap *maps);
+bool make_token_map(CUtensorMap *m, const void *base, int d, int H, int T, int B);
 cudaError_t launch_fwd_tc(const FwdArgs &a);
 // `overlap`: launch as a programmatic dependent of the previous kernel in the
 // stream, so that it may start before that kernel ends (only where the two
 // touch disjoint data).
+// tp: non-null for the backward, which keeps every chunk's T and P there (16 KB per record).
 cudaError_t launch_prep(const FwdArgs &a, const CUtensorMap *maps, uint8_t *ws, int c0, int ncw, int WC,
-                        bool overlap);
+                        bool overlap, uint8_t *tp = nullptr);
 cudaError_t launch_chain(const FwdArgs &a, int dvt, const uint8_t *ws, uint8_t *sx, const float *S_in,
                          float *S_out, int ncw, int WC, bool overlap);
 cudaError_t launch_out(const FwdArgs &a, const CUtensorMap *tm_g, const uint8_t *ws, const uint8_t *sx, int c0,

@@ -342,14 +342,16 @@ static __device__ __noinline__ void prep_bounded(uint8_t *sm, int tid, int bar_i
 // prep_issue_loads has been issued for it: `sm` is their PrepLayout region
 // (1024-byte aligned), `tmem` the first of their 256 tensor-memory columns,
 // `bar_mma` an mbarrier for UMMA completion whose phase parity `mma_phase`
-// tracks, and `rec` the chunk's record.  Returns false (every thread alike)
-// when a wait timed out.
-template <int DV>
+// tracks, and `rec` the chunk's record.  With TP (the backward) the chunk's T
+// and P also go to `tp`: two bf16 [64][64] tiles (T, then P), rows of 128 bytes
+// with the 128-byte swizzle, as they sit in shared memory.  Returns false
+// (every thread alike) when a wait timed out.
+template <int DV, bool TP = false>
 __device__ __forceinline__ bool prep_chunk(uint8_t *sm, uint32_t tmem, int tid, int bar_id, uint64_t *bar_tma,
                                            uint32_t tma_phase, uint64_t *bar_mma, uint32_t &mma_phase,
                                            const bf16 *__restrict__ vg, const bf16 *__restrict__ wg,
                                            const GateSrc &gs, uint8_t *__restrict__ rec, int Tlen, int H, int t0,
-                                           int h, int bi, unsigned int *err)
+                                           int h, int bi, unsigned int *err, uint8_t *__restrict__ tp = nullptr)
 {
     using L = PrepLayout;
     using R = Record<DV>;
@@ -699,6 +701,14 @@ __device__ __forceinline__ bool prep_chunk(uint8_t *sm, uint32_t tmem, int tid, 
         }
         fence_proxy_async_smem();
         named_bar(bar_id, kPrepThreads);
+        if (TP) {  // T and P, final from here on, for the backward
+#pragma unroll
+            for (int m = 0; m < 2; ++m) {
+                const int idx = tid + m * kPrepThreads;
+                reinterpret_cast<uint4 *>(tp)[idx] = reinterpret_cast<const uint4 *>(sm + L::TB)[idx];
+                reinterpret_cast<uint4 *>(tp + 8192)[idx] = reinterpret_cast<const uint4 *>(sm + L::PO)[idx];
+            }
+        }
 
         // ---------------------------------------------------------- Khat^T T (M = 128),  PT = P T (M = 64)
         if (tid == 0) {

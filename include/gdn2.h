@@ -267,9 +267,14 @@ gdn2_status gdn2_layer_fwd(const void *q, const void *k, const void *v,
  * must use the modulated keys and values, the per-channel gates staying inside
  * the gradient aggregation).  b and w get gradients of their own, per channel.
  * The forward is recomputed first (its chunk-entry states are the backward's
- * checkpoints, held in a workspace from the library's pool); all arithmetic is
- * fp32 on the CUDA cores, and every decay between two tokens is a running
- * product of alpha, so any log_alpha <= 0 is handled.
+ * checkpoints, held in a workspace from the library's pool), then the gradient
+ * of every chunk's exit state by a reverse pass over the chunks, then the
+ * gradients of each chunk, all chunks at once.  Any log_alpha <= 0 is handled:
+ * pairwise decays that a split around the chunk midpoint cannot hold are
+ * running products of alpha.
+ *   bf16 inputs with dk = 128: tensor cores (bf16 operands, fp32 accumulation
+ *     and state), within the bf16 tolerance of the forward;
+ *   fp32 inputs, and dk = 64: fp32 on the CUDA cores.
  *
  *   q, k, v, b, w, log_alpha, S0, B, T, H, dk, dv, dtype   as for gdn2_fwd_chunked
  *   dO          [B][T][H][dv]  dtype   incoming gradient of o

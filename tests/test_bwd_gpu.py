@@ -1,14 +1,15 @@
 """gdn2_bwd_chunked on the GPU against the fp64 oracle's backpropagation
 through the token recurrence (gdn2_oracle_bwd), every gradient, element by
-element.  The backward computes in fp32 from the input values (bf16 inputs
-are upcast exactly), so the fp32 tolerance applies to both input dtypes."""
+element.  bf16 inputs with dk = 128 run on the tensor cores (bf16 operands,
+fp32 accumulation and state) and are held to the bf16 tolerance; fp32 inputs,
+and dk = 64, run in fp32 on the CUDA cores and are held to the fp32 one."""
 import pytest
 import torch
 
 import oracle
 import synth
 import gated_delta_rule_118_b200 as g
-from parity import TOL_F32, rel_err, to_dev
+from parity import TOL_BF16, TOL_F32, rel_err, to_dev
 
 pytestmark = pytest.mark.gpu
 NAMES = ("q", "k", "v", "b", "w", "log_alpha")
@@ -25,12 +26,17 @@ def case(B, T, H, dk, dv, dtype, seed, s0=0.05, with_dst=True, kind=None):
     return d
 
 
-def check(d, tol=TOL_F32):
+def tolerance(d):
+    return TOL_BF16 if d["q"].dtype == torch.bfloat16 and d["q"].shape[-1] == 128 else TOL_F32
+
+
+def check(d, tol=None):
+    tol = tolerance(d) if tol is None else tol
     dd = to_dev(d)
     got = g.gdn2_bwd_chunked(*(dd[n] for n in NAMES), dd["S0"], dd["dO"], dd["dS_T"])
     ref = oracle.bwd(*(d[n] for n in NAMES), d["S0"], d["dO"], d["dS_T"])
     errs = {n: rel_err(got[n], ref[n]) for n in GRADS}
-    assert all(e <= tol for e in errs.values()), errs
+    assert all(e <= tol for e in errs.values()), ", ".join(f"{n} {e:.3g}" for n, e in errs.items())
     return errs
 
 
@@ -57,15 +63,30 @@ def test_zero_initial_state_and_no_final_gradient():
     check(case(1, 150, 2, 128, 128, torch.bfloat16, seed=950, s0=0.0, with_dst=False))
 
 
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16], ids=["f32", "bf16"])
 @pytest.mark.parametrize("kind", synth.DECAY_KINDS)
-def test_strong_decay_every_gradient(kind):
-    check(case(1, 200, 2, 128, 128, torch.float32, seed=960, kind=kind))
+def test_strong_decay_every_gradient(kind, dtype):
+    """Chunks in the bounded form (running products of alpha) and, for bf16,
+    the tensor-core backward's walks of the pairwise decays."""
+    check(case(1, 200, 2, 128, 128, dtype, seed=960, kind=kind))
 
 
-def test_erase_gate_up_to_2():
-    d = case(1, 150, 2, 128, 128, torch.float32, seed=970)
-    d["b"] = 2.0 * d["b"]
+@pytest.mark.parametrize("dv", [64, 128])
+def test_strong_decay_tensor_core_value_widths(dv):
+    check(case(2, 130, 2, 128, dv, torch.bfloat16, seed=965, kind=synth.DECAY_KINDS[-1]))
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16], ids=["f32", "bf16"])
+def test_erase_gate_up_to_2(dtype):
+    d = case(1, 150, 2, 128, 128, dtype, seed=970)
+    d["b"] = (2.0 * d["b"].float()).to(dtype)
     check(d)
+
+
+@pytest.mark.parametrize("T", [64, 65, 127, 640])
+def test_tensor_core_chunk_edges(T):
+    """Whole and ragged last chunks, one chunk and many, dv = 64 and 128."""
+    check(case(1, T, 3, 128, 64 if T % 2 else 128, torch.bfloat16, seed=975 + T))
 
 
 def test_oracle_sized_fp32_workload():
