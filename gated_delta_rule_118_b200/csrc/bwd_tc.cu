@@ -17,10 +17,10 @@
 //
 // Steps (one stream, no host synchronisation):
 //   1. prep of every chunk (prep_body.cuh), keeping T and P beside the records;
-//   2. the forward chain over every chunk: bf16 images of each chunk's entry
-//      state;
-//   3. the adjoint chain over the chunks in reverse: images of each chunk's dS',
-//      and dS0;
+//   2. in one launch, on separate CTAs, the forward chain over every chunk (bf16
+//      images of each chunk's entry state) and the adjoint chain over the chunks
+//      in reverse (images of each chunk's dS', and dS0): the adjoint chain needs
+//      the records and dO, not the forward's states;
 //   4. grad_kernel: one CTA per (chunk, head, batch), all in parallel, the
 //      products above as tcgen05 UMMAs with fp32 accumulators in tensor memory.
 //
@@ -722,17 +722,21 @@ grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     }
 }
 
-// The adjoint chain: one CTA per (batch, head, value tile), chunks in reverse.
+// Both chains of the backward: CTAs x < DV / DVT run the forward chain of value
+// tile x of one (batch, head), the others the adjoint chain of tile x - DV / DVT.
 template <int DV, int DVT>
 __global__ void __launch_bounds__(chain::kChainThreads, 1)
-adj_chain_kernel(const __grid_constant__ CUtensorMap tm_do, const uint8_t *__restrict__ recs,
-                 uint8_t *__restrict__ dsx, const float *dS_T, float *dS0, int H, int n, unsigned int *err)
+chains_kernel(const __grid_constant__ CUtensorMap tm_do, const uint8_t *__restrict__ recs, uint8_t *__restrict__ sx,
+              uint8_t *__restrict__ dsx, const float *S0, const float *dS_T, float *dS0, int H, int n,
+              unsigned int *err)
 {
     using CL = chain::ChainLayout<DV, DVT>;
+    constexpr int NT = DV / DVT;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int tid = threadIdx.x, warp = tid >> 5;
-    const int tile = blockIdx.x, h = blockIdx.y, bi = blockIdx.z;
+    const bool adj = (int)blockIdx.x >= NT;
+    const int tile = adj ? (int)blockIdx.x - NT : (int)blockIdx.x, h = blockIdx.y, bi = blockIdx.z;
     uint32_t *slot = reinterpret_cast<uint32_t *>(sm + CL::SLOT);
     const long pair = (long)bi * H + h;
     if (tid == 0) chain::chain_init<DV, DVT>(sm);
@@ -744,9 +748,14 @@ adj_chain_kernel(const __grid_constant__ CUtensorMap tm_do, const uint8_t *__res
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *slot;
-    const chain::ReverseFlow<DV> f{recs + pair * n * (long)Record<DV>::BYTES, dsx + pair * n * (long)SxSlot<DV>::BYTES,
-                                   &tm_do, n, h, bi};
-    chain::chain_run<DV, DVT, chain::ReverseFlow<DV>, true>(sm, tmem, tid, f, dS_T, dS0, pair, tile, n, err);
+    const uint8_t *r = recs + pair * n * (long)Record<DV>::BYTES;
+    if (adj) {
+        const chain::ReverseFlow<DV> f{r, dsx + pair * n * (long)SxSlot<DV>::BYTES, &tm_do, n, h, bi};
+        chain::chain_run<DV, DVT, chain::ReverseFlow<DV>, true>(sm, tmem, tid, f, dS_T, dS0, pair, tile, n, err);
+    } else {
+        const chain::WindowFlow<DV> f{r, sx + pair * n * (long)SxSlot<DV>::BYTES};
+        chain::chain_run<DV, DVT>(sm, tmem, tid, f, S0, nullptr, pair, tile, n, err);
+    }
     tc_fence_before();
     __syncthreads();
     if (warp == 0) {
@@ -779,15 +788,16 @@ Plan plan(int B, int T, int H, int dv)
 }
 
 template <int DV, int DVT>
-cudaError_t launch_adj(const CUtensorMap &tm_do, const uint8_t *recs, uint8_t *dsx, const float *dS_T, float *dS0,
-                       int B, int H, int n, cudaStream_t s, unsigned int *err)
+cudaError_t launch_chains(const CUtensorMap &tm_do, const uint8_t *recs, uint8_t *sx, uint8_t *dsx, const float *S0,
+                          const float *dS_T, float *dS0, int B, int H, int n, cudaStream_t s, unsigned int *err)
 {
     using CL = chain::ChainLayout<DV, DVT>;
-    auto kern = adj_chain_kernel<DV, DVT>;
+    auto kern = chains_kernel<DV, DVT>;
     static std::atomic<unsigned long long> smem_set{0};
     cudaError_t e = ensure_smem_limit(kern, CL::BYTES, smem_set);
     if (e != cudaSuccess) return e;
-    kern<<<dim3(DV / DVT, H, B), chain::kChainThreads, CL::BYTES, s>>>(tm_do, recs, dsx, dS_T, dS0, H, n, err);
+    kern<<<dim3(2 * (DV / DVT), H, B), chain::kChainThreads, CL::BYTES, s>>>(tm_do, recs, sx, dsx, S0, dS_T, dS0, H,
+                                                                               n, err);
     return cudaGetLastError();
 }
 
@@ -826,16 +836,17 @@ cudaError_t launch_bwd_tc(const BwdArgs &a, uint8_t *ws, unsigned int *err, int 
     gmaps[2] = fmaps[2];
     if (!make_token_map(&gmaps[3], a.dO, a.dv, a.H, a.T, a.B)) return cudaErrorInvalidValue;
 
-    const int dvt = (a.dv == 64 || pl.pairs * 2 <= 148) ? 64 : 128;
+    // value tiles of the chains: 64 wide while both chains' CTAs (four per pair) fit the SMs
+    const int dvt = (a.dv == 64 || pl.pairs * 4 <= num_sms) ? 64 : 128;
     cudaError_t e = launch_prep(f, fmaps, recs, 0, pl.n, pl.n, false, tp);
-    if (e == cudaSuccess) e = launch_chain(f, dvt, recs, sx, a.S0, nullptr, pl.n, pl.n, false);
     if (e == cudaSuccess) {
         if (a.dv == 64)
-            e = launch_adj<64, 64>(gmaps[3], recs, dsx, a.dS_T, a.dS0, a.B, a.H, pl.n, a.stream, err);
+            e = launch_chains<64, 64>(gmaps[3], recs, sx, dsx, a.S0, a.dS_T, a.dS0, a.B, a.H, pl.n, a.stream, err);
         else if (dvt == 64)
-            e = launch_adj<128, 64>(gmaps[3], recs, dsx, a.dS_T, a.dS0, a.B, a.H, pl.n, a.stream, err);
+            e = launch_chains<128, 64>(gmaps[3], recs, sx, dsx, a.S0, a.dS_T, a.dS0, a.B, a.H, pl.n, a.stream, err);
         else
-            e = launch_adj<128, 128>(gmaps[3], recs, dsx, a.dS_T, a.dS0, a.B, a.H, pl.n, a.stream, err);
+            e = launch_chains<128, 128>(gmaps[3], recs, sx, dsx, a.S0, a.dS_T, a.dS0, a.B, a.H, pl.n, a.stream,
+                                        err);
     }
     if (e == cudaSuccess) {
         GradArgs ga{};
