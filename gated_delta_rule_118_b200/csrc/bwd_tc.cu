@@ -80,8 +80,8 @@ struct GradLayout {
     static constexpr int QPROD = MISC + 4096;     // [4][128] quarter products of alpha (bounded form)
     static constexpr int DGC = MISC + 6144;       // [2][128] halves of rowsum(dS' o e^{Gamma_C} S)
     static constexpr int DIAG = MISC + 7168;      // [64] dP_tt
-    static constexpr int BAR = MISC + 7424;       // bar_ld, bar_mma
-    static constexpr int SLOT = BAR + 16;         // tensor-memory address
+    static constexpr int BAR = MISC + 7424;       // bar_ld, bar_mma, bar_raw
+    static constexpr int SLOT = BAR + 32;         // tensor-memory address
     static constexpr int DATA = SLOT + 16;
     static constexpr int BYTES = DATA + 1024;
     // reused by the epilogue, once the products that read them have completed
@@ -90,6 +90,8 @@ struct GradLayout {
     static constexpr int DGS = G;                 // dGamma without K and the diagonal, fp32 [64][128]
     static constexpr int ALPHA = U;               // bounded: alpha, fp32 [64][128] (U and XG)
     static constexpr int RQ = EQ, RB = EQ + 16384, RK = KT;  // bounded: raw q, b, k, bf16 [64][128]
+    // midpoint: raw q, b, k again by TMA for the epilogue (128-byte swizzle, 64-channel halves)
+    static constexpr int TQ = U, TB = XG, TK = TT;
     // tensor-memory columns
     static constexpr uint32_t TM_DX0 = 0, TM_GU = 128, TM_U = 256, TM_DX = 384;  // Ebar S, gU, U, dX
     // dk' holds U dS_c^T, dk2 the pairwise part (dP^T Qhat + dA^T Ehat) once [dP; dA] is read
@@ -128,7 +130,7 @@ grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     const int c = blockIdx.x, h = blockIdx.y, bi = blockIdx.z;
     const int t0 = c * kChunk, Lc = min(kChunk, g.T - t0);
     const long pair = (long)bi * g.H + h, idx = pair * g.n + c;
-    uint64_t *bar_ld = reinterpret_cast<uint64_t *>(sm + L::BAR), *bar_mma = bar_ld + 1;
+    uint64_t *bar_ld = reinterpret_cast<uint64_t *>(sm + L::BAR), *bar_mma = bar_ld + 1, *bar_raw = bar_ld + 2;
     uint32_t *slot = reinterpret_cast<uint32_t *>(sm + L::SLOT);
     float *sig_s = reinterpret_cast<float *>(sm + L::SIG_S), *sig_d = reinterpret_cast<float *>(sm + L::SIG_D);
     float *grv = reinterpret_cast<float *>(sm + L::GRV), *gcv = reinterpret_cast<float *>(sm + L::GCV);
@@ -140,6 +142,7 @@ grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     if (tid == 0) {
         mbar_init(bar_ld, 1);
         mbar_init(bar_mma, 1);
+        mbar_init(bar_raw, 1);
         fence_mbar_init();
         mbar_arrive_expect_tx(bar_ld, (uint32_t)(3 * 16384 + NBV * 8192 + 2 * SXB + 16384));
         for (int kb = 0; kb < 2; ++kb) {
@@ -161,6 +164,25 @@ grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     tc_fence_after();
     const uint32_t tmem = *slot;
     uint32_t mph = 0;
+    // M = 64 accumulators: row t = 16 wq + l sits in lane 32 wq + l (l < 16)
+    const int wq = warp & 3, wh = warp >> 2;
+    const int tr = 16 * wq + lane;
+    const bool row_on = lane < 16;
+    const bool row_live = row_on && tr < Lc;
+    const uint32_t lbase = tmem + ((uint32_t)(32 * wq) << 16);
+    // v and w of this thread's row and value columns [wh HC, +HC), fetched while UMMAs run
+    constexpr int NV = HC / 8;
+    uint4 pv[NV], pw[NV];
+    auto fetch_vw = [&]() {
+#pragma unroll
+        for (int i = 0; i < NV; ++i) {
+            pv[i] = pw[i] = make_uint4(0, 0, 0, 0);
+            if (row_live) {
+                pv[i] = __ldg(reinterpret_cast<const uint4 *>(g.v + tok(tr) * DV + wh * HC + 8 * i));
+                pw[i] = __ldg(reinterpret_cast<const uint4 *>(g.w + tok(tr) * DV + wh * HC + 8 * i));
+            }
+        }
+    };
     auto mma_done = [&]() {
         const bool mine = (tid == 0) ? mbar_wait(bar_mma, mph, g.err) : true;
         mph ^= 1;
@@ -322,19 +344,13 @@ grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                           smem_desc(sbase + L::G + ks * 2048, 16384, 1024, kSw128), idp, 1);
             umma_commit(bar_mma);
         }
+        fetch_vw();
         ok = mma_done();
     }
 
-    // M = 64 accumulators: row t = 16 wq + l sits in lane 32 wq + l (l < 16)
-    const int wq = warp & 3, wh = warp >> 2;
-    const int tr = 16 * wq + lane;
-    const bool row_on = lane < 16;
-    const bool row_live = row_on && tr < Lc;
-    const uint32_t lbase = tmem + ((uint32_t)(32 * wq) << 16);
-
     if (ok) {
         // -------------------------------------------- X = Z - Ebar S -> XG;  gU -> U (bf16, rows = tokens)
-#pragma unroll 1
+#pragma unroll
         for (int cc = 0; cc < HC; cc += 32) {
             const int col = wh * HC + cc;
             float d[32], gu[32];
@@ -346,17 +362,11 @@ grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
 #pragma unroll
                 for (int q8 = 0; q8 < 4; ++q8) {
                     const int cb = col + q8 * 8;
-                    float z[8];
-                    if (row_live) {
-                        float fv[8], fw[8];
-                        unpack8(__ldg(reinterpret_cast<const uint4 *>(g.v + tok(tr) * DV + cb)), fv);
-                        unpack8(__ldg(reinterpret_cast<const uint4 *>(g.w + tok(tr) * DV + cb)), fw);
+                    float z[8], fv[8], fw[8];
+                    unpack8(pv[cc / 8 + q8], fv);
+                    unpack8(pw[cc / 8 + q8], fw);
 #pragma unroll
-                        for (int u = 0; u < 8; ++u) z[u] = fv[u] * fw[u] - d[q8 * 8 + u];
-                    } else {
-#pragma unroll
-                        for (int u = 0; u < 8; ++u) z[u] = -d[q8 * 8 + u];
-                    }
+                    for (int u = 0; u < 8; ++u) z[u] = fv[u] * fw[u] - d[q8 * 8 + u];
                     const uint32_t off = (uint32_t)((cb >> 6) * 8192) + swz_off(tr, (cb & 63) * 2, 128);
                     *reinterpret_cast<uint4 *>(sm + L::XG + off) = pack8(z);
                     *reinterpret_cast<uint4 *>(sm + L::U + off) = pack8(gu + q8 * 8);
@@ -381,12 +391,13 @@ grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                           smem_desc(sbase + L::U + ks * 2048, 8192, 1024, kSw128), idt, ks > 0);
             umma_commit(bar_mma);
         }
+        fetch_vw();
         ok = mma_done();
     }
 
     if (ok) {
         // -------------------------------------------- U -> U;  dv, dw;  -dX -> G
-#pragma unroll 1
+#pragma unroll
         for (int cc = 0; cc < HC; cc += 32) {
             const int col = wh * HC + cc;
             float uu[32], dx[32];
@@ -406,8 +417,8 @@ grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                     *reinterpret_cast<uint4 *>(sm + L::G + (cb >> 6) * 16384 + 8192 + sw) = pack8(nd);
                     if (row_live) {
                         float fv[8], fw[8];
-                        unpack8(__ldg(reinterpret_cast<const uint4 *>(g.v + tok(tr) * DV + cb)), fv);
-                        unpack8(__ldg(reinterpret_cast<const uint4 *>(g.w + tok(tr) * DV + cb)), fw);
+                        unpack8(pv[cc / 8 + q8], fv);
+                        unpack8(pw[cc / 8 + q8], fw);
                         float4 *ov = reinterpret_cast<float4 *>(g.gv + tok(tr) * DV + cb);
                         float4 *ow = reinterpret_cast<float4 *>(g.gw + tok(tr) * DV + cb);
                         const float *x = dx + q8 * 8;
@@ -450,6 +461,15 @@ grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     }
 
     if (ok) {
+        // raw q, b and k for the epilogue, into tiles whose products have completed
+        if (tid == 0 && !bounded) {
+            mbar_arrive_expect_tx(bar_raw, 3 * 16384);
+            for (int kb = 0; kb < 2; ++kb) {
+                tma_load_4d(sm + L::TQ + kb * 8192, &tm_q, bar_raw, kb * 64, h, t0, bi);
+                tma_load_4d(sm + L::TB + kb * 8192, &tm_b, bar_raw, kb * 64, h, t0, bi);
+                tma_load_4d(sm + L::TK + kb * 8192, &tm_k, bar_raw, kb * 64, h, t0, bi);
+            }
+        }
         // -------------------------------------------- [dP; dA] strictly lower -> DPA (bf16, rows t / 64 + t);
         // the diagonal of dP (fp32) -> diag
         {
@@ -535,8 +555,9 @@ grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         const float *xs = reinterpret_cast<const float *>(sm + L::XST);
         const float *alp = reinterpret_cast<const float *>(sm + L::ALPHA);
         float *dgs = reinterpret_cast<float *>(sm + L::DGS), *kst = reinterpret_cast<float *>(sm + L::KST);
+        if (!bounded) ok = named_bar_and(kBar, kGT, (tid == 0) ? mbar_wait(bar_raw, 0, g.err) : true) != 0;
 #pragma unroll 1
-        for (int pass = 0; pass < 4; ++pass) {
+        for (int pass = 0; pass < 4 && ok; ++pass) {
             const int j0 = wh * 64 + pass * 16;
             float aq[16], ae[16], ak[16], ap[16];
             __syncwarp();
@@ -549,16 +570,13 @@ grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
             const int t = tr;
             float qv[16], bv[16], kv[16], fq[16], fk[16];
             if (!bounded) {
-                if (row_live) {
-                    unpack8(__ldg(reinterpret_cast<const uint4 *>(g.q + tok(t) * kDK + j0)), qv);
-                    unpack8(__ldg(reinterpret_cast<const uint4 *>(g.q + tok(t) * kDK + j0 + 8)), qv + 8);
-                    unpack8(__ldg(reinterpret_cast<const uint4 *>(g.b + tok(t) * kDK + j0)), bv);
-                    unpack8(__ldg(reinterpret_cast<const uint4 *>(g.b + tok(t) * kDK + j0 + 8)), bv + 8);
-                    unpack8(__ldg(reinterpret_cast<const uint4 *>(g.k + tok(t) * kDK + j0)), kv);
-                    unpack8(__ldg(reinterpret_cast<const uint4 *>(g.k + tok(t) * kDK + j0 + 8)), kv + 8);
-                } else {
+                // (zero rows past the sequence end, from the TMA's fill)
 #pragma unroll
-                    for (int u = 0; u < 16; ++u) qv[u] = bv[u] = kv[u] = 0.f;
+                for (int h8 = 0; h8 < 16; h8 += 8) {
+                    const uint32_t o = (uint32_t)((j0 >> 6) * 8192) + swz_off(t, ((j0 & 63) + h8) * 2, 128);
+                    unpack8(*reinterpret_cast<const uint4 *>(sm + L::TQ + o), qv + h8);
+                    unpack8(*reinterpret_cast<const uint4 *>(sm + L::TB + o), bv + h8);
+                    unpack8(*reinterpret_cast<const uint4 *>(sm + L::TK + o), kv + h8);
                 }
 #pragma unroll
                 for (int u4 = 0; u4 < 16; u4 += 4) {
