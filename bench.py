@@ -46,7 +46,7 @@ NCU_TRAFFIC_BYTES = {"fwd": 118119424 + 55336448, "train": 4 * (234994176 + 1384
                                                                    + 151028480 + 16768000),
                      "long": 1888002048 + 1315758848, "decode": 281043456 + 212228864,
                      "decode_tokens_T16": 469875456 + 245164288,
-                     "bwd": None}
+                     "bwd": 117527552 + 57630208 + 117638144 + 34749696 + 221228288 + 149556992}
 EXTRA_CASES = ((synth.TRAIN_BF16, "train", 3, 10), (synth.LONG_BF16, "long", 3, 10))
 
 
