@@ -168,6 +168,23 @@ def draw_log_alpha(B, T, H, dk, kind, *, seed):
     raise ValueError(kind)
 
 
+def collinear_keys(d, *, eps, seed, erase_lo=1.95):
+    """Ill-conditioned chunks: within each 64-token chunk of a (batch, head) the
+    keys are one unit direction plus eps * noise (normalised), and the erase gate
+    is drawn in [erase_lo, 2).  Replaces k and b of a forward batch."""
+    B, T, H, dk = d["k"].shape
+    g = torch.Generator(device="cpu").manual_seed(int(seed))
+    nc = (T + 63) // 64
+    base = torch.randn(B, nc, H, dk, generator=g)
+    base = base.repeat_interleave(64, dim=1)[:, :T]
+    k = _l2norm(_l2norm(base) + eps * torch.randn(B, T, H, dk, generator=g))
+    b = erase_lo + (2.0 - erase_lo) * torch.rand(B, T, H, dk, generator=g)
+    out = dict(d)
+    out["k"] = k.to(d["k"].dtype).contiguous()
+    out["b"] = b.to(d["b"].dtype).contiguous()
+    return out
+
+
 def scalar_gates(d, layout, *, seed, gate_sigma=1.0):
     """Replace b, w and/or log_alpha of a forward batch by one value per (token,
     head) ([B,T,H]), as the gdn2_gate_layout bits in `layout` say: bit 1 erase
