@@ -127,6 +127,7 @@ FwdTcPlan plan_fwd_tc(int B, int T, int H, int dv, size_t budget, int num_sms)
     if (wc > p.nchunks) wc = p.nchunks;
     p.wc = (int)wc;
     p.nwindows = p.nchunks ? (p.nchunks + p.wc - 1) / p.wc : 0;
+    if (num_sms > 0 && p.nwindows > 0 && p.slots > p.nwindows) p.slots = p.nwindows;  // no idle slots
     p.rec_total = (size_t)p.wc * bh * p.rec_bytes;
     p.sx_total = (size_t)p.wc * bh * p.sx_bytes;
     p.carry_bytes = p.nwindows > 1 ? (size_t)bh * 128 * dv * sizeof(float) : 0;
