@@ -156,16 +156,21 @@ __device__ __forceinline__ Item decode_item(int n, int P, int bh)
     return {-1, 0, 0};
 }
 
-template <int DV, int DVT>
+// GEN: any gate layout and the fused layer's processing; without it the
+// operator's plain form (per-channel gates, plain outputs), whose code is
+// compiled without those branches.
+template <int DV, int DVT, bool GEN>
 __global__ void __launch_bounds__(kPersistThreads, 1)
 persist_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ CUtensorMap tm_la,
                const __grid_constant__ CUtensorMap tm_g,
-               const bf16 *__restrict__ vg, const bf16 *__restrict__ wg, const prep::GateSrc gs,
-               const outp::OutEpi epi, bf16 *__restrict__ o, const float *S0,
+               const bf16 *__restrict__ vg, const bf16 *__restrict__ wg, const prep::GateSrc gs_arg,
+               const outp::OutEpi epi_arg, bf16 *__restrict__ o, const float *S0,
                float *S_T, uint8_t *__restrict__ recs, uint8_t *__restrict__ sxs, uint32_t *flags, int B, int T,
                int H, int nchain, unsigned int *err)
 {
+    const prep::GateSrc gs = GEN ? gs_arg : prep::GateSrc{gs_arg.b, gs_arg.la, 0u};
+    const outp::OutEpi epi = GEN ? epi_arg : outp::OutEpi{nullptr, nullptr, 0.f};
     using CL = chain::ChainLayout<DV, DVT>;
     constexpr int NT = DV / DVT;  // chain CTAs per head
     extern __shared__ uint8_t smem_raw[];
@@ -328,10 +333,13 @@ cudaError_t launch_persist(const FwdArgs &a, const CUtensorMap *maps, uint8_t *w
     uint32_t *flags = reinterpret_cast<uint32_t *>(ws + p.rec_total + p.sx_total);
     cudaError_t e = cudaMemsetAsync(flags, 0, p.flag_bytes, a.stream);
     if (e != cudaSuccess) return e;
-    auto kern = a.dv == 64 ? persist_kernel<64, 64> : p.dvt == 128 ? persist_kernel<128, 128> : persist_kernel<128, 64>;
+    const bool gen = a.layout != 0 || a.g != nullptr;
+    auto kern = a.dv == 64 ? (gen ? persist_kernel<64, 64, true> : persist_kernel<64, 64, false>)
+                : p.dvt == 128 ? (gen ? persist_kernel<128, 128, true> : persist_kernel<128, 128, false>)
+                               : (gen ? persist_kernel<128, 64, true> : persist_kernel<128, 64, false>);
     const int smem = a.dv == 64 ? persist_smem<64, 64>() : p.dvt == 128 ? persist_smem<128, 128>() : persist_smem<128, 64>();
-    static std::atomic<unsigned long long> smem_set[3] = {};
-    e = ensure_smem_limit(kern, smem, smem_set[a.dv == 64 ? 0 : p.dvt == 128 ? 1 : 2]);
+    static std::atomic<unsigned long long> smem_set[6] = {};
+    e = ensure_smem_limit(kern, smem, smem_set[(a.dv == 64 ? 0 : p.dvt == 128 ? 1 : 2) + (gen ? 3 : 0)]);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg{};
     cudaLaunchAttribute attr[1];
