@@ -249,6 +249,28 @@ cudaError_t run_fwd_tc_overlapped(const FwdArgs &a, const FwdTcPlan &p, uint8_t 
     return e;
 }
 
+// Wide batches, whose chains take most SMs so that prep and chain take turns,
+// with plain outputs: per window the prep, then the chain CTAs, which also
+// compute the window's outputs (fwd_chain_out.cu).  No output pass, no state
+// images in the workspace.
+cudaError_t run_fwd_tc_chain_out(const FwdArgs &a, const FwdTcPlan &p, uint8_t *ws)
+{
+    CUtensorMap maps[5];
+    if (!make_input_maps(a, maps)) return cudaErrorInvalidValue;
+    const size_t slot_bytes = p.rec_total + p.sx_total;
+    float *carry = p.carry_bytes ? reinterpret_cast<float *>(ws + p.slots * slot_bytes) : nullptr;
+    cudaError_t e = cudaSuccess;
+    for (int w = 0; w < p.nwindows && e == cudaSuccess; ++w) {
+        const int c0 = w * p.wc, ncw = (p.nchunks - c0 < p.wc) ? p.nchunks - c0 : p.wc;
+        uint8_t *recs = ws + (w % p.slots) * slot_bytes;
+        const float *S_in = (w == 0) ? a.S0 : carry;
+        float *S_out = (w == p.nwindows - 1) ? a.S_T : carry;
+        e = launch_prep(a, maps, recs, c0, ncw, p.wc, false);
+        if (e == cudaSuccess) e = launch_chain_out(a, p.dvt, recs, S_in, S_out, c0, ncw, p.wc, false);
+    }
+    return e;
+}
+
 // The persistent launch (fwd_persist.cu) for shapes whose chains leave most
 // SMs free; returns false (nothing enqueued) when the device cannot hold the
 // cooperative grid, so that the windowed schedule runs instead.
@@ -293,7 +315,9 @@ cudaError_t launch_fwd_tc(const FwdArgs &a)
     void *ws = nullptr;
     e = cudaMallocFromPoolAsync(&ws, bytes, pool, a.stream);
     if (e != cudaSuccess) return e;
-    {
+    if (!p.overlap && !a.g) {
+        e = run_fwd_tc_chain_out(a, p, static_cast<uint8_t *>(ws));
+    } else {
         std::lock_guard<std::mutex> lock(ss->mu);
         e = run_fwd_tc_overlapped(a, p, static_cast<uint8_t *>(ws), *ss);
     }

@@ -118,6 +118,9 @@ cudaError_t launch_chain(const FwdArgs &a, int dvt, const uint8_t *ws, uint8_t *
                          float *S_out, int ncw, int WC, bool overlap);
 cudaError_t launch_out(const FwdArgs &a, const CUtensorMap *tm_g, const uint8_t *ws, const uint8_t *sx, int c0,
                        int ncw, int WC, bool overlap);
+// The chain of a window with the window's (plain) outputs in the same CTAs.
+cudaError_t launch_chain_out(const FwdArgs &a, int dvt, const uint8_t *ws, const float *S_in, float *S_out, int c0,
+                             int ncw, int WC, bool overlap);
 // Persistent forward (fwd_persist.cu): prep, chain and output work in one
 // cooperative launch of one CTA per SM, records and state images in rings of
 // kRing chunks per (batch, head); the outputs of chunk c are handed out after
