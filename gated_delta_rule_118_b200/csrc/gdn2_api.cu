@@ -299,7 +299,9 @@ extern "C" int gdn2_fwd_chunked_launches(int B, int T, int H, int dk, int dv, gd
         }
         if (sms <= 0) sms = 148;
         if (plan_fwd_persist(B, T, H, dv, sms).use) return 1;
-        return 3 * plan_fwd_tc(B, T, H, dv, kWindowBudgetBytes, sms).nwindows;
+        // per window: prep and chain with the outputs (wide batches), or prep, chain and outputs
+        const FwdTcPlan p = plan_fwd_tc(B, T, H, dv, kWindowBudgetBytes, sms);
+        return (p.overlap ? 3 : 2) * p.nwindows;
     }
     return 1;
 }

@@ -125,9 +125,11 @@ typedef struct CUstream_st *gdn2_stream_t;
  * another (each such wait gives up after one second and reports
  * GDN2_ERR_DEVICE_TIMEOUT); it starts once every SM is free, so kernels of
  * other streams delay it or wait for it.  If the device cannot hold that grid
- * the call falls back to the windowed schedule: three kernels per window of
- * chunks on `stream`, the output kernels on a library-owned side stream that
- * forks from and joins back into `stream`.
+ * the call falls back to the windowed schedule.  There, when the chains take
+ * more than half of the SMs, each window of chunks is two kernels on `stream`:
+ * the prep, then the chains, which also compute the outputs.  Otherwise it is
+ * three kernels per window, with the output kernels on a library-owned side
+ * stream that forks from and joins back into `stream`.
  */
 gdn2_status gdn2_fwd_chunked(const void *q, const void *k, const void *v,
                              const void *b, const void *w, const float *log_alpha,
@@ -308,8 +310,8 @@ gdn2_status gdn2_check_device_error(gdn2_stream_t stream);
  * gdn2_fwd_chunked would reject).  The bf16 path launches one persistent
  * kernel when the sequences' chains (batch * heads * dv / 64 CTAs, or
  * batch * heads from 16384 tokens on) take at most a quarter of the SMs, else
- * three kernels per window of chunks, the
- * window size depending on the device's SM count, which is the only thing this
+ * per window of chunks two kernels (chains on more than half of the SMs) or
+ * three, the window size depending on the device's SM count, which is the only thing this
  * queries (without a device it plans for 148 SMs); the fp32 path launches one
  * kernel.  A zeroing memset of a few kilobytes of flags precedes the persistent
  * kernel and is not counted.
