@@ -60,8 +60,8 @@ constexpr int persist_smem()
                                                                          : kTmemSlot + 16 + 1024;
 }
 static_assert(outp::OutLayout<128>::DATA <= kHalfData, "output region");
-static_assert(chain::ChainLayout<128, 128>::NS >= 3 && chain::ChainLayout<128, 64>::NS >= 3, "chain ring depth");
-static_assert(persist_smem<128, 128>() <= 232448, "shared memory");
+static_assert(chain::ChainLayout<128, 64>::NS >= 3 && chain::ChainLayout<64, 64>::NS >= 3, "chain ring depth");
+static_assert(persist_smem<128, 64>() <= 232448, "shared memory");
 
 struct FlagLayout {
     int bh, nt;
@@ -311,10 +311,11 @@ PersistPlan plan_fwd_persist(int B, int T, int H, int dv, int num_sms)
 {
     PersistPlan p{};
     const long bh = (long)B * H;
-    // Value tile of a chain CTA: a 128-wide tile leaves SMs to the workers (long
-    // sequences are worker-bound: B1 H16 T65536 1.49 -> 1.39 ms), a 64-wide one
-    // steps faster (B1 H16 T4096: 121.6 -> 117.6 us).
-    p.dvt = (dv == 128 && T >= kPersistWideT) ? 128 : 64;
+    // Value tile of a chain CTA: 64 columns.  Its step is shorter than a 128-wide
+    // tile's (B1 H16 T4096: 121.6 -> 117.6 us), and at B1 H16 T65536, where the
+    // wider tile would leave more SMs to the workers, the two measured 1.50 against
+    // 1.75 ms on some devices and 1.48 against 1.46 ms on others.
+    p.dvt = 64;
     const int nt = dv / p.dvt;
     p.nchain = (int)(bh * nt);
     // the chain CTAs must leave most SMs to the workers
@@ -335,11 +336,10 @@ cudaError_t launch_persist(const FwdArgs &a, const CUtensorMap *maps, uint8_t *w
     if (e != cudaSuccess) return e;
     const bool gen = a.layout != 0 || a.g != nullptr;
     auto kern = a.dv == 64 ? (gen ? persist_kernel<64, 64, true> : persist_kernel<64, 64, false>)
-                : p.dvt == 128 ? (gen ? persist_kernel<128, 128, true> : persist_kernel<128, 128, false>)
                                : (gen ? persist_kernel<128, 64, true> : persist_kernel<128, 64, false>);
-    const int smem = a.dv == 64 ? persist_smem<64, 64>() : p.dvt == 128 ? persist_smem<128, 128>() : persist_smem<128, 64>();
-    static std::atomic<unsigned long long> smem_set[6] = {};
-    e = ensure_smem_limit(kern, smem, smem_set[(a.dv == 64 ? 0 : p.dvt == 128 ? 1 : 2) + (gen ? 3 : 0)]);
+    const int smem = a.dv == 64 ? persist_smem<64, 64>() : persist_smem<128, 64>();
+    static std::atomic<unsigned long long> smem_set[4] = {};
+    e = ensure_smem_limit(kern, smem, smem_set[(a.dv == 64 ? 0 : 1) + (gen ? 2 : 0)]);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg{};
     cudaLaunchAttribute attr[1];

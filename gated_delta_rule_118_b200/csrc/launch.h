@@ -129,7 +129,6 @@ cudaError_t launch_chain_out(const FwdArgs &a, int dvt, const uint8_t *ws, const
 // of the chain; outputs are handed out kLag chunks behind it, when they can run.
 constexpr int kRing = 24;
 constexpr int kLag = 16;
-constexpr int kPersistWideT = 16384;  // from this sequence length on, 128-wide chain tiles
 struct PersistPlan {
     bool use;           // the shape suits the persistent launch
     int dvt;            // value tile of a chain CTA

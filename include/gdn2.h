@@ -308,8 +308,8 @@ gdn2_status gdn2_check_device_error(gdn2_stream_t stream);
  * gdn2_fwd_chunked_launches -- number of kernel launches one gdn2_fwd_chunked
  * call on the current device makes for this problem (-1 for arguments
  * gdn2_fwd_chunked would reject).  The bf16 path launches one persistent
- * kernel when the sequences' chains (batch * heads * dv / 64 CTAs, or
- * batch * heads from 16384 tokens on) take at most a quarter of the SMs, else
+ * kernel when the sequences' chains (batch * heads * dv / 64 CTAs) take at
+ * most a quarter of the SMs, else
  * per window of chunks two kernels (chains on more than half of the SMs) or
  * three, the window size depending on the device's SM count, which is the only thing this
  * queries (without a device it plans for 148 SMs); the fp32 path launches one

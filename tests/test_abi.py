@@ -37,8 +37,7 @@ def test_library_is_built_for_sm100a(lib):
 
 def test_launch_count_query(lib):
     # one persistent launch where the chains take at most a quarter of the SMs
-    # (16 heads x 2 value tiles of 64, or one tile of 128 from 16384 tokens on,
-    # of 148), else three per window of chunks
+    # (16 heads x 2 value tiles of 64, of 148), else per window of chunks
     assert g.gdn2_fwd_chunked_launches(1, 4096, 16, 128, 128) == 1
     assert g.gdn2_fwd_chunked_launches(1, 65536, 16, 128, 128) == 1
     # the training batch: prep and chains with the outputs, one window over 64 chunks

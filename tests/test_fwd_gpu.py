@@ -88,14 +88,14 @@ def test_full_size_every_element(case):
 
 
 # The bf16 forward has two schedules: one persistent launch whose chain CTAs
-# (batch * heads * dv / 64, or batch * heads from 16384 tokens on) take at most
-# a quarter of the SMs, with records in rings of 24 chunks per head, and
-# windows of three launches otherwise.
+# (batch * heads * dv / 64) take at most a quarter of the SMs, with records in
+# rings of 24 chunks per head, and windows otherwise (three launches beside the
+# chain, two where prep and chain take turns).
 SCHEDULES = [
     # B, T, H, dv, pairs checked, what it covers
     (1, 2600, 3, 128, None, "persistent, rings wrap, ragged tail"),
     (1, 1500, 2, 64, None, "persistent, dv = 64"),
-    (1, 16500, 1, 128, None, "persistent, 128-wide chain tile, ragged tail"),
+    (1, 16500, 1, 128, None, "persistent, long sequence, ragged tail"),
     (2, 700, 12, 128, [(0, 0), (1, 11)], "windows beside the chain (24 heads x 2 tiles)"),
     (2, 700, 24, 64, [(0, 0), (1, 23)], "windows beside the chain (48 heads, dv = 64)"),
 ]
