@@ -170,7 +170,8 @@ grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     const bool row_on = lane < 16;
     const bool row_live = row_on && tr < Lc;
     const uint32_t lbase = tmem + ((uint32_t)(32 * wq) << 16);
-    // v and w of this thread's row and value columns [wh HC, +HC), fetched while UMMAs run
+    // v and w of this thread's row and value columns [wh HC, +HC), fetched while the first
+    // UMMAs run and kept for both readouts
     constexpr int NV = HC / 8;
     uint4 pv[NV], pw[NV];
     auto fetch_vw = [&]() {
@@ -391,12 +392,11 @@ grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                           smem_desc(sbase + L::U + ks * 2048, 8192, 1024, kSw128), idt, ks > 0);
             umma_commit(bar_mma);
         }
-        fetch_vw();
         ok = mma_done();
     }
 
     if (ok) {
-        // -------------------------------------------- U -> U;  dv, dw;  -dX -> G
+        // -------------------------------------------- U -> U;  dv, dw (v and w still in registers);  -dX -> G
 #pragma unroll
         for (int cc = 0; cc < HC; cc += 32) {
             const int col = wh * HC + cc;
