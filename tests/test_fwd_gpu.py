@@ -96,8 +96,10 @@ SCHEDULES = [
     (1, 2600, 3, 128, None, "persistent, rings wrap, ragged tail"),
     (1, 1500, 2, 64, None, "persistent, dv = 64"),
     (1, 16500, 1, 128, None, "persistent, long sequence, ragged tail"),
-    (2, 700, 12, 128, [(0, 0), (1, 11)], "windows beside the chain (24 heads x 2 tiles)"),
-    (2, 700, 24, 64, [(0, 0), (1, 23)], "windows beside the chain (48 heads, dv = 64)"),
+    (2, 700, 12, 128, None, "windows beside the chain (24 heads x 2 tiles)"),
+    (2, 700, 24, 64, None, "windows beside the chain (48 heads, dv = 64)"),
+    (2, 300, 40, 64, None, "prep, then chains that compute the outputs (80 heads, dv = 64)"),
+    (8, 4500, 16, 128, None, "prep, then chains that compute the outputs: two windows, the state carried"),
 ]
 
 
