@@ -42,7 +42,7 @@ N_INPUT_SETS = 4  # rotating input sets: 4 x 136 MB > 126 MB of L2
 # dram__bytes_read.sum + dram__bytes_write.sum per call from an ncu capture of
 # the current kernels (None once a kernel has changed since the capture), summed
 # over the kernels of one call; the captures are summarised under profiles/.
-NCU_TRAFFIC_BYTES = {"fwd": 118119424 + 55336448, "train": 939820032 + 695288576 + 742467328 + 117185280,
+NCU_TRAFFIC_BYTES = {"fwd": 118233344 + 57096704, "train": 939820032 + 695288576 + 742467328 + 117185280,
                      "long": 1880952832 + 1364458496, "decode": 281043456 + 212228864,
                      "decode_tokens_T16": 469875456 + 245164288,
                      "bwd": 117527552 + 57630208 + 117638144 + 34749696 + 221228288 + 149556992}
