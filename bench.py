@@ -535,6 +535,28 @@ def main():
                              "traffic": NCU_TRAFFIC_BYTES["bwd"]},
                 "launches": 3, "l2": "two input sets (> 126 MB of L2 between calls)"}
     del bsets
+    # the training batch (one input set: 1.1 GB of inputs and dO, larger than L2)
+    tc_ = synth.TRAIN_BF16
+    tb = synth.draw_fwd_device(tc_.B, tc_.T, tc_.H, tc_.dk, tc_.dv, seed=650 + rank, device=dev, dtype=tc_.dtype,
+                               log_alpha_range=tc_.log_alpha_range, gate_sigma=tc_.gate_sigma)
+    tb["dO"] = torch.randn(tc_.B, tc_.T, tc_.H, tc_.dv, device=dev).to(tc_.dtype)
+    g.gdn2_bwd_chunked(*(tb[n] for n in names), None, tb["dO"], check=False)
+    torch.cuda.synchronize()
+    barrier(ws)
+    reps = 3
+    x0.record(stream)
+    for i in range(reps):
+        g.gdn2_bwd_chunked(*(tb[n] for n in names), None, tb["dO"], check=False)
+    x1.record(stream)
+    torch.cuda.synchronize()
+    ms = max_over_ranks(x0.elapsed_time(x1), ws) / reps
+    bb = bwd_algorithmic_bytes(tc_.B, tc_.T, tc_.H, tc_.dk, tc_.dv)
+    bwd_line["train"] = {"workload": tc_.name, "us_per_call": ms * 1e3,
+                         "tokens_per_s": tc_.B * tc_.T * ws / (ms / 1e3),
+                         "roofline": {"bound": "hbm", "achieved": bb / (ms / 1e3) / 1e9, "peak": hbm_peak,
+                                      "unit": "GB/s", "frac": bb / (ms / 1e3) / 1e9 / hbm_peak,
+                                      "algorithmic_bytes_per_call": bb, "traffic": None}}
+    del tb
     if g.gdn2_check_device_error() != g.GDN2_OK:
         raise RuntimeError("device error while timing the backward")
 

@@ -98,9 +98,10 @@ def test_oracle_sized_fp32_workload():
     check(d)
 
 
-@pytest.mark.parametrize("wl", [synth.LAYER_BF16, synth.TRAIN_BF16], ids=lambda c: c.name)
+@pytest.mark.parametrize("wl", [synth.LAYER_BF16, synth.TRAIN_BF16, synth.LONG_BF16], ids=lambda c: c.name)
 def test_full_size_every_gradient(wl):
-    """The layer and the training batch at full size (gradients of the bf16 forward's inputs)."""
+    """The layer, the training batch and the long context at full size (gradients of the
+    bf16 forward's inputs)."""
     d = synth.draw_case(wl)
     gen = torch.Generator().manual_seed(990)
     d["dO"] = torch.randn(wl.B, wl.T, wl.H, wl.dv, generator=gen).to(wl.dtype)
