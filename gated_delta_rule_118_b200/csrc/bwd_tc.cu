@@ -46,6 +46,8 @@
 //   * what remains of dGamma_C is rowsum(dS' o e^{Gamma_C} S).
 #include <cuda.h>
 
+#include <algorithm>
+
 #include "chain_body.cuh"
 #include "launch.h"
 
@@ -82,7 +84,8 @@ struct GradLayout {
     static constexpr int DIAG = MISC + 7168;      // [64] dP_tt
     static constexpr int BAR = MISC + 7424;       // bar_ld, bar_mma, bar_raw
     static constexpr int SLOT = BAR + 32;         // tensor-memory address
-    static constexpr int DATA = SLOT + 16;
+    static constexpr int FIX = SLOT + 16;         // [8] flag masks of the fix-up grid
+    static constexpr int DATA = FIX + 32;
     static constexpr int BYTES = DATA + 1024;
     // reused by the epilogue, once the products that read them have completed
     static constexpr int XST = SR;                // x = Gamma - Gamma_r, fp32 [64][128] (fo layout)
@@ -109,25 +112,32 @@ struct GradArgs {
     const float *la;
     const uint8_t *sx;      // [pairs][n] images of the state entering each chunk
     const uint8_t *dsx;     // [pairs][n] images of dS' (the gradient of the state leaving each chunk)
-    const uint8_t *tp;      // [pairs][n] T and P
+    const uint8_t *tp;      // [pairs][n] T, P and, for ill-conditioned chunks, T - bf16(T) (kTpBytes each)
+    const uint8_t *recs;    // [pairs][n] prep records (the ill-conditioned flag)
     float *gq, *gk, *gb, *gla, *gv, *gw;
     int T, H, n;
     unsigned int *err;
 };
 
-template <int DV>
-__global__ void __launch_bounds__(kGT, 1)
-grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-            const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ CUtensorMap tm_do, const GradArgs g)
+// The gradients of chunk c of (batch bi, head h): one CTA of kGT threads, `sm`
+// the 1024-byte aligned shared memory.  ILL: the chunk's T is far from the
+// identity (the prep's flag), and T and X enter U = T X and dX = T^T gU as bf16
+// pairs (hi + lo): U = T X_hi + T X_lo + T_lo X_hi, dX = T^T gU + T_lo^T gU, for
+// U and dX are then alternating sums whose cancellation would amplify the
+// roundings of bf16 T and X; the CTA then keeps its tensor-memory allocation
+// permit and, unless a wait timed out, leaves its barriers invalidated, so that
+// it may take another chunk.  Returns false when a wait timed out (in-flight
+// copies may then still land).
+template <int DV, bool ILL>
+__device__ __forceinline__ bool grad_chunk(const CUtensorMap &tm_q, const CUtensorMap &tm_k, const CUtensorMap &tm_b,
+                                           const CUtensorMap &tm_do, const GradArgs &g, uint8_t *sm, int c, int h,
+                                           int bi)
 {
     using L = GradLayout;
     constexpr int NBV = DV / 64;           // 64-value blocks
     constexpr int SXB = 128 * DV * 2;      // bytes of a state image
     constexpr int HC = DV / 2;             // value columns per warp half in the M = 64 readouts
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int c = blockIdx.x, h = blockIdx.y, bi = blockIdx.z;
     const int t0 = c * kChunk, Lc = min(kChunk, g.T - t0);
     const long pair = (long)bi * g.H + h, idx = pair * g.n + c;
     uint64_t *bar_ld = reinterpret_cast<uint64_t *>(sm + L::BAR), *bar_mma = bar_ld + 1, *bar_raw = bar_ld + 2;
@@ -144,7 +154,7 @@ grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         mbar_init(bar_mma, 1);
         mbar_init(bar_raw, 1);
         fence_mbar_init();
-        mbar_arrive_expect_tx(bar_ld, (uint32_t)(3 * 16384 + NBV * 8192 + 2 * SXB + 16384));
+        mbar_arrive_expect_tx(bar_ld, (uint32_t)(3 * 16384 + NBV * 8192 + 2 * SXB + 16384 + (ILL ? 8192 : 0)));
         for (int kb = 0; kb < 2; ++kb) {
             tma_load_4d(sm + L::EQ + kb * 16384, &tm_b, bar_ld, kb * 64, h, t0, bi);
             tma_load_4d(sm + L::EQ + kb * 16384 + 8192, &tm_q, bar_ld, kb * 64, h, t0, bi);
@@ -153,11 +163,14 @@ grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         for (int kb = 0; kb < NBV; ++kb) tma_load_4d(sm + L::G + kb * 16384, &tm_do, bar_ld, kb * 64, h, t0, bi);
         bulk_load(sm + L::SR, g.sx + idx * SXB, SXB, bar_ld);
         bulk_load(sm + L::DSC, g.dsx + idx * SXB, SXB, bar_ld);
-        bulk_load(sm + L::TT, g.tp + idx * 16384, 16384, bar_ld);  // T, then P
+        bulk_load(sm + L::TT, g.tp + idx * kTpBytes, 16384, bar_ld);  // T, then P
+        // T - bf16(T) (free space until dP and dA are read out)
+        if (ILL) bulk_load(sm + L::DPA, g.tp + idx * kTpBytes + 16384, 8192, bar_ld);
     }
     if (warp == 0) {
         tmem_alloc(slot, L::TMEM_COLS);
-        tmem_relinquish();
+        // (a CTA that allocates again for its next chunk keeps the permit)
+        if (!ILL) tmem_relinquish();
     }
     tc_fence_before();
     __syncthreads();
@@ -368,9 +381,15 @@ grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                     unpack8(pw[cc / 8 + q8], fw);
 #pragma unroll
                     for (int u = 0; u < 8; ++u) z[u] = fv[u] * fw[u] - d[q8 * 8 + u];
-                    const uint32_t off = (uint32_t)((cb >> 6) * 8192) + swz_off(tr, (cb & 63) * 2, 128);
+                    const uint32_t sw = swz_off(tr, (cb & 63) * 2, 128);
+                    const uint32_t off = (uint32_t)((cb >> 6) * 8192) + sw;
                     *reinterpret_cast<uint4 *>(sm + L::XG + off) = pack8(z);
                     *reinterpret_cast<uint4 *>(sm + L::U + off) = pack8(gu + q8 * 8);
+                    if (ILL) {  // X - bf16(X) into the -dX half of G (free until dX is read out)
+#pragma unroll
+                        for (int u = 0; u < 8; ++u) z[u] -= __bfloat162float(__float2bfloat16_rn(z[u]));
+                        *reinterpret_cast<uint4 *>(sm + L::G + (cb >> 6) * 16384 + 8192 + sw) = pack8(z);
+                    }
                 }
             }
         }
@@ -379,17 +398,30 @@ grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         named_bar(kBar, kGT);
 
         // -------------------------------------------- U = T X,  dX = T^T gU
+        // In ill-conditioned chunks (the prep's flag) T and X are bf16 pairs (hi + lo):
+        // U = T X_hi + T X_lo + T_lo X_hi and dX = T^T gU + T_lo^T gU, as U and dX
+        // are alternating sums whose cancellation would amplify the roundings of
+        // bf16 T and X.
         if (tid == 0) {
             tc_fence_after();
             const uint32_t id = idesc_bf16(64, DV, 0, 1), idt = idesc_bf16(64, DV, 1, 1);
 #pragma unroll
-            for (int ks = 0; ks < 4; ++ks)
-                umma_bf16(tmem + L::TM_U, smem_desc(sbase + L::TT + ks * 32, 16, 1024, kSw128),
-                          smem_desc(sbase + L::XG + ks * 2048, 8192, 1024, kSw128), id, ks > 0);
+            for (int ks = 0; ks < 4; ++ks) {
+                const uint64_t xh = smem_desc(sbase + L::XG + ks * 2048, 8192, 1024, kSw128);
+                umma_bf16(tmem + L::TM_U, smem_desc(sbase + L::TT + ks * 32, 16, 1024, kSw128), xh, id, ks > 0);
+                if (ILL) {
+                    umma_bf16(tmem + L::TM_U, smem_desc(sbase + L::TT + ks * 32, 16, 1024, kSw128),
+                              smem_desc(sbase + L::G + 8192 + ks * 2048, 16384, 1024, kSw128), id, 1);
+                    umma_bf16(tmem + L::TM_U, smem_desc(sbase + L::DPA + ks * 32, 16, 1024, kSw128), xh, id, 1);
+                }
+            }
 #pragma unroll
-            for (int ks = 0; ks < 4; ++ks)
-                umma_bf16(tmem + L::TM_DX, smem_desc(sbase + L::TT + ks * 2048, 8192, 1024, kSw128),
-                          smem_desc(sbase + L::U + ks * 2048, 8192, 1024, kSw128), idt, ks > 0);
+            for (int ks = 0; ks < 4; ++ks) {
+                const uint64_t gu = smem_desc(sbase + L::U + ks * 2048, 8192, 1024, kSw128);
+                umma_bf16(tmem + L::TM_DX, smem_desc(sbase + L::TT + ks * 2048, 8192, 1024, kSw128), gu, idt, ks > 0);
+                if (ILL)
+                    umma_bf16(tmem + L::TM_DX, smem_desc(sbase + L::DPA + ks * 2048, 8192, 1024, kSw128), gu, idt, 1);
+            }
             umma_commit(bar_mma);
         }
         ok = mma_done();
@@ -732,12 +764,71 @@ grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         }
     }
 
+    // (the next chunk's copies land where this one's threads wrote)
+    if (ILL) fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
     if (warp == 0) {
         tc_fence_after();
         tmem_dealloc(tmem, L::TMEM_COLS);
     }
+    if (ILL && ok && tid == 0) {
+        mbar_inval(bar_ld);
+        mbar_inval(bar_mma);
+        mbar_inval(bar_raw);
+    }
+    return ok;
+}
+
+template <int DV>
+__global__ void __launch_bounds__(kGT, 1)
+grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+            const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ CUtensorMap tm_do, const GradArgs g)
+{
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    // the fix-up grid (below) may take the SMs this grid's last CTAs leave
+    allow_dependent_launch();
+    grad_chunk<DV, false>(tm_q, tm_k, tm_b, tm_do, g, sm, blockIdx.x, blockIdx.y, blockIdx.z);
+}
+
+// The chunks the prep flagged (T far from the identity) again, with the bf16
+// pairs, over the gradients grad_kernel wrote for them.  Launched as a
+// programmatic dependent of grad_kernel with up to one CTA per SM: CTA x takes
+// the chunks x, x + gridDim.x, ... of the [pairs][n] order, reads their flags
+// while grad_kernel runs, and waits for it to end before its first chunk.
+template <int DV>
+__global__ void __launch_bounds__(kGT, 1)
+grad_fix_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ CUtensorMap tm_do, const GradArgs g,
+                long total)
+{
+    using L = GradLayout;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint32_t *masks = reinterpret_cast<uint32_t *>(sm + L::FIX);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    bool ok = true;
+    for (long j0 = 0; ok && (long)blockIdx.x + (long)gridDim.x * j0 < total; j0 += kGT) {
+        const long idx = (long)blockIdx.x + (long)gridDim.x * (j0 + tid);
+        const bool f = idx < total && *reinterpret_cast<const uint32_t *>(g.recs + idx * (long)Record<DV>::BYTES +
+                                                                           Record<DV>::DEC + 512) != 0;
+        const uint32_t m = __ballot_sync(0xffffffffu, f);
+        if (lane == 0) masks[warp] = m;
+        if (!__syncthreads_or(f)) continue;
+        wait_prior_grid();
+        for (int w = 0; ok && w < kGT / 32; ++w) {
+            for (uint32_t mw = masks[w]; ok && mw; mw &= mw - 1) {
+                const long ci = (long)blockIdx.x + (long)gridDim.x * (j0 + w * 32 + __ffs(mw) - 1);
+                const long pair = ci / g.n;
+                ok = grad_chunk<DV, true>(tm_q, tm_k, tm_b, tm_do, g, sm, (int)(ci % g.n), (int)(pair % g.H),
+                                          (int)(pair / g.H));
+            }
+        }
+        __syncthreads();  // masks of this round read by all before the next round writes them
+    }
+    // end only after grad_kernel, whose outputs this grid overwrites
+    wait_prior_grid();
 }
 
 // Both chains of the backward: CTAs x < DV / DVT run the forward chain of value
@@ -798,7 +889,7 @@ Plan plan(int B, int T, int H, int dv)
     const size_t per = (size_t)p.pairs * p.n;
     size_t off = 0;
     p.rec = off; off += per * rb;
-    p.tp = off; off += per * 16384;
+    p.tp = off; off += per * kTpBytes;
     p.sx = off; off += per * xb;
     p.dsx = off; off += per * xb;
     p.total = off;
@@ -820,14 +911,19 @@ cudaError_t launch_chains(const CUtensorMap &tm_do, const uint8_t *recs, uint8_t
 }
 
 template <int DV>
-cudaError_t launch_grad(const CUtensorMap *maps, const GradArgs &ga, int B, cudaStream_t s)
+cudaError_t launch_grad(const CUtensorMap *maps, const GradArgs &ga, int B, cudaStream_t s, int num_sms)
 {
     auto kern = grad_kernel<DV>;
-    static std::atomic<unsigned long long> smem_set{0};
+    auto fix = grad_fix_kernel<DV>;
+    static std::atomic<unsigned long long> smem_set{0}, fix_smem_set{0};
     cudaError_t e = ensure_smem_limit(kern, GradLayout::BYTES, smem_set);
+    if (e == cudaSuccess) e = ensure_smem_limit(fix, GradLayout::BYTES, fix_smem_set);
     if (e != cudaSuccess) return e;
     kern<<<dim3(ga.n, ga.H, B), kGT, GradLayout::BYTES, s>>>(maps[0], maps[1], maps[2], maps[3], ga);
-    return cudaGetLastError();
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    const long total = (long)B * ga.H * ga.n;
+    LaunchCfg lc(dim3((unsigned)std::min<long>(total, num_sms)), dim3(kGT), GradLayout::BYTES, s, true);
+    return cudaLaunchKernelEx(&lc.cfg, fix, maps[0], maps[1], maps[2], maps[3], ga, total);
 }
 
 }  // namespace bwdtc
@@ -870,10 +966,11 @@ cudaError_t launch_bwd_tc(const BwdArgs &a, uint8_t *ws, unsigned int *err, int 
         GradArgs ga{};
         ga.q = (const bf16 *)a.q; ga.k = (const bf16 *)a.k; ga.b = (const bf16 *)a.b;
         ga.v = (const bf16 *)a.v; ga.w = (const bf16 *)a.w; ga.la = a.log_alpha;
-        ga.sx = sx; ga.dsx = dsx; ga.tp = tp;
+        ga.sx = sx; ga.dsx = dsx; ga.tp = tp; ga.recs = recs;
         ga.gq = a.gq; ga.gk = a.gk; ga.gb = a.gb; ga.gla = a.gla; ga.gv = a.gv; ga.gw = a.gw;
         ga.T = a.T; ga.H = a.H; ga.n = pl.n; ga.err = err;
-        e = a.dv == 128 ? launch_grad<128>(gmaps, ga, a.B, a.stream) : launch_grad<64>(gmaps, ga, a.B, a.stream);
+        e = a.dv == 128 ? launch_grad<128>(gmaps, ga, a.B, a.stream, num_sms)
+                         : launch_grad<64>(gmaps, ga, a.B, a.stream, num_sms);
     }
     return e;
 }

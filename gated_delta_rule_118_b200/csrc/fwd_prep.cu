@@ -12,8 +12,8 @@ namespace {
 using namespace sm100;
 using namespace prep;
 
-// TP: the backward's prep, which also keeps every chunk's T and P in `tp`
-// (16 KB per chunk, indexed like the records).
+// TP: the backward's prep, which also keeps every chunk's T, P and the low
+// part of T in `tp` (kTpBytes per chunk, indexed like the records).
 template <int DV, bool TP>
 __global__ void __launch_bounds__(kPrepThreads, 2)
 prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -52,7 +52,7 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     const uint32_t tmem = *slot;
     uint32_t mma_phase = 0;
     prep_chunk<DV, TP>(sm, tmem, tid, 0, bar_tma, 0, bar_mma, mma_phase, vg, wg, gs, rec, Tlen, H, t0, h, bi, err,
-                       TP ? tp + idx * 16384 : nullptr);
+                       TP ? tp + idx * kTpBytes : nullptr);
     tc_fence_before();
     __syncthreads();
     if (warp == 0) {

@@ -111,7 +111,9 @@ cudaError_t launch_fwd_tc(const FwdArgs &a);
 // `overlap`: launch as a programmatic dependent of the previous kernel in the
 // stream, so that it may start before that kernel ends (only where the two
 // touch disjoint data).
-// tp: non-null for the backward, which keeps every chunk's T and P there (16 KB per record).
+// tp: non-null for the backward, which keeps every chunk's T, P and T - bf16(T) there
+// (kTpBytes per record).
+constexpr int kTpBytes = 3 * 8192;
 cudaError_t launch_prep(const FwdArgs &a, const CUtensorMap *maps, uint8_t *ws, int c0, int ncw, int WC,
                         bool overlap, uint8_t *tp = nullptr);
 cudaError_t launch_chain(const FwdArgs &a, int dvt, const uint8_t *ws, uint8_t *sx, const float *S_in,

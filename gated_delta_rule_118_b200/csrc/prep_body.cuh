@@ -83,6 +83,10 @@ struct GateSrc {
 constexpr unsigned kEraseScalar = 1u, kWriteScalar = 2u, kDecayScalar = 4u;  // gdn2_gate_layout bits
 constexpr unsigned kLayerInputs = 8u;  // raw q, k and gate logits (the fused layer entry point)
 constexpr float kL2Eps = 1e-6f;
+// T entries off the identity by more than this mark an ill-conditioned chunk for
+// the backward (random keys stay below 0.35 on every workload; nearly collinear
+// keys with erase gates near 2 reach 0.4 to 1.8)
+constexpr float kIllT = 0.5f;
 
 // sigmoid(x) = (1 + tanh(x / 2)) / 2, one MUFU operation (tanh.approx.f32,
 // relative error about 2^-11: below the bf16 rounding of the gates)
@@ -343,8 +347,11 @@ static __device__ __noinline__ void prep_bounded(uint8_t *sm, int tid, int bar_i
 // (1024-byte aligned), `tmem` the first of their 256 tensor-memory columns,
 // `bar_mma` an mbarrier for UMMA completion whose phase parity `mma_phase`
 // tracks, and `rec` the chunk's record.  With TP (the backward) the chunk's T
-// and P also go to `tp`: two bf16 [64][64] tiles (T, then P), rows of 128 bytes
-// with the 128-byte swizzle, as they sit in shared memory.  Returns false
+// and P also go to `tp`: bf16 [64][64] tiles T and P, rows of 128 bytes with the
+// 128-byte swizzle, as they sit in shared memory.  A chunk whose T has an entry
+// off the identity by more than kIllT (nearly collinear keys with erase gates
+// near 2: its products with T are alternating sums) also gets a third tile,
+// T - bf16(T), and a nonzero word at byte 512 of the record's decay area.  Returns false
 // (every thread alike) when a wait timed out.
 template <int DV, bool TP = false>
 __device__ __forceinline__ bool prep_chunk(uint8_t *sm, uint32_t tmem, int tid, int bar_id, uint64_t *bar_tma,
@@ -587,6 +594,7 @@ __device__ __forceinline__ bool prep_chunk(uint8_t *sm, uint32_t tmem, int tid, 
             named_bar(bar_id, kPrepThreads);
         }
 
+        bool ill = false;  // (the backward) T far from the identity
         // ---------------------------------------------------------- T = (I + A)^{-1}
         // (a) diagonal 16x16 blocks: one column per thread, rows of A read as float4
         if (tid < 64) {
@@ -698,9 +706,30 @@ __device__ __forceinline__ bool prep_chunk(uint8_t *sm, uint32_t tmem, int tid, 
             }
             *reinterpret_cast<uint4 *>(sm + L::TB + swz_off(t, g * 2, 128)) = pack8(f);
             *reinterpret_cast<uint4 *>(sm + L::TB + swz_off(t, g * 2 + 16, 128)) = pack8(f + 8);
+            if (TP) {
+#pragma unroll
+                for (int u = 0; u < 16; ++u) ill = ill || fabsf(f[u] - (g + u == t ? 1.f : 0.f)) > kIllT;
+            }
         }
         fence_proxy_async_smem();
-        named_bar(bar_id, kPrepThreads);
+        if (TP)
+            ill = !named_bar_and(bar_id, kPrepThreads, !ill);
+        else
+            named_bar(bar_id, kPrepThreads);
+        if (TP && ill) {  // what the bf16 image of T drops (the fp32 T is still in place)
+            const int t = tid >> 2, g = (tid & 3) * 16;
+            float f[16];
+#pragma unroll
+            for (int u = 0; u < 16; u += 4) {
+                const float4 v4 = *reinterpret_cast<const float4 *>(Tf + af_off(t, g + u));
+                f[u] = v4.x; f[u + 1] = v4.y; f[u + 2] = v4.z; f[u + 3] = v4.w;
+            }
+#pragma unroll
+            for (int u = 0; u < 16; ++u) f[u] -= __bfloat162float(__float2bfloat16_rn(f[u]));
+            *reinterpret_cast<uint4 *>(tp + 16384 + swz_off(t, g * 2, 128)) = pack8(f);
+            *reinterpret_cast<uint4 *>(tp + 16384 + swz_off(t, g * 2 + 16, 128)) = pack8(f + 8);
+        }
+        if (TP && tid == 0) *reinterpret_cast<uint32_t *>(rec + R::DEC + 512) = ill ? 1u : 0u;
         if (TP) {  // T and P, final from here on, for the backward
 #pragma unroll
             for (int m = 0; m < 2; ++m) {

@@ -38,12 +38,14 @@ def test_forward_near_singular_chunks(T, dtype, eps):
     assert eo <= tol and es <= tol, (eo, es)
 
 
-@pytest.mark.parametrize("dtype,eps", [(torch.bfloat16, 0.1), (torch.float32, 0.02)], ids=["bf16", "f32"])
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32], ids=["bf16", "f32"])
+@pytest.mark.parametrize("eps", [0.02, 0.1, 0.3])
 def test_backward_near_singular_chunks(dtype, eps):
-    """bf16 at key noise 0.1; fp32 at 0.02.  At 0.02 (cosines >= 0.93 within a
-    chunk, erase gates in [1.95, 2)) the bf16 gradient of q comes to about 2e-2:
-    the alternating sums of near-reflections amplify the bf16 rounding of the
-    operands X and T of U = T X."""
+    """Key noise 0.02 (cosines >= 0.93 within a chunk), 0.1 and 0.3, erase gates in
+    [1.95, 2).  In bf16 the chunks are flagged ill-conditioned (T off the identity
+    by more than 0.5) and U = T X, dX = T^T gU take T and X as bf16 pairs: the
+    alternating sums of near-reflections would otherwise amplify their rounding
+    (about 2e-2 on dq at key noise 0.02)."""
     d = case(200, dtype, 8300, eps)
     gen = torch.Generator().manual_seed(8301)
     d["dO"] = torch.randn(1, 200, 2, 128, generator=gen).to(dtype)
@@ -54,3 +56,28 @@ def test_backward_near_singular_chunks(dtype, eps):
     tol = TOL_BF16 if dtype == torch.bfloat16 else TOL_F32
     errs = {n: rel_err(got[n], ref[n]) for n in GRADS}
     assert all(e <= tol for e in errs.values()), ", ".join(f"{n} {e:.3g}" for n, e in errs.items())
+
+
+def test_backward_flagged_chunks_beyond_one_per_sm():
+    """256 chunks (more than one per SM, so that the CTAs that recompute the
+    flagged chunks take several each), near-collinear keys in the even chunks
+    of every (batch, head) and random ones in the odd: the flagged chunks get
+    the bf16 pairs, the others keep the plain path's gradients.  Sequences of
+    four chunks: with erase gates near 2 the chunks are near-reflections, and
+    over long sequences the bf16 records of the state chains (not the chunk
+    gradients) would set the error."""
+    B, T, H = 8, 256, 8
+    d = synth.draw_fwd(B, T, H, 128, 128, seed=8400, dtype=torch.bfloat16, s0_sigma=0.05)
+    ill = synth.collinear_keys(d, eps=0.02, seed=8401)
+    even = ((torch.arange(T) // 64) % 2 == 0).view(1, T, 1, 1)
+    for n in ("k", "b"):
+        d[n] = torch.where(even, ill[n], d[n]).contiguous()
+    gen = torch.Generator().manual_seed(8402)
+    d["dO"] = torch.randn(B, T, H, 128, generator=gen).to(torch.bfloat16)
+    d["dS_T"] = torch.randn(B, H, 128, 128, generator=gen)
+    dd = to_dev(d)
+    got = g.gdn2_bwd_chunked(*(dd[n] for n in NAMES), dd["S0"], dd["dO"], dd["dS_T"])
+    assert g.gdn2_check_device_error() == g.GDN2_OK
+    ref = oracle.bwd(*(d[n] for n in NAMES), d["S0"], d["dO"], d["dS_T"])
+    errs = {n: rel_err(got[n], ref[n]) for n in GRADS}
+    assert all(e <= TOL_BF16 for e in errs.values()), ", ".join(f"{n} {e:.3g}" for n, e in errs.items())
