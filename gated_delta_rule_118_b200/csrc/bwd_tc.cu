@@ -46,8 +46,6 @@
 //   * what remains of dGamma_C is rowsum(dS' o e^{Gamma_C} S).
 #include <cuda.h>
 
-#include <algorithm>
-
 #include "chain_body.cuh"
 #include "launch.h"
 
@@ -84,8 +82,7 @@ struct GradLayout {
     static constexpr int DIAG = MISC + 7168;      // [64] dP_tt
     static constexpr int BAR = MISC + 7424;       // bar_ld, bar_mma, bar_raw
     static constexpr int SLOT = BAR + 32;         // tensor-memory address
-    static constexpr int FIX = SLOT + 16;         // [8] flag masks of the fix-up grid
-    static constexpr int DATA = FIX + 32;
+    static constexpr int DATA = SLOT + 16;
     static constexpr int BYTES = DATA + 1024;
     // reused by the epilogue, once the products that read them have completed
     static constexpr int XST = SR;                // x = Gamma - Gamma_r, fp32 [64][128] (fo layout)
@@ -124,9 +121,7 @@ struct GradArgs {
 // identity (the prep's flag), and T and X enter U = T X and dX = T^T gU as bf16
 // pairs (hi + lo): U = T X_hi + T X_lo + T_lo X_hi, dX = T^T gU + T_lo^T gU, for
 // U and dX are then alternating sums whose cancellation would amplify the
-// roundings of bf16 T and X; the CTA then keeps its tensor-memory allocation
-// permit and, unless a wait timed out, leaves its barriers invalidated, so that
-// it may take another chunk.  Returns false when a wait timed out (in-flight
+// roundings of bf16 T and X.  Returns false when a wait timed out (in-flight
 // copies may then still land).
 template <int DV, bool ILL>
 __device__ __forceinline__ bool grad_chunk(const CUtensorMap &tm_q, const CUtensorMap &tm_k, const CUtensorMap &tm_b,
@@ -168,9 +163,8 @@ __device__ __forceinline__ bool grad_chunk(const CUtensorMap &tm_q, const CUtens
         if (ILL) bulk_load(sm + L::DPA, g.tp + idx * kTpBytes + 16384, 8192, bar_ld);
     }
     if (warp == 0) {
+        // (no relinquish: a flagged chunk allocates again for its second pass)
         tmem_alloc(slot, L::TMEM_COLS);
-        // (a CTA that allocates again for its next chunk keeps the permit)
-        if (!ILL) tmem_relinquish();
     }
     tc_fence_before();
     __syncthreads();
@@ -764,71 +758,53 @@ __device__ __forceinline__ bool grad_chunk(const CUtensorMap &tm_q, const CUtens
         }
     }
 
-    // (the next chunk's copies land where this one's threads wrote)
-    if (ILL) fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
     if (warp == 0) {
         tc_fence_after();
         tmem_dealloc(tmem, L::TMEM_COLS);
     }
-    if (ILL && ok && tid == 0) {
-        mbar_inval(bar_ld);
-        mbar_inval(bar_mma);
-        mbar_inval(bar_raw);
-    }
     return ok;
 }
 
+// The bf16-pair pass, out of line: the plain pass keeps its schedule.
+template <int DV>
+__device__ __noinline__ void grad_chunk_pairs(const CUtensorMap &tm_q, const CUtensorMap &tm_k, const CUtensorMap &tm_b,
+                                              const CUtensorMap &tm_do, const GradArgs &g, uint8_t *sm, int c, int h,
+                                              int bi)
+{
+    grad_chunk<DV, true>(tm_q, tm_k, tm_b, tm_do, g, sm, c, h, bi);
+}
+
+// One CTA per (chunk, head, batch).  A chunk the prep flagged (T far from the
+// identity) is computed twice: the plain pass, then the bf16-pair pass over its
+// gradients.
 template <int DV>
 __global__ void __launch_bounds__(kGT, 1)
 grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-            const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ CUtensorMap tm_do, const GradArgs g)
-{
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    // the fix-up grid (below) may take the SMs this grid's last CTAs leave
-    allow_dependent_launch();
-    grad_chunk<DV, false>(tm_q, tm_k, tm_b, tm_do, g, sm, blockIdx.x, blockIdx.y, blockIdx.z);
-}
-
-// The chunks the prep flagged (T far from the identity) again, with the bf16
-// pairs, over the gradients grad_kernel wrote for them.  Launched as a
-// programmatic dependent of grad_kernel with up to one CTA per SM: CTA x takes
-// the chunks x, x + gridDim.x, ... of the [pairs][n] order, reads their flags
-// while grad_kernel runs, and waits for it to end before its first chunk.
-template <int DV>
-__global__ void __launch_bounds__(kGT, 1)
-grad_fix_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ CUtensorMap tm_do, const GradArgs g,
-                long total)
+            const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ CUtensorMap tm_do,
+            const __grid_constant__ GradArgs g)
 {
     using L = GradLayout;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint32_t *masks = reinterpret_cast<uint32_t *>(sm + L::FIX);
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    bool ok = true;
-    for (long j0 = 0; ok && (long)blockIdx.x + (long)gridDim.x * j0 < total; j0 += kGT) {
-        const long idx = (long)blockIdx.x + (long)gridDim.x * (j0 + tid);
-        const bool f = idx < total && *reinterpret_cast<const uint32_t *>(g.recs + idx * (long)Record<DV>::BYTES +
-                                                                           Record<DV>::DEC + 512) != 0;
-        const uint32_t m = __ballot_sync(0xffffffffu, f);
-        if (lane == 0) masks[warp] = m;
-        if (!__syncthreads_or(f)) continue;
-        wait_prior_grid();
-        for (int w = 0; ok && w < kGT / 32; ++w) {
-            for (uint32_t mw = masks[w]; ok && mw; mw &= mw - 1) {
-                const long ci = (long)blockIdx.x + (long)gridDim.x * (j0 + w * 32 + __ffs(mw) - 1);
-                const long pair = ci / g.n;
-                ok = grad_chunk<DV, true>(tm_q, tm_k, tm_b, tm_do, g, sm, (int)(ci % g.n), (int)(pair % g.H),
-                                          (int)(pair / g.H));
-            }
+    const int tid = threadIdx.x, c = blockIdx.x, h = blockIdx.y, bi = blockIdx.z;
+    // the prep's flag, issued now and first used after the plain pass
+    uint32_t flag = 0;
+    if (tid == 0)
+        flag = ld_nc_u32(g.recs + (((long)bi * g.H + h) * g.n + c) * (long)Record<DV>::BYTES + Record<DV>::DEC + 512);
+    const bool ok = grad_chunk<DV, false>(tm_q, tm_k, tm_b, tm_do, g, sm, c, h, bi);
+    // (the second pass's copies land where the first pass's threads wrote)
+    fence_proxy_async_smem();
+    if (__syncthreads_or(flag != 0) && ok) {
+        if (tid == 0) {
+            uint64_t *bar = reinterpret_cast<uint64_t *>(sm + L::BAR);
+            mbar_inval(bar);
+            mbar_inval(bar + 1);
+            mbar_inval(bar + 2);
         }
-        __syncthreads();  // masks of this round read by all before the next round writes them
+        grad_chunk_pairs<DV>(tm_q, tm_k, tm_b, tm_do, g, sm, c, h, bi);
     }
-    // end only after grad_kernel, whose outputs this grid overwrites
-    wait_prior_grid();
 }
 
 // Both chains of the backward: CTAs x < DV / DVT run the forward chain of value
@@ -911,19 +887,14 @@ cudaError_t launch_chains(const CUtensorMap &tm_do, const uint8_t *recs, uint8_t
 }
 
 template <int DV>
-cudaError_t launch_grad(const CUtensorMap *maps, const GradArgs &ga, int B, cudaStream_t s, int num_sms)
+cudaError_t launch_grad(const CUtensorMap *maps, const GradArgs &ga, int B, cudaStream_t s)
 {
     auto kern = grad_kernel<DV>;
-    auto fix = grad_fix_kernel<DV>;
-    static std::atomic<unsigned long long> smem_set{0}, fix_smem_set{0};
+    static std::atomic<unsigned long long> smem_set{0};
     cudaError_t e = ensure_smem_limit(kern, GradLayout::BYTES, smem_set);
-    if (e == cudaSuccess) e = ensure_smem_limit(fix, GradLayout::BYTES, fix_smem_set);
     if (e != cudaSuccess) return e;
     kern<<<dim3(ga.n, ga.H, B), kGT, GradLayout::BYTES, s>>>(maps[0], maps[1], maps[2], maps[3], ga);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    const long total = (long)B * ga.H * ga.n;
-    LaunchCfg lc(dim3((unsigned)std::min<long>(total, num_sms)), dim3(kGT), GradLayout::BYTES, s, true);
-    return cudaLaunchKernelEx(&lc.cfg, fix, maps[0], maps[1], maps[2], maps[3], ga, total);
+    return cudaGetLastError();
 }
 
 }  // namespace bwdtc
@@ -969,8 +940,7 @@ cudaError_t launch_bwd_tc(const BwdArgs &a, uint8_t *ws, unsigned int *err, int 
         ga.sx = sx; ga.dsx = dsx; ga.tp = tp; ga.recs = recs;
         ga.gq = a.gq; ga.gk = a.gk; ga.gb = a.gb; ga.gla = a.gla; ga.gv = a.gv; ga.gw = a.gw;
         ga.T = a.T; ga.H = a.H; ga.n = pl.n; ga.err = err;
-        e = a.dv == 128 ? launch_grad<128>(gmaps, ga, a.B, a.stream, num_sms)
-                         : launch_grad<64>(gmaps, ga, a.B, a.stream, num_sms);
+        e = a.dv == 128 ? launch_grad<128>(gmaps, ga, a.B, a.stream) : launch_grad<64>(gmaps, ga, a.B, a.stream);
     }
     return e;
 }

@@ -28,6 +28,15 @@ __device__ __forceinline__ void fence_mbar_init()
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
 }
 
+// A 32-bit load of data this kernel does not write, issued where it stands
+// (volatile), so that its latency overlaps the work before its first use.
+__device__ __forceinline__ uint32_t ld_nc_u32(const void *p)
+{
+    uint32_t v;
+    asm volatile("ld.global.nc.u32 %0, [%1];" : "=r"(v) : "l"(p));
+    return v;
+}
+
 // Invalidate an mbarrier with no phase pending, so that its word may be initialised again.
 __device__ __forceinline__ void mbar_inval(uint64_t *bar)
 {

@@ -277,10 +277,10 @@ gdn2_status gdn2_layer_fwd(const void *q, const void *k, const void *v,
  *   bf16 inputs with dk = 128: tensor cores (bf16 operands, fp32 accumulation
  *     and state), within the bf16 tolerance of the forward.  A chunk whose
  *     T = (I + A)^{-1} has an entry off the identity by more than 0.5 (nearly
- *     collinear keys with erase gates near 2) is recomputed by a fourth kernel
- *     with T and X = Z - Ebar S (the chunk's written values less what its
- *     erases read from the entry state) as bf16 pairs (hi + lo), over the plain
- *     kernel's gradients for it: four launches a call;
+ *     collinear keys with erase gates near 2) is computed a second time by the
+ *     same CTA, with T and X = Z - Ebar S (the chunk's written values less what
+ *     its erases read from the entry state) as bf16 pairs (hi + lo), over its
+ *     plain gradients; three launches a call;
  *   fp32 inputs, and dk = 64: fp32 on the CUDA cores.
  *
  *   q, k, v, b, w, log_alpha, S0, B, T, H, dk, dv, dtype   as for gdn2_fwd_chunked
