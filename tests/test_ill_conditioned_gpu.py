@@ -42,10 +42,11 @@ def test_forward_near_singular_chunks(T, dtype, eps):
 @pytest.mark.parametrize("eps", [0.02, 0.1, 0.3])
 def test_backward_near_singular_chunks(dtype, eps):
     """Key noise 0.02 (cosines >= 0.93 within a chunk), 0.1 and 0.3, erase gates in
-    [1.95, 2).  In bf16 the chunks are flagged ill-conditioned (T off the identity
-    by more than 0.5) and U = T X, dX = T^T gU take T and X as bf16 pairs: the
+    [1.95, 2).  In bf16 a chunk whose T lies more than 0.5 off the identity is
+    computed again with T and X as bf16 pairs in U = T X and dX = T^T gU: the
     alternating sums of near-reflections would otherwise amplify their rounding
-    (about 2e-2 on dq at key noise 0.02)."""
+    (about 2e-2 on dq at key noise 0.02).  Every chunk crosses that threshold at
+    0.02 and 0.1; at 0.3 chunks lie on both sides of it."""
     d = case(200, dtype, 8300, eps)
     gen = torch.Generator().manual_seed(8301)
     d["dO"] = torch.randn(1, 200, 2, 128, generator=gen).to(dtype)

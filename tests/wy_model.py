@@ -50,6 +50,17 @@ def chunk_record(q, k, b, la, C):
     return np.exp(G[-1]), NG, QS, Y, PT
 
 
+def chunk_T(k, b, la, C):
+    """T = (I + A)^{-1} of one chunk of L <= C tokens, A formed from the midpoint
+    factors as in chunk_record."""
+    L = k.shape[0]
+    G = np.cumsum(la, axis=0)
+    r = min(C // 2, L)
+    Gr = G[r - 1] if r > 0 else np.zeros_like(G[0])
+    A = np.tril((np.exp(G - Gr) * (b * k)) @ (np.exp(Gr - G) * k).T, -1)
+    return np.linalg.inv(np.eye(L) + A)
+
+
 def chunk_step(q, k, v, b, w, la, S, C):
     """One chunk of L <= C tokens for one (batch, head): returns (O, S_C)."""
     gc, NG, QS, Y, PT = chunk_record(q, k, b, la, C)
