@@ -1,0 +1,89 @@
+"""The chunkwise backward's algebra (fp64 model of what the tensor-core backward
+computes) equals the oracle's gradients, and the bf16-pair products for chunks
+with T far from the identity remove the share of the error that the rounding
+of T and X contributes (CPU)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from oracle_pins import _inputs
+from wy_bwd_model import wy_backward
+
+GRADS = ("dq", "dk", "dv", "db", "dw", "dlog_alpha", "dS0")
+
+
+def rel(got, ref):
+    ref = np.asarray(ref)
+    return float(np.abs(got - ref).max() / np.abs(ref).max())
+
+
+def grads_case(T, dk, dv, seed, *, B=1, H=2, wide=False):
+    q, k, v, b, w, la, s0 = _inputs(T, dk, dv, seed=seed, B=B, H=H)
+    if wide:  # the long context's decay range and erase gates up to 2
+        la = -np.exp(np.random.default_rng(seed).uniform(-9.0, 3.0, q.shape))
+        b = 2 * b
+    r = np.random.default_rng(seed + 1)
+    return (q, k, v, b, w, la, s0), r.standard_normal(v.shape), r.standard_normal(s0.shape)
+
+
+@pytest.mark.parametrize("regrouped", [True, False], ids=["regrouped", "plain"])
+@pytest.mark.parametrize("C,T,wide", [(16, 150, False), (64, 200, False), (64, 64, True), (64, 200, True)])
+def test_chunk_backward_matches_oracle(C, T, wide, regrouped):
+    """Chunks of 16 and 64 with a ragged last chunk; decays down to -e^3 per token
+    (a chunk's decay far beyond what a midpoint split holds) and erase gates in
+    [0, 2]; dlog_alpha both regrouped (the kernel's form) and plain."""
+    x, dO, dST = grads_case(T, 8, 6, seed=40 + T + C + wide, wide=wide)
+    ref = oracle.bwd(*x, dO, dST)
+    got = wy_backward(*x, dO, dST, C=C, regrouped=regrouped)
+    errs = {n: rel(got[n], ref[n]) for n in GRADS}
+    assert all(e <= 1e-11 for e in errs.values()), errs
+
+
+def test_chunk_backward_without_initial_state_or_final_gradient():
+    x, dO, _ = grads_case(100, 8, 8, seed=77)
+    x = x[:-1] + (None,)
+    ref = oracle.bwd(*x, dO, None)
+    got = wy_backward(*x, dO, None, C=64)
+    assert all(rel(got[n], ref[n]) <= 1e-11 for n in GRADS if n != "dS0")
+    assert rel(got["dS0"], ref["dS0"]) <= 1e-11
+
+
+def _bf16(x):
+    return torch.from_numpy(np.asarray(x, dtype=np.float32)).to(torch.bfloat16).double().numpy()
+
+
+def _collinear_case(eps):
+    d = synth.draw_fwd(1, 200, 2, 128, 128, seed=8300, dtype=torch.bfloat16, s0_sigma=0.05)
+    if eps is not None:
+        d = synth.collinear_keys(d, eps=eps, seed=8301)
+    gen = torch.Generator().manual_seed(8301)
+    dO = torch.randn(1, 200, 2, 128, generator=gen).to(torch.bfloat16).double().numpy()
+    dST = torch.randn(1, 2, 128, 128, generator=gen).double().numpy()
+    x = [d[n].double().numpy() for n in ("q", "k", "v", "b", "w", "log_alpha")] + [d["S0"].double().numpy()]
+    return x, dO, dST
+
+
+def test_pairs_remove_the_T_and_X_share_of_the_error():
+    """Near-collinear keys (noise 0.02) and erase gates near 2: with bf16 T, X and
+    gU in U = T X and dX = T^T gU (and everything else exact), dq's error is about
+    6.6e-3; with T and X as bf16 pairs it falls to about 1.4e-5.  dv and dw keep
+    the share of gU's rounding, which the pairs do not cover (about 9e-3)."""
+    x, dO, dST = _collinear_case(0.02)
+    ref = oracle.bwd(*x, dO, dST)
+    plain = wy_backward(*x, dO, dST, rounding=_bf16, pairs=False)
+    pairs = wy_backward(*x, dO, dST, rounding=_bf16, pairs=True)
+    assert rel(plain["dq"], ref["dq"]) > 3e-3
+    assert rel(pairs["dq"], ref["dq"]) < 1e-4
+    for n in ("dk", "dlog_alpha", "dS0"):
+        assert rel(pairs[n], ref[n]) < 0.5 * rel(plain[n], ref[n]), n
+    assert rel(pairs["dv"], ref["dv"]) > 3e-3
+
+
+def test_random_keys_need_no_pairs():
+    """Random keys: bf16 T, X and gU alone stay far below the bf16 bar of 2e-2."""
+    x, dO, dST = _collinear_case(None)
+    ref = oracle.bwd(*x, dO, dST)
+    plain = wy_backward(*x, dO, dST, rounding=_bf16, pairs=False)
+    assert max(rel(plain[n], ref[n]) for n in GRADS) < 5e-3
