@@ -50,3 +50,17 @@ def test_pair_composition_odd_chunk_count():
     o, s = wy_forward_pairs(q, k, v, b, w, la, S0=s0, C=16)
     assert np.abs(o - o_ref).max() <= 1e-11 * np.abs(o_ref).max()
     assert np.abs(s - s_ref).max() <= 1e-11 * np.abs(s_ref).max()
+
+
+@pytest.mark.parametrize("m,C,T", [(2, 16, 150), (3, 16, 150), (4, 64, 200), (8, 8, 100), (5, 4, 37)])
+def test_group_composition_matches_oracle(m, C, T):
+    """m chunk records composed into one state map per step of the chain (the
+    chain then takes one step per m chunks), each chunk's entry state from its
+    group's by the prefix of the composed product; ragged last groups and
+    chunks."""
+    from wy_model import group_forward
+    q, k, v, b, w, la, s0 = _inputs(T, 8, 6, seed=400 + m * C, B=1, H=2)
+    o_ref, s_ref = oracle.fwd(q, k, v, b, w, la, S0=s0)
+    o, s = group_forward(q, k, v, b, w, la, S0=s0, C=C, m=m)
+    assert np.abs(o - o_ref).max() <= 1e-12 * np.abs(o_ref).max()
+    assert np.abs(s - s_ref).max() <= 1e-12 * np.abs(s_ref).max()

@@ -134,3 +134,42 @@ def wy_forward_pairs(q, k, v, b, w, log_alpha, S0=None, C=64):
                 S = gp[:, None] * S + NGp @ S + Y1p @ Z1 + r2[3] @ Z2
             ST[bi, h] = S
     return o, ST
+
+
+def group_forward(q, k, v, b, w, log_alpha, S0=None, C=64, m=4, rounding=None, store=None, n_rounded=False):
+    """wy_forward with the state carried over groups of m chunks: one step of the
+    serial chain per group, with the group's composed map
+        S_out = Diag(gp) S + NGp S + Np,   A_i = Diag(gc_i) + NG_i,
+        Diag(gp) + NGp = A_m ... A_1,      Np = sum_j (A_m ... A_{j+1}) Y_j Z_j,
+    and each chunk's entry state from the group's by the prefix of that product
+    (state-independent work, off the serial path).  `rounding` (bf16) is applied
+    to every tensor-core operand and `store` (fp32) to every stored accumulator,
+    as the bf16 kernels do; `n_rounded` also rounds Np where it is read.  [B,T,H,d]
+    inputs -> (o, S_T)."""
+    rd = rounding or (lambda x: x)
+    st = store or (lambda x: x)
+    q, k, v, b, w, la = (np.asarray(x, dtype=np.float64) for x in (q, k, v, b, w, log_alpha))
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    o = np.zeros((B, T, H, dv))
+    ST = np.zeros((B, H, dk, dv))
+    for bi in range(B):
+        for h in range(H):
+            S = np.zeros((dk, dv)) if S0 is None else np.array(S0[bi, h], dtype=np.float64)
+            chunks = [slice(t0, min(T, t0 + C)) for t0 in range(0, T, C)]
+            for g0 in range(0, len(chunks), m):
+                Sx = rd(S)
+                gp, NGp, Np = np.ones(dk), np.zeros((dk, dk)), np.zeros((dk, dv))
+                for sl in chunks[g0:g0 + m]:
+                    gc, NG, QS, Y, PT = chunk_record(q[bi, sl, h], k[bi, sl, h], b[bi, sl, h], la[bi, sl, h], C)
+                    gc, NG, QS, Y, PT = st(gc), rd(NG), rd(QS), rd(Y), rd(PT)
+                    Z = rd(w[bi, sl, h] * v[bi, sl, h])
+                    Nr = rd(Np) if n_rounded else Np
+                    Si = st(gp[:, None] * S + rd(NGp) @ Sx + Nr)           # this chunk's entry state
+                    o[bi, sl, h] = rd(QS @ rd(Si) + PT @ Z) if rounding else QS @ Si + PT @ Z
+                    NGp, Np = (st(gc[:, None] * NGp + NG * gp[None, :] + NG @ rd(NGp)),
+                               st(gc[:, None] * Np + NG @ rd(Np) + Y @ Z))
+                    gp = st(gc * gp)
+                S = st(gp[:, None] * S + rd(NGp) @ Sx + (rd(Np) if n_rounded else Np))
+            ST[bi, h] = S
+    return o, ST
