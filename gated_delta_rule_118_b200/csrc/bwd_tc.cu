@@ -16,13 +16,15 @@
 // chunk's map applied to dS' and dO (the adjoint chain, chain_body.cuh ADJ).
 //
 // Steps (one stream, no host synchronisation):
-//   1. prep of every chunk (prep_body.cuh), keeping T and P beside the records;
+//   1. prep of every chunk (prep_body.cuh), keeping T and P beside the records
+//      (and T - bf16(T), with a flag in the record, where T is far from the identity);
 //   2. in one launch, on separate CTAs, the forward chain over every chunk (bf16
 //      images of each chunk's entry state) and the adjoint chain over the chunks
 //      in reverse (images of each chunk's dS', and dS0): the adjoint chain needs
 //      the records and dO, not the forward's states;
-//   4. grad_kernel: one CTA per (chunk, head, batch), all in parallel, the
-//      products above as tcgen05 UMMAs with fp32 accumulators in tensor memory.
+//   3. grad_kernel: one CTA per (chunk, head, batch), all in parallel, the
+//      products above as tcgen05 UMMAs with fp32 accumulators in tensor memory;
+//      a flagged chunk then runs again with T and X as bf16 pairs.
 //
 // In grad_kernel the decays split at the chunk midpoint r like the forward's
 // prep (Ehat = e^{Gamma - Gamma_r} e, Qhat, Khat = e^{Gamma_r - Gamma} k), the

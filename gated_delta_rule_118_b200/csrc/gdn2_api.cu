@@ -221,7 +221,8 @@ extern "C" gdn2_status gdn2_bwd_chunked(const void *q, const void *k, const void
     cudaMemPool_t pool = workspace_pool(dev);
     if (!pool) return GDN2_ERR_CUDA;
     // bf16 inputs with dk = 128 run on the tensor cores (workspace: the prep
-    // records with T and P, and the state and dS' images of every chunk); fp32
+    // records with T and P (and T - bf16(T) where T is far from the identity),
+    // and the state and dS' images of every chunk); fp32
     // inputs and dk = 64 on the fp32 pipes (per chunk: T and P, the state
     // entering it, U, dU and the adjoint at its end)
     const bool tc = dtype == GDN2_BF16 && dk == 128;
