@@ -87,3 +87,22 @@ def test_random_keys_need_no_pairs():
     ref = oracle.bwd(*x, dO, dST)
     plain = wy_backward(*x, dO, dST, rounding=_bf16, pairs=False)
     assert max(rel(plain[n], ref[n]) for n in GRADS) < 5e-3
+
+
+@pytest.mark.parametrize("m,C,T", [(1, 64, 200), (2, 16, 150), (4, 16, 150), (3, 8, 100), (8, 4, 37)])
+def test_grouped_adjoint_chain(m, C, T):
+    """The adjoint chain stepping once per group of m composed chunk maps gives
+    the oracle's dS0, and the gradient leaving every chunk (what each chunk's
+    gradients take): the oracle's dS0 of the sequence's remainder after that
+    chunk, started from the state the oracle reaches there."""
+    from wy_model import group_adjoint
+    x, dO, dST = grads_case(T, 8, 6, seed=500 + m * C)
+    q, k, v, b, w, la, s0 = x
+    ref = oracle.bwd(*x, dO, dST)
+    dS0, dS_out = group_adjoint(q, k, v, b, w, la, dO, dST, C=C, m=m)
+    assert rel(dS0, ref["dS0"]) <= 1e-11
+    for i, t1 in enumerate(range(C, T, C)):
+        _, s_mid = oracle.fwd(*(a[:, :t1] for a in (q, k, v, b, w, la)), S0=s0)
+        tail = oracle.bwd(*(a[:, t1:] for a in (q, k, v, b, w, la)), np.asarray(s_mid), dO[:, t1:], dST)
+        assert rel(dS_out[:, :, i], tail["dS0"]) <= 1e-11, i
+    assert np.array_equal(dS_out[:, :, -1], dST)

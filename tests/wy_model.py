@@ -173,3 +173,46 @@ def group_forward(q, k, v, b, w, log_alpha, S0=None, C=64, m=4, rounding=None, s
                 S = st(gp[:, None] * S + rd(NGp) @ Sx + (rd(Np) if n_rounded else Np))
             ST[bi, h] = S
     return o, ST
+
+
+def group_adjoint(q, k, v, b, w, log_alpha, dO, dS_T=None, C=64, m=4):
+    """The adjoint chain over groups of m chunks: dS, the gradient of
+    sum(o * dO) + sum(S_T * dS_T) with respect to the state entering each chunk,
+    stepping once per group.  With A_i = Diag(gc_i) + NG_i the chunk transition,
+    the gradient entering a group is (A_m ... A_1)^T dS_out + sum_i (A_{i-1} ... A_1)^T
+    QS_i^T dO_i, and the gradient leaving chunk i inside the group (what each
+    chunk's gradients need) follows from dS_out by the suffix products.  The
+    outputs O_i = QS_i S_i + PT_i Z_i only make the dO terms; Z does not enter.
+    [B,T,H,d] inputs -> (dS0 [B,H,dk,dv], dS_out [B,H,nchunks,dk,dv])."""
+    q, k, b, la, dO = (np.asarray(x, dtype=np.float64) for x in (q, k, b, log_alpha, dO))
+    B, T, H, dk = q.shape
+    dv = dO.shape[-1]
+    chunks = [slice(t0, min(T, t0 + C)) for t0 in range(0, T, C)]
+    dS0 = np.zeros((B, H, dk, dv))
+    dS_out = np.zeros((B, H, len(chunks), dk, dv))
+    for bi in range(B):
+        for h in range(H):
+            g = np.zeros((dk, dv)) if dS_T is None else np.array(dS_T[bi, h], dtype=np.float64)
+            for g0 in reversed(range(0, len(chunks), m)):
+                idx = list(range(g0, min(g0 + m, len(chunks))))
+                A, QO = [], []
+                for i in idx:
+                    sl = chunks[i]
+                    gc, NG, QS, _, _ = chunk_record(q[bi, sl, h], k[bi, sl, h], b[bi, sl, h], la[bi, sl, h], C)
+                    A.append(np.diag(gc) + NG)
+                    QO.append(QS.T @ dO[bi, sl, h])
+                # gradient leaving each chunk of the group: suffix products from the group's exit
+                for j, i in enumerate(idx):
+                    d = g.copy()
+                    for l in range(len(idx) - 1, j, -1):   # chunks after i, innermost last
+                        d = A[l].T @ d + QO[l]
+                    dS_out[bi, h, i] = d
+                # gradient entering the group: the composed map and the prefix-weighted dO terms
+                Ag = np.eye(dk)
+                acc = np.zeros((dk, dv))
+                for j in range(len(idx)):
+                    acc += Ag.T @ QO[j]                    # (A_{j-1} ... A_1)^T QS_j^T dO_j
+                    Ag = A[j] @ Ag
+                g = Ag.T @ g + acc
+            dS0[bi, h] = g
+    return dS0, dS_out
