@@ -106,3 +106,43 @@ def test_grouped_adjoint_chain(m, C, T):
         tail = oracle.bwd(*(a[:, t1:] for a in (q, k, v, b, w, la)), np.asarray(s_mid), dO[:, t1:], dST)
         assert rel(dS_out[:, :, i], tail["dS0"]) <= 1e-11, i
     assert np.array_equal(dS_out[:, :, -1], dST)
+
+
+def _f32(x):
+    return np.asarray(x, dtype=np.float32).astype(np.float64)
+
+
+FULL = dict(rounding=_bf16, gram=_bf16, operands=_bf16, images=(_bf16, _f32))
+
+
+def test_midpoint_route_of_the_gradient_products_is_exact():
+    x, dO, dST = _collinear_case(None)
+    ref = oracle.bwd(*x, dO, dST)
+    got = wy_backward(*x, dO, dST, operands=lambda a: a)
+    assert max(rel(got[n], ref[n]) for n in GRADS) <= 1e-12
+
+
+def test_emulated_bf16_backward_random_keys():
+    """Every bf16 rounding point of the tensor-core backward emulated (the two
+    chains' records and images, the prep's Gram, T, X, gU, and the gradient
+    products' operands): within half the bf16 bar on random keys (about 6e-3 at
+    most, db)."""
+    x, dO, dST = _collinear_case(None)
+    ref = oracle.bwd(*x, dO, dST)
+    got = wy_backward(*x, dO, dST, pairs=True, **FULL)
+    errs = {n: rel(got[n], ref[n]) for n in GRADS}
+    assert max(errs.values()) <= 1e-2, errs
+
+
+def test_emulated_bf16_backward_needs_the_pairs_on_collinear_keys():
+    """Key noise 0.02, erase gates near 2: with T and X as pairs every gradient
+    meets the bf16 bar (dq about 1.3e-2); without them dq reaches it (about
+    2.1e-2).  The rest of dq's error is spread over the gradient products'
+    operands (U and dX, the decayed factors, dP and dA: about 8e-3 each alone)."""
+    x, dO, dST = _collinear_case(0.02)
+    ref = oracle.bwd(*x, dO, dST)
+    with_pairs = wy_backward(*x, dO, dST, pairs=True, **FULL)
+    errs = {n: rel(with_pairs[n], ref[n]) for n in GRADS}
+    assert max(errs.values()) <= 2e-2, errs
+    without = wy_backward(*x, dO, dST, pairs=False, **FULL)
+    assert rel(without["dq"], ref["dq"]) >= 1.8e-2

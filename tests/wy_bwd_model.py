@@ -28,10 +28,16 @@ which cancel do so exactly: P's diagonal enters dq and dk but not dGamma;
 Ktil's share K_t = k_t e^{Gamma_C - Gamma_t} dKtil_t adds sum_{t < u} K_t; the
 rest of dGamma_C is rowsum(dS' o e^{Gamma_C} S).
 
-`rounding` (optional) is applied to the operands of U = T X and dX = T^T gU,
-to study what their bf16 rounding costs; pairs=True takes T and X (not gU) as
-bf16 pairs, hi + lo: U = T_hi X_hi + T_hi X_lo + T_lo X_hi and
-dX = T_hi^T gU + T_lo^T gU, the products the kernel adds for flagged chunks.
+The bf16 tensor-core backward's rounding points can be emulated one group at a
+time (each option a rounding function, bf16 in the tests):
+  * `rounding`: the operands of U = T X and dX = T^T gU; pairs=True takes T and
+    X (not gU) as bf16 pairs, hi + lo: U = T_hi X_hi + T_hi X_lo + T_lo X_hi and
+    dX = T_hi^T gU + T_lo^T gU, the products the kernel adds for flagged chunks;
+  * `gram`: A and P from the Gram of bf16 midpoint factors (the prep);
+  * `operands`: U, dX, dP, dA and the midpoint factors where the gradient
+    products take them;
+  * `images` (rounding, store): both chains over bf16 records, and bf16 images
+    of every chunk's entry state and exit gradient.
 """
 import numpy as np
 
@@ -57,16 +63,29 @@ def _mm(a, b, rounding, pair_a, pair_b):
     return r
 
 
-def chunk_bwd(q, k, v, b, w, la, S, dO, dSn, *, regrouped=True, rounding=None, pairs=False):
-    """Gradients of one chunk: returns (dq, dk, dv, db, dw, dla, dS)."""
+def chunk_bwd(q, k, v, b, w, la, S, dO, dSn, *, regrouped=True, rounding=None, pairs=False, gram=None,
+              operands=None):
+    """Gradients of one chunk: returns (dq, dk, dv, db, dw, dla, dS).  `gram`
+    (rounding): A and P from the Gram of bf16 midpoint factors, as the prep forms
+    them on the tensor cores.  `operands` (rounding): the gradient products take
+    bf16 U, dX, dP, dA and midpoint factors Qhat, Khat, Ehat, as the gradient
+    kernel's UMMAs do (dP and dA against the factors; fp32 accumulation); only
+    with regrouped=True and chunks within the midpoint split's range."""
     L = q.shape[0]
     G = np.cumsum(la, axis=0)
     GC = G[-1]
     e = b * k
     D = _pair_decay(G)
     strict = np.tril(np.ones((L, L)), -1)
-    A = np.einsum("td,tsd,sd->ts", e, D, k) * strict
-    P = np.einsum("td,tsd,sd->ts", q, D, k)
+    if gram is None:
+        A = np.einsum("td,tsd,sd->ts", e, D, k) * strict
+        P = np.einsum("td,tsd,sd->ts", q, D, k)
+    else:
+        r = min(32, L)
+        Gr = G[r - 1]
+        Eh, Qh, Kh = (gram(np.exp(G - Gr) * e), gram(np.exp(G - Gr) * q), gram(np.exp(Gr - G) * k))
+        A = (Eh @ Kh.T) * strict
+        P = np.tril(Qh @ Kh.T)
     T = np.linalg.inv(np.eye(L) + A)
     Eb, Qb, Kt = np.exp(G) * e, np.exp(G) * q, np.exp(GC - G) * k
     X = w * v - Eb @ S
@@ -74,18 +93,29 @@ def chunk_bwd(q, k, v, b, w, la, S, dO, dSn, *, regrouped=True, rounding=None, p
     gU = Kt @ dSn + P.T @ dO
     dX = _mm(T.T, gU, rounding, pairs, False)
     dv, dw = dX * w, dX * v
-    dQb, dEb, dKt = dO @ S.T, -dX @ S.T, U @ dSn.T
-    dP = np.tril(dO @ U.T)
-    dA = -(dX @ U.T) * strict
+    rq = operands or (lambda a: a)
+    Uo, dXo = rq(U), rq(dX)
+    dQb, dEb, dKt = dO @ S.T, -dXo @ S.T, Uo @ dSn.T
+    dP = np.tril(dO @ Uo.T)
+    dA = -(dXo @ Uo.T) * strict
     dS = np.exp(GC)[:, None] * dSn + Qb.T @ dO - Eb.T @ dX
     if regrouped:
         dPs = dP * strict                       # P's diagonal: apart
         diag = np.diag(dP)[:, None]
     else:
         dPs, diag = dP, np.zeros((L, 1))
-    dq = np.exp(G) * dQb + np.einsum("ts,tsd,sd->td", dPs, D, k)
-    de = np.exp(G) * dEb + np.einsum("ts,tsd,sd->td", dA, D, k)
-    dkw_pair = np.einsum("ts,tsd,td->sd", dPs, D, q) + np.einsum("ts,tsd,td->sd", dA, D, e)
+    if operands is None:
+        dq = np.exp(G) * dQb + np.einsum("ts,tsd,sd->td", dPs, D, k)
+        de = np.exp(G) * dEb + np.einsum("ts,tsd,sd->td", dA, D, k)
+        dkw_pair = np.einsum("ts,tsd,td->sd", dPs, D, q) + np.einsum("ts,tsd,td->sd", dA, D, e)
+    else:  # through the midpoint split: e^{Gamma_t - Gamma_s} = e^{Gamma_t - Gamma_r} e^{Gamma_r - Gamma_s}
+        r = min(32, L)
+        up, dn = np.exp(G - G[r - 1]), np.exp(G[r - 1] - G)
+        Kh, Qh, Eh = rq(dn * k), rq(up * q), rq(up * e)
+        dPo, dAo = rq(dPs), rq(dA)
+        dq = np.exp(G) * dQb + up * (dPo @ Kh)
+        de = np.exp(G) * dEb + up * (dAo @ Kh)
+        dkw_pair = dn * (dPo.T @ Qh + dAo.T @ Eh)
     Ks = np.exp(GC - G) * dKt * k               # Ktil's share, per token and channel
     if regrouped:
         dG = q * dq + e * de - k * dkw_pair     # without P's diagonal and Ktil's share
@@ -113,9 +143,40 @@ def _chunk_fwd(q, k, v, b, w, la, S):
     return np.exp(G[-1])[:, None] * S + (np.exp(G[-1] - G) * k).T @ U
 
 
-def wy_backward(q, k, v, b, w, log_alpha, S0, dO, dS_T, C=64, **kw):
+def _chains_rounded(x, S0, dO, dS_T, C, rd, st):
+    """The two chains of the bf16 backward: the forward recompute over bf16 chunk
+    records (NG, Y, Z) with the fp32 state read as a bf16 image, and the adjoint
+    chain dS = e^{Gamma_C} dS' + NG^T bf16(dS') + QS^T dO over the same records.
+    Returns the entry states and exit gradients of every chunk (fp32), for one
+    (batch, head) given as [T, d] arrays."""
+    from wy_model import chunk_record
+    q, k, v, b, w, la = x
+    T, dk = q.shape
+    dv = v.shape[1]
+    S = np.zeros((dk, dv)) if S0 is None else S0.copy()
+    recs, entry = [], []
+    for c0 in range(0, T, C):
+        sl = slice(c0, min(c0 + C, T))
+        gc, NG, QS, Y, _ = chunk_record(q[sl], k[sl], b[sl], la[sl], C)
+        gc, NG, QS, Y = st(gc), rd(NG), rd(QS), rd(Y)
+        recs.append((sl, gc, NG, QS))
+        entry.append(S)
+        S = st(gc[:, None] * S + NG @ rd(S) + Y @ rd(w[sl] * v[sl]))
+    dS = np.zeros((dk, dv)) if dS_T is None else dS_T.copy()
+    exit_ = [None] * len(recs)
+    for i in reversed(range(len(recs))):
+        sl, gc, NG, QS = recs[i]
+        exit_[i] = dS
+        dS = st(gc[:, None] * dS + NG.T @ rd(dS) + QS.T @ dO[sl])
+    return entry, exit_, dS
+
+
+def wy_backward(q, k, v, b, w, log_alpha, S0, dO, dS_T, C=64, images=None, **kw):
     """Gradients of sum(o * dO) + sum(S_T * dS_T) over [B,T,H,d] inputs, chunk by
-    chunk in reverse; returns a dict like the oracle's backward."""
+    chunk in reverse; returns a dict like the oracle's backward.  `images`
+    (rounding, store): the chains run over bf16 records and every chunk's
+    gradients take the bf16 images of its entry state and exit gradient, as in
+    the tensor-core backward; dS0 is then the adjoint chain's."""
     B, T, H, dk = q.shape
     dv = v.shape[-1]
     out = {n: np.zeros(q.shape) for n in ("dq", "dk", "db", "dlog_alpha")}
@@ -123,6 +184,19 @@ def wy_backward(q, k, v, b, w, log_alpha, S0, dO, dS_T, C=64, **kw):
     out["dS0"] = np.zeros((B, H, dk, dv))
     for bi in range(B):
         for h in range(H):
+            if images is not None:
+                rd, st = images
+                xs = [a[bi, :, h] for a in (q, k, v, b, w, log_alpha)]
+                entry, exit_, d0 = _chains_rounded(xs, None if S0 is None else S0[bi, h], dO[bi, :, h],
+                                                   None if dS_T is None else dS_T[bi, h], C, rd, st)
+                for i, c0 in enumerate(range(0, T, C)):
+                    sl = slice(c0, min(c0 + C, T))
+                    g = chunk_bwd(*(a[bi, sl, h] for a in (q, k, v, b, w, log_alpha)), rd(entry[i]),
+                                  dO[bi, sl, h], rd(exit_[i]), **kw)
+                    for n, x in zip(("dq", "dk", "dv", "db", "dw", "dlog_alpha"), g[:6]):
+                        out[n][bi, sl, h] = x
+                out["dS0"][bi, h] = d0
+                continue
             S = np.zeros((dk, dv)) if S0 is None else S0[bi, h].copy()
             starts = list(range(0, T, C))
             entry = []
