@@ -146,3 +146,28 @@ def test_emulated_bf16_backward_needs_the_pairs_on_collinear_keys():
     assert max(errs.values()) <= 2e-2, errs
     without = wy_backward(*x, dO, dST, pairs=False, **FULL)
     assert rel(without["dq"], ref["dq"]) >= 1.8e-2
+
+
+def _tf32(x):
+    """Round to the tf32 format (10 explicit mantissa bits), to nearest even."""
+    a = np.ascontiguousarray(np.asarray(x, dtype=np.float32))
+    bits = a.view(np.uint32).astype(np.uint64)
+    bits = (bits + 0x0FFF + ((bits >> 13) & 1)) & ~np.uint64(0x1FFF)
+    return bits.astype(np.uint32).view(np.float32).astype(np.float64)
+
+
+def test_tf32_rounding_helper():
+    # 1 + 2^-10 is a tf32 number; 1 + 2^-11 (a tie) rounds to even (1); 1 + 3 * 2^-11 rounds up to 1 + 2^-9
+    xs = np.array([1 + 2.0 ** -10, 1 + 2.0 ** -11, 1 + 3 * 2.0 ** -11, -3.0])
+    assert np.array_equal(_tf32(xs), [1 + 2.0 ** -10, 1.0, 1 + 2.0 ** -9, -3.0])
+
+
+def test_tf32_second_pass_would_reach_random_key_accuracy():
+    """A flagged chunk's gradient products in tf32 instead of bf16 (the prep's Gram,
+    the chains and the images staying bf16): every gradient within 5e-3 at key
+    noise 0.02, against 1.3e-2 for dq with the bf16 pairs."""
+    x, dO, dST = _collinear_case(0.02)
+    ref = oracle.bwd(*x, dO, dST)
+    got = wy_backward(*x, dO, dST, rounding=_tf32, gram=_bf16, operands=_tf32, images=(_bf16, _f32))
+    errs = {n: rel(got[n], ref[n]) for n in GRADS}
+    assert max(errs.values()) <= 5e-3, errs
